@@ -1,0 +1,324 @@
+"""Plain fp64 CPU oracle for the VSA tile-sparse attention layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product imports this module: only
+the tests, the smoke check and the benchmark's CPU-baseline leg call it.  It
+shares no code with the CUDA path (no tables, helpers or constants); the two
+meet only in the seeded input generator ``tile_sparse_video_b200.inputs``.
+
+Every step is the plain definition, written for a reader to check by eye:
+numpy fp64 arithmetic, a matrix product or a sort from the library where the
+definition calls for one, and no blocking, fusion or reordering.
+
+Sources ("the pages"):
+  [SNACK]  "ComfyUI-Ref2VA-VSA proves a sparse attention gate can be
+           transplanted ..." (SnackOnAI analysis): sections "The Architecture,
+           Unpacked", "The Code, Annotated" (snippets one, two, four) and
+           "It In Action".
+  [WIKI]   "Ref2VA VSA: Sparse Attention Node for H3 Reference-to-Video"
+           (ComfyUI wiki news): section "The two-tier attention patch".
+  [VEDA]   "Veda Sparse Attention" (ComfyUI wiki news, Japanese): the node's
+           input table (generated_sparsity) and section "Performance".
+  [README] The ComfyUI-Ref2VA-VSA README: "Technical Architecture".
+
+Readings taken where the pages are silent are marked "Reading:" below.
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+facts the pages or the mathematics fix (the pages' worked tile counts, an
+independent coordinate formula, a library attention routine, closed forms).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# Step 1: the geometry plan (segment-pure prefix tiles, then video cubes).
+# ---------------------------------------------------------------------------
+
+@dataclass
+class Plan:
+    R: int                  # rows per tile
+    n_tokens: int           # N real tokens (prefix + video)
+    n_prefix_tiles: int     # n_p: tiles [0, n_p) hold the prefix
+    n_tiles: int            # T
+    untile: np.ndarray      # int64[N]: token -> row of the padded tile layout
+    row_src: np.ndarray     # int64[T*R]: row -> token, or -1 for a pad row
+    block_len: np.ndarray   # int64[T]: live (real) rows of each tile
+    tile_seg: np.ndarray    # int64[T]: prefix segment of the tile, -1 = video
+
+    @property
+    def n_padded(self) -> int:
+        return self.n_tiles * self.R
+
+    @property
+    def n_video_tiles(self) -> int:
+        return self.n_tiles - self.n_prefix_tiles
+
+
+def plan(prefix_lens, grid, tile) -> Plan:
+    """Build the token -> padded-row map.
+
+    [SNACK] snippet one: every prefix segment (text, reference image, reference
+    audio, ...) is cut into tiles of R rows, the last tile of a segment may be
+    short, and each segment begins on a fresh tile; the prefix tiles come
+    first.  The generated video is flattened t-major, then h, then w, and cut
+    into cubes visited in loop order t0, h0, w0 ([WIKI] "3D spatio-temporal
+    tiles"; [README] "4x4x4").  Real rows sit at the head of their tile and
+    ``block_len`` counts them, so pad rows never enter a score.
+
+    Reading (edge cubes): a grid extent that is not a multiple of the cube
+    extent gives clipped, partly filled cubes; this is the only rule that
+    reproduces the pages' worked count of 660 video tiles and 43,904 padded
+    rows for a 37 x 24 x 42 grid ([SNACK] "It In Action", step two).
+    Reading (order inside a cube): lexicographic (t, h, w).  The layer's output
+    does not depend on it; it only fixes the permutation table.
+    """
+    tt, th, tw = (int(v) for v in tile)
+    R = tt * th * tw
+    Tg, Hg, Wg = (int(v) for v in grid)
+    prefix_lens = [int(v) for v in prefix_lens]
+    if R <= 0 or min(Tg, Hg, Wg) < 0 or any(v < 0 for v in prefix_lens):
+        raise ValueError("bad geometry")
+    P = sum(prefix_lens)
+    N = P + Tg * Hg * Wg
+    untile = np.full(N, -1, dtype=np.int64)
+    block_len, tile_seg = [], []
+
+    src = 0
+    tile_id = 0
+    for seg, length in enumerate(prefix_lens):
+        left = length
+        while left > 0:
+            n = min(R, left)
+            untile[src:src + n] = tile_id * R + np.arange(n)
+            block_len.append(n)
+            tile_seg.append(seg)
+            src += n
+            left -= n
+            tile_id += 1
+    n_prefix_tiles = tile_id
+
+    for t0 in range(0, Tg, tt):
+        for h0 in range(0, Hg, th):
+            for w0 in range(0, Wg, tw):
+                ts = np.arange(t0, min(t0 + tt, Tg))
+                hs = np.arange(h0, min(h0 + th, Hg))
+                ws = np.arange(w0, min(w0 + tw, Wg))
+                tok = P + (ts[:, None, None] * Hg + hs[None, :, None]) * Wg + ws[None, None, :]
+                tok = tok.reshape(-1)            # lexicographic (t, h, w)
+                untile[tok] = tile_id * R + np.arange(tok.size)
+                block_len.append(tok.size)
+                tile_seg.append(-1)
+                tile_id += 1
+
+    T = tile_id
+    row_src = np.full(T * R, -1, dtype=np.int64)
+    row_src[untile] = np.arange(N)
+
+    # Guard rails as in [SNACK] snippet one: refuse a broken map outright.
+    if N and (untile.min() < 0 or np.unique(untile).size != N):
+        raise RuntimeError("untile map is not injective")
+    if np.count_nonzero(row_src >= 0) != N:
+        raise RuntimeError("a token was placed twice or not at all")
+    return Plan(R=R, n_tokens=N, n_prefix_tiles=n_prefix_tiles, n_tiles=T,
+                untile=untile, row_src=row_src,
+                block_len=np.asarray(block_len, dtype=np.int64),
+                tile_seg=np.asarray(tile_seg, dtype=np.int64))
+
+
+def keep_count(n_video_tiles: int, n_prefix_tiles: int, keep_ratio=None,
+               keep_tiles=None) -> int:
+    """Number k of video key tiles each video query tile keeps.
+
+    Ratio mode: keep_ratio = clamp(1 - sparsity, 0, 1) ([SNACK] snippet two)
+    and k = ceil(keep_ratio * n_video).  Reading: ceiling, with a 1e-9 guard
+    against binary-fraction artefacts; the pages' own figures (165 and 66 of
+    660 tiles at 75 % and 90 %, [SNACK] "It In Action", step three) need it.
+    Integer mode ([VEDA] generated_sparsity = 24): keep exactly that many,
+    capped at n_video.  Reading: k = 0 is only meaningful when prefix sinks
+    exist (else a query tile would have no key at all).
+    """
+    if keep_tiles is not None and keep_tiles >= 0:
+        k = min(int(keep_tiles), n_video_tiles)
+    else:
+        r = min(1.0, max(0.0, float(keep_ratio)))
+        k = min(n_video_tiles, int(math.ceil(r * n_video_tiles - 1e-9)))
+    if k == 0 and n_prefix_tiles == 0 and n_video_tiles > 0:
+        raise ValueError("no key tile left to attend to")
+    return k
+
+
+# ---------------------------------------------------------------------------
+# Step 1 (data movement): permute into / out of the padded tile layout.
+# ---------------------------------------------------------------------------
+
+def permute(x: np.ndarray, p: Plan) -> np.ndarray:
+    """x_t[..., untile[n], :] = x[..., n, :]; pad rows are zero
+    ([SNACK] snippet two: ``x_t = zeros(...); x_t[untile] = x``)."""
+    out = np.zeros(x.shape[:-2] + (p.n_padded, x.shape[-1]), dtype=x.dtype)
+    out[..., p.untile, :] = x
+    return out
+
+
+def unpermute(x_t: np.ndarray, p: Plan) -> np.ndarray:
+    """x[..., n, :] = x_t[..., untile[n], :] (pad rows dropped)."""
+    return x_t[..., p.untile, :]
+
+
+# ---------------------------------------------------------------------------
+# Step 2: coarse attention over mean-pooled tiles.
+# ---------------------------------------------------------------------------
+
+def pool(x_t: np.ndarray, p: Plan) -> np.ndarray:
+    """Per-tile mean over the live rows only.
+
+    Reading: the pages name "coarse tile selection" ([SNACK] "References",
+    the VSA paper) without defining the pooling; the plainest reading is the
+    arithmetic mean of the tile's real tokens (pad rows are excluded,
+    [SNACK] snippet two on block_len).
+    """
+    shp = x_t.shape[:-2]
+    out = np.zeros(shp + (p.n_tiles, x_t.shape[-1]), dtype=np.float64)
+    for t in range(p.n_tiles):
+        rows = x_t[..., t * p.R: t * p.R + p.block_len[t], :].astype(np.float64)
+        out[..., t, :] = rows.sum(axis=-2) / p.block_len[t]
+    return out
+
+
+def coarse_attention(qbar, kbar, vbar, scale):
+    """Coarse attention of every pooled query tile over every pooled key tile.
+
+    s[i, j] = scale * <qbar_i, kbar_j>;  o_coarse_i = sum_j softmax_j(s_i)_j vbar_j.
+    Reading: all T tiles are coarse keys and every query tile (prefix ones
+    too) gets a coarse output; softmax is the two-pass max / sum form.
+    Returns (s [.., T, T], o_coarse [.., T, D]), fp64.
+    """
+    s = scale * (qbar @ np.swapaxes(kbar, -1, -2))
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    prob = e / e.sum(axis=-1, keepdims=True)
+    return s, prob @ vbar
+
+
+# ---------------------------------------------------------------------------
+# Step 3: per-head top-k over the video key tiles.
+# ---------------------------------------------------------------------------
+
+def select_topk(s: np.ndarray, p: Plan, k: int) -> np.ndarray:
+    """For each video query tile i (n_p <= i < T) and head: the k video key
+    tiles with the highest coarse score s[i, j], ties broken towards the lower
+    tile index, returned in ascending tile order ([WIKI] "Sparse video only":
+    top-k applies strictly to the generated-video key tiles; [VEDA]
+    "head-aware top-k").  Prefix key tiles are never candidates: they are
+    always-kept sinks.  Result: int64 [.., n_v, k] of global tile indices.
+    """
+    n_p, T = p.n_prefix_tiles, p.n_tiles
+    lead = s.shape[:-2]
+    out = np.zeros(lead + (T - n_p, k), dtype=np.int64)
+    cand = np.arange(n_p, T)
+    for idx in np.ndindex(*lead):
+        for i in range(n_p, T):
+            scores = s[idx + (i,)][n_p:]
+            # sort by score descending, then by tile index ascending
+            order = np.lexsort((cand, -scores))
+            out[idx + (i - n_p,)] = np.sort(cand[order[:k]])
+    return out
+
+
+def key_tiles(p: Plan, i: int, kept_row) -> np.ndarray:
+    """Key tile set of query tile i: all tiles for a prefix query tile (prefix
+    queries attend densely, [SNACK] snippet two ``sink_q``); the prefix sinks
+    plus the kept video tiles for a video query tile (``sink_blocks``)."""
+    if i < p.n_prefix_tiles:
+        return np.arange(p.n_tiles)
+    return np.concatenate([np.arange(p.n_prefix_tiles), np.asarray(kept_row, dtype=np.int64)])
+
+
+# ---------------------------------------------------------------------------
+# Step 4: block-sparse fine attention.
+# ---------------------------------------------------------------------------
+
+def fine_tile(q_t, k_t, v_t, p: Plan, i: int, tiles, scale):
+    """Softmax attention of the live query rows of tile i over the live key
+    rows of ``tiles`` (one head: q_t, k_t, v_t are [N_pad, D]).
+
+    Returns (o [block_len[i], D], lse [block_len[i]]) in fp64.
+    """
+    rows = np.concatenate([j * p.R + np.arange(p.block_len[j]) for j in tiles])
+    q = q_t[i * p.R: i * p.R + p.block_len[i]].astype(np.float64)
+    kk = k_t[rows].astype(np.float64)
+    vv = v_t[rows].astype(np.float64)
+    s = scale * (q @ kk.T)
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e @ vv) / l, (m + np.log(l))[:, 0]
+
+
+def fine(q_t, k_t, v_t, p: Plan, kept, scale):
+    """o_fine for every live row of every tile (pad rows zero), and its
+    log-sum-exp.  q_t, k_t, v_t: [B, H, N_pad, D]; kept: [B, H, n_v, k]."""
+    B, H = q_t.shape[:2]
+    o = np.zeros(q_t.shape, dtype=np.float64)
+    lse = np.zeros(q_t.shape[:-1], dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for i in range(p.n_tiles):
+                row = kept[b, h, i - p.n_prefix_tiles] if i >= p.n_prefix_tiles else None
+                oi, li = fine_tile(q_t[b, h], k_t[b, h], v_t[b, h], p, i,
+                                   key_tiles(p, i, row), scale)
+                n = p.block_len[i]
+                o[b, h, i * p.R: i * p.R + n] = oi
+                lse[b, h, i * p.R: i * p.R + n] = li
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Step 5: gated combine.
+# ---------------------------------------------------------------------------
+
+def sigmoid(x):
+    """Logistic function 1 / (1 + e^-x), in fp64 (e^-x may overflow to inf,
+    which gives the correct limit 0)."""
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-x))
+
+
+def gate_combine(o_fine, g_t, o_coarse, p: Plan):
+    """out = o_fine + sigmoid(g) * o_coarse[tile(row)] on live rows, 0 on pads.
+
+    g is the bias-free ``to_gate_compress`` projection of the layer input,
+    split into heads ([SNACK] snippet two: ``gate_t`` viewed as
+    [1, S_pad, heads, head_dim] and passed as ``coarse_gate``).  Reading: the
+    gate weighs the coarse branch element-wise through a logistic sigmoid.
+    """
+    tile_of_row = np.repeat(np.arange(p.n_tiles), p.R)
+    live = p.row_src >= 0
+    out = o_fine + sigmoid(g_t.astype(np.float64)) * o_coarse[..., tile_of_row, :]
+    out[..., ~live, :] = 0.0
+    return out
+
+
+# ---------------------------------------------------------------------------
+# The whole layer.
+# ---------------------------------------------------------------------------
+
+def layer(q, k, v, g, p: Plan, kk: int, scale=None, kept=None):
+    """Steps 1-5 on natural-order inputs [B, H, N, D] (any float dtype,
+    converted exactly to fp64).  ``kept`` overrides the top-k selection (used
+    to evaluate the oracle under another legal tie-break).  Returns a dict of
+    every intermediate, all fp64 except the integer selection."""
+    D = q.shape[-1]
+    scale = D ** -0.5 if scale is None else scale
+    q_t, k_t, v_t, g_t = (permute(np.asarray(x, dtype=np.float64), p) for x in (q, k, v, g))
+    qbar, kbar, vbar = pool(q_t, p), pool(k_t, p), pool(v_t, p)
+    s, o_coarse = coarse_attention(qbar, kbar, vbar, scale)
+    sel = select_topk(s, p, kk) if kept is None else np.asarray(kept, dtype=np.int64)
+    o_fine, lse = fine(q_t, k_t, v_t, p, sel, scale)
+    out_t = gate_combine(o_fine, g_t, o_coarse, p)
+    return dict(q_t=q_t, k_t=k_t, v_t=v_t, g_t=g_t, qbar=qbar, kbar=kbar, vbar=vbar,
+                scores=s, o_coarse=o_coarse, topk=sel, o_fine=o_fine, lse=lse,
+                out_t=out_t, out=unpermute(out_t, p))
