@@ -1,0 +1,180 @@
+/*
+ * vsa.h -- C ABI of libvsa, the B200 (sm_100a) VSA tile-sparse attention layer
+ * for reference-to-video.
+ *
+ * The layer works in five steps (pages: "ComfyUI-Ref2VA-VSA proves a sparse
+ * attention gate can be transplanted ..." (SnackOnAI), "The Code, Annotated";
+ * "Ref2VA VSA: Sparse Attention Node for H3 Reference-to-Video" (ComfyUI wiki),
+ * "The two-tier attention patch"; "Veda Sparse Attention" (ComfyUI wiki), the
+ * node input table):
+ *   1. plan + permute: prefix segments into segment-pure tiles, video into
+ *      3-D cubes, tokens scattered into a zero-padded tile layout;
+ *   2. coarse attention over per-tile mean-pooled Q/K/V;
+ *   3. per-head top-k over the video key tiles (prefix tiles are sinks);
+ *   4. block-sparse attention over the kept tiles (prefix queries dense);
+ *   5. out = o_fine + sigmoid(g) * o_coarse, g = the gate projection.
+ *
+ * Conventions for every call below
+ *   - Tensors are row-major with the last dimension contiguous.  "bf16" means
+ *     IEEE bfloat16 stored as uint16.  [B,H,N,D] is the natural token order,
+ *     [B,H,N_pad,D] the padded tile layout (row r = tile r / R, slot r % R).
+ *   - Device pointers are owned by the caller, must be on the plan's device
+ *     and 16-byte aligned; nothing is allocated behind the caller's back
+ *     except the plan's own tables (vsa_plan_create).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); launches are
+ *     asynchronous on it, and the calling thread's current device must be the
+ *     plan's device.
+ *   - Arguments are checked synchronously before any launch; a failed check
+ *     returns an error and launches nothing.  vsa_last_error() then holds a
+ *     message (thread-local).  Faults found by a kernel (a wait that timed out,
+ *     an index out of range) are recorded in the plan's device status word and
+ *     reported by vsa_sync_status().
+ *   - Supported: D in {64, 128}; R = tile_t*tile_h*tile_w in {64, 128}.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VSA_API_VERSION 1
+
+typedef enum vsa_status {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size, wrong device   */
+  VSA_ERR_UNSUPPORTED = 2,     /* D not in {64,128}, R not in {64,128}               */
+  VSA_ERR_PLAN = 3,            /* geometry gives a non-injective or impure plan      */
+  VSA_ERR_WORKSPACE = 4,       /* workspace missing or smaller than required         */
+  VSA_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed                  */
+  VSA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel wait exceeded its bound and bailed out    */
+  VSA_ERR_DEVICE_INDEX = 7     /* a kernel met a kept-tile index outside its range   */
+} vsa_status;
+
+typedef struct vsa_plan_s* vsa_plan;
+
+/* Geometry of one layer call.  prefix_lens[s] is the length of prefix segment s
+ * (text, reference image(s), reference audio, ...) in sequence order; zero-length
+ * segments are allowed and take no tile.  The video follows the prefix, flattened
+ * t-major, then h, then w.  tile_* is the video cube: 4x4x4 = 64 rows (VSA) or
+ * 4x8x4 = 128 rows (Veda's 128-token key tiles); prefix tiles use the same R. */
+typedef struct vsa_geometry {
+  int32_t n_prefix_segments;
+  const int64_t* prefix_lens;        /* host pointer, n_prefix_segments entries */
+  int32_t grid_t, grid_h, grid_w;    /* latent video grid                       */
+  int32_t tile_t, tile_h, tile_w;    /* cube extent                             */
+} vsa_geometry;
+
+/* Step 1 (host).  Build the plan: every prefix segment is cut into R-row tiles
+ * (its last tile may be short) and each segment starts a fresh tile; then the
+ * video is cut into cubes (clipped at the grid's far edges) visited t0, h0, w0,
+ * tokens inside a cube in lexicographic (t, h, w) order at the head of the
+ * tile.  Source: SnackOnAI, "The Code, Annotated", snippet one; clipped cubes
+ * reproduce that page's "It In Action" count (26 + 660 tiles, 43,904 rows).
+ * `device` >= 0 uploads the tables to that CUDA device (synchronously);
+ * device = -1 builds a host-only plan (tables and keep counts only, no
+ * launches).  Returns VSA_ERR_PLAN when the map is not injective, a tile would
+ * mix segments, or the grid is negative.  *out is owned by the caller and
+ * released with vsa_plan_destroy. */
+vsa_status vsa_plan_create(const vsa_geometry* geom, int device, vsa_plan* out);
+
+/* Sizes of a plan: N real tokens, N_pad = T * R padded rows, T tiles, of which
+ * n_p prefix tiles, R rows per tile.  Any output pointer may be NULL. */
+vsa_status vsa_plan_info(vsa_plan plan, int64_t* n_tokens, int64_t* n_padded,
+                         int32_t* n_tiles, int32_t* n_prefix_tiles, int32_t* tile_rows);
+
+/* Host copies of the plan tables (any pointer may be NULL):
+ *   untile[N]     token -> padded row;
+ *   row_src[N_pad] padded row -> token, -1 for a pad row;
+ *   block_len[T]  live rows of each tile (real rows sit at the head);
+ *   tile_seg[T]   prefix segment of the tile, -1 for a video tile. */
+vsa_status vsa_plan_tables(vsa_plan plan, int32_t* untile, int32_t* row_src,
+                           int32_t* block_len, int32_t* tile_seg);
+
+/* Number k of video key tiles each video query tile keeps (step 3).
+ * keep_tiles >= 0: Veda integer mode, k = min(keep_tiles, n_v) ("Veda Sparse
+ * Attention", generated_sparsity = 24 keeps exactly 24 key tiles).
+ * keep_tiles < 0: ratio mode, k = min(n_v, ceil(clamp(keep_ratio,0,1) * n_v - 1e-9))
+ * (SnackOnAI snippet two: keep_ratio = 1 - sparsity; the ceiling reproduces
+ * that page's 165 and 66 of 660 tiles).  k = 0 with no prefix tile is
+ * rejected (VSA_ERR_INVALID_ARG): a query tile would have no key. */
+vsa_status vsa_keep_count(vsa_plan plan, double keep_ratio, int32_t keep_tiles, int32_t* k);
+
+vsa_status vsa_plan_destroy(vsa_plan plan);
+
+/* Bytes of device workspace vsa_coarse_topk needs for B, H, D, k (the pooled
+ * means; vsa_sparse_attn needs none and accepts ws = NULL).  Layout (fp32):
+ * qbar at offset 0, kbar at B*H*T*D*4, vbar at 2*B*H*T*D*4, each [B,H,T,D]. */
+vsa_status vsa_workspace_size(vsa_plan plan, int B, int H, int D, int k, size_t* bytes);
+
+/* Step 1 (device).  x_t[b,h,untile[n],:] = x[b,h,n,:]; pad rows are written 0.
+ * x: bf16 [B,H,N,D]; x_t: bf16 [B,H,N_pad,D].  Source: SnackOnAI snippet two
+ * (x_t = zeros(padded); x_t[untile] = x).  Applied to Q, K, V and the gate. */
+vsa_status vsa_permute(vsa_plan plan, const void* x, void* x_t, int B, int H, int D,
+                       void* stream);
+
+/* Inverse of vsa_permute: x[b,h,n,:] = x_t[b,h,untile[n],:] (pad rows dropped). */
+vsa_status vsa_unpermute(vsa_plan plan, const void* x_t, void* x, int B, int H, int D,
+                         void* stream);
+
+/* Steps 2 and 3.  Pools q_t, k_t, v_t (bf16 [B,H,N_pad,D]) into fp32 per-tile
+ * means over the live rows (into `ws`), then for every query tile i and head:
+ *   s[i,j] = scale * <qbar_i, kbar_j> over all T tiles (fp32),
+ *   o_coarse[b,h,i,:] = sum_j softmax_j(s[i,:]) vbar_j        (fp32 [B,H,T,D]),
+ * and for every video query tile i (n_p <= i < T) the k video key tiles j with
+ * the largest s[i,j], ties to the lower j, written in ascending j order to
+ * topk_idx[b,h,i-n_p,:] (int32 [B,H,n_v,k], global tile indices).  topk_score
+ * (nullable, fp32 [B,H,n_v,k]) receives s[i,j] of each kept tile.  Sources:
+ * the wiki page's "two-tier attention patch" (top-k strictly over generated-
+ * video key tiles, prefix exempt), Veda's head-aware top-k; the mean pooling
+ * and the coarse softmax are this library's reading of "coarse tile
+ * selection" (SnackOnAI, "References", the VSA paper).  k may be 0 (nothing
+ * written to topk_idx) when n_p > 0. */
+vsa_status vsa_coarse_topk(vsa_plan plan, const void* q_t, const void* k_t, const void* v_t,
+                           int B, int H, int D, float scale, int k,
+                           float* o_coarse, int32_t* topk_idx, float* topk_score,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Step 4.  For every live query row of tile i and head: softmax over the live
+ * key rows of S_i, o_fine = sum p v, with S_i = all T tiles when i < n_p
+ * (prefix queries are dense) and S_i = {0..n_p-1} U topk_idx[b,h,i-n_p,:]
+ * otherwise (prefix tiles are always-kept sinks).  Source: SnackOnAI snippet
+ * two (sink_blocks / sink_q = [0, num_prefix_tiles), block_len, scale =
+ * head_dim^-0.5 there; here `scale` is an argument).  o_fine_t: bf16
+ * [B,H,N_pad,D], pad rows written 0.  lse_t (nullable): fp32 [B,H,N_pad],
+ * natural-log log-sum-exp of each live row's scaled scores (0 on pad rows).
+ * topk_idx must hold valid, distinct video tile indices (as vsa_coarse_topk
+ * writes them); a kernel that meets an index outside [n_p, T) skips it and
+ * records VSA_ERR_DEVICE_INDEX.  ws may be NULL. */
+vsa_status vsa_sparse_attn(vsa_plan plan, const void* q_t, const void* k_t, const void* v_t,
+                           const int32_t* topk_idx, int B, int H, int D, int k, float scale,
+                           void* o_fine_t, float* lse_t, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Step 5.  out = o_fine + sigmoid(g) * o_coarse[tile(row)], element-wise over
+ * D, fp32 arithmetic, bf16 round-to-nearest-even store.  o_fine_t and gate_t:
+ * bf16 [B,H,N_pad,D] (the gate is the bias-free to_gate_compress projection of
+ * the layer input, split into heads and permuted like Q: SnackOnAI snippet
+ * two, gate_t passed as coarse_gate); o_coarse: fp32 [B,H,T,D].
+ * out_natural = 0: out is bf16 [B,H,N_pad,D] with pad rows 0;
+ * out_natural = 1: out is bf16 [B,H,N,D] in natural token order (the
+ * unpermute fused in). */
+vsa_status vsa_gate_combine(vsa_plan plan, const void* o_fine_t, const void* gate_t,
+                            const float* o_coarse, void* out, int out_natural,
+                            int B, int H, int D, void* stream);
+
+/* Synchronise `stream`, then read and clear the plan's device status word.
+ * Returns VSA_OK, VSA_ERR_DEVICE_TIMEOUT, VSA_ERR_DEVICE_INDEX or VSA_ERR_CUDA. */
+vsa_status vsa_sync_status(vsa_plan plan, void* stream);
+
+/* Message of the calling thread's last failed call ("" if none). */
+const char* vsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

@@ -1,0 +1,679 @@
+// Block-sparse fine attention over the kept K/V tiles (step 4 of the layer),
+// for sm_100a: TMA tile loads driven by the kept-tile list, tcgen05 MMAs that
+// accumulate in tensor memory (TMEM), and an online softmax.
+//
+// Semantics (SnackOnAI, "The Code, Annotated", snippet two: sink_blocks and
+// sink_q = [0, num_prefix_tiles), block_len): query tile i attends to every
+// tile when i < n_p (prefix queries are dense) and to the n_p prefix sink tiles
+// plus its kept video tiles otherwise; key rows at or past block_len[j] are
+// masked; o = softmax(scale * q k^T) v per live query row.
+//
+// Design (one persistent CTA per SM, static round-robin over work items):
+//   work item = (b*h, query tile i); prefix items (n_p of them per head, each
+//   T key tiles long) come first, then the video items head by head, so the
+//   CTAs share one or two heads' K/V in L2 at any time.
+//   warp 4  (TMA)    loads Q once per item and K_j, V_j per kept tile into an
+//                    NS-stage ring (128-byte swizzled boxes of 64 columns).
+//   warp 5  (MMA)    one elected lane issues S = Q K_j^T (M=128, N=R, K=D) into
+//                    one of two TMEM S buffers, then O += P V_{j-1} (M=128,
+//                    N=D, K=R) once the softmax has written P_{j-1}; every
+//                    completion is signalled with tcgen05.commit on an mbarrier.
+//   warps 0-3        thread t owns query row t = TMEM lane t: it loads its S
+//                    row from TMEM, applies the block_len mask and the running
+//                    max, writes P = exp2(S*scale*log2e - m) as bf16 into a
+//                    swizzled shared-memory tile (the A operand of the PV MMA),
+//                    rescales its O row in TMEM when the max grew, and in the
+//                    epilogue divides by the row sum and stores bf16 rows.
+// TMEM columns: S0 [0,R), S1 [R,2R), O [2R, 2R+D).
+// With R = 64 the MMA still runs with M = 128 (rows 64..127 of the Q box are
+// the next rows of the tensor, or zero past its end); their results are never
+// stored and warps 2-3 skip the softmax work for them.
+//
+// Every mbarrier wait is bounded (kWaitLimitNs of wall time); on expiry the
+// CTA raises an abort flag, records VSA_ERR_DEVICE_TIMEOUT in the status word,
+// drains its own TMA loads and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+constexpr int kBM = 128;                 // MMA M (query rows per item)
+constexpr int kThreadsAttn = 192;        // 4 softmax warps + TMA warp + MMA warp
+constexpr int kWarpTma = 4, kWarpMma = 5;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100
+// descriptor version 1.  Addresses and offsets are in bytes.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) |
+         (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+#define VSA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
+                  "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+#define VSA_P8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), \
+                  "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+#define VSA_I8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
+                  "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
+
+// 32 consecutive fp32 columns of this thread's TMEM lane, then wait for them.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : VSA_R8(0), VSA_R8(8), VSA_R8(16), VSA_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+// Waits for outstanding tcgen05.ld; the registers are tied in so no use of
+// them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : VSA_P8(0), VSA_P8(8), VSA_P8(16), VSA_P8(24)
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      VSA_I8(0), VSA_I8(8), VSA_I8(16), VSA_I8(24)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t u;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(hi), "f"(lo));
+  return u;
+}
+
+// ---------------------------------------------------------------- kernel
+
+struct AttnArgs {
+  const int32_t* topk;        // [BH, n_v, k]
+  const int32_t* block_len;   // [T]
+  uint16_t* out;              // bf16 [BH, N_pad, D]
+  float* lse;                 // [BH, N_pad] or null
+  unsigned int* status;       // device status word
+  int T, n_p, k, n_items;
+  int64_t n_pad;
+  float scale_log2;           // scale * log2(e)
+};
+
+template <int R, int D>
+struct Cfg {
+  static constexpr int BN = R;
+  static constexpr int NS = (R == 128) ? 2 : 4;         // K/V pipeline stages
+  static constexpr int QBYTES = kBM * D * 2;
+  static constexpr int KVBYTES = BN * D * 2;             // one K (or V) tile
+  static constexpr int PBYTES = kBM * BN * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QBYTES;
+  static constexpr int OFF_V = OFF_K + NS * KVBYTES;
+  static constexpr int OFF_P = OFF_V + NS * KVBYTES;
+  static constexpr int OFF_BAR = OFF_P + PBYTES;
+  // barriers: q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], s_empty[2],
+  //           p_full, pv_done, o_empty, drain
+  static constexpr int NBAR = 2 + 2 * NS + 4 + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag
+  static constexpr int OFF_LISTS = OFF_MISC + 16;
+  static constexpr uint32_t TMEM_COLS = (2 * BN + D) <= 256 ? 256u : 512u;
+  static constexpr uint32_t IDESC_QK = idesc_bf16(kBM, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, false, true);
+};
+
+__device__ __forceinline__ void record(unsigned int* status, unsigned int code, unsigned int info) {
+  if (atomicCAS(status, 0u, code) == 0u) atomicExch(status + 1, info);
+}
+
+// Bounded wait; false when the CTA is aborting (flag already set, or this wait
+// timed out, in which case it sets the flag and records the timeout).
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                      unsigned int* status, unsigned int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        record(status, kStatusTimeout, where);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait that ignores the abort flag (used only while draining on abort).
+__device__ __noinline__ void wait_bar_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitLimitNs) return;
+  }
+}
+
+__device__ __forceinline__ void decode_item(int item, int bh_np, int n_p, int n_v, int64_t& bh,
+                                            int& i) {
+  if (item < bh_np) {
+    bh = item / n_p;
+    i = item % n_p;
+  } else {
+    const int v = item - bh_np;
+    bh = v / n_v;
+    i = n_p + v % n_v;
+  }
+}
+
+// Kept video tile x of item (bh, i), clamped into [n_p, T) (recording a fault).
+__device__ __forceinline__ int kept_tile(const AttnArgs& a, int64_t bh, int i, int x) {
+  const int n_v = a.T - a.n_p;
+  int j = __ldg(a.topk + (bh * n_v + (i - a.n_p)) * int64_t(a.k) + x);
+  if (j < a.n_p || j >= a.T) {
+    record(a.status, kStatusBadIndex, unsigned(j));
+    j = a.n_p;
+  }
+  return j;
+}
+
+template <int R, int D>
+__global__ void __launch_bounds__(kThreadsAttn, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using C = Cfg<R, D>;
+  constexpr int BN = C::BN, NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V,
+                 sP = s_base + C::OFF_P;
+  const uint32_t bar0 = s_base + C::OFF_BAR;
+  const uint32_t q_full = bar0, q_empty = bar0 + 8;
+  const uint32_t kv_full = bar0 + 16, kv_empty = kv_full + 8 * NS;
+  const uint32_t s_full = kv_empty + 8 * NS, s_empty = s_full + 16;
+  const uint32_t p_full = s_empty + 16, pv_done = p_full + 8, o_empty = pv_done + 8,
+                 drain = o_empty + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int16_t* s_blen = reinterpret_cast<int16_t*>(smem + C::OFF_LISTS);         // [T]
+  int32_t* s_plist = reinterpret_cast<int32_t*>(smem + C::OFF_LISTS + ((2 * a.T + 15) & ~15));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_v = a.T - a.n_p;
+  const int bh_np = a.n_items - (a.n_items / a.T) * n_v;   // = BH * n_p
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(kv_full + 8 * s, 1);
+      mbar_init(kv_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + 8 * s, 1);
+      mbar_init(s_empty + 8 * s, 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(o_empty, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kWarpTma && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == kWarpMma) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ TMA producer
+    uint32_t g = 0, q_issued = 0;
+    int t = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+      int64_t bh;
+      int i;
+      decode_item(item, bh_np, a.n_p, n_v, bh, i);
+      const bool dense = i < a.n_p;
+      const int nk = dense ? a.T : a.n_p + a.k;
+      if (!dense)
+        for (int x = lane; x < a.k; x += 32) s_plist[x] = kept_tile(a, bh, i, x);
+      __syncwarp();
+      if (lane == 0) {
+        const int64_t row0 = bh * a.n_pad;
+        if (t > 0) ok = wait_bar(q_empty, (t - 1) & 1, abort_flag, a.status, 1);
+        if (ok) {
+          ++q_issued;
+          mbar_expect_tx(q_full, C::QBYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sQ + c * kBM * 128, &tm_q, q_full, c * 64, int(row0 + int64_t(i) * R));
+        }
+        for (int n = 0; n < nk && ok; ++n, ++g) {
+          const uint32_t s = g % NS;
+          if (g >= uint32_t(NS)) {
+            ok = wait_bar(kv_empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, 2);
+            if (!ok) break;
+          }
+          const int j = (dense || n < a.n_p) ? n : s_plist[n - a.n_p];
+          const int row = int(row0 + int64_t(j) * R);
+          mbar_expect_tx(kv_full + 8 * s, 2 * C::KVBYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(sK + s * C::KVBYTES + c * BN * 128, &tm_k, kv_full + 8 * s, c * 64, row);
+            tma_load_2d(sV + s * C::KVBYTES + c * BN * 128, &tm_v, kv_full + 8 * s, c * 64, row);
+          }
+        }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      __syncwarp();
+    }
+    if (lane == 0 && !ok) {
+      // Abort: make sure none of our TMA writes is still in flight.
+      for (uint32_t x = (g > uint32_t(NS) ? g - NS : 0); x < g; ++x)
+        wait_bar_drain(kv_full + 8 * (x % NS), (x / NS) & 1);
+      if (q_issued > 0) wait_bar_drain(q_full, (q_issued - 1) & 1);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t g = 0;
+      int t = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gp, int np_) -> bool {
+        if (np_ == 0 && t > 0)
+          if (!wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) return false;
+        if (!wait_bar(p_full, gp & 1, abort_flag, a.status, 4)) return false;
+        tc_fence_after();
+        const uint32_t sp = gp % NS;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          const uint64_t ad = sdesc_sw128(sP + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sV + sp * C::KVBYTES + ks * 16 * 128, BN * 128, 1024);
+          umma_bf16(tmem + 2 * BN, ad, bd, C::IDESC_PV, (np_ > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(pv_done);
+        umma_commit(kv_empty + 8 * sp);
+        return true;
+      };
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+        int64_t bh;
+        int i;
+        decode_item(item, bh_np, a.n_p, n_v, bh, i);
+        const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
+        if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
+        tc_fence_after();
+        for (int n = 0; n < nk; ++n, ++g) {
+          const uint32_t s = g % NS, sb = g & 1;
+          if (!wait_bar(kv_full + 8 * s, (g / NS) & 1, abort_flag, a.status, 6)) { ok = false; break; }
+          if (g >= 2 && !wait_bar(s_empty + 8 * sb, ((g >> 1) - 1) & 1, abort_flag, a.status, 7)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ad = sdesc_sw128(sQ + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
+            const uint64_t bd =
+                sdesc_sw128(sK + s * C::KVBYTES + (ks / 4) * BN * 128 + (ks % 4) * 32, 16, 1024);
+            umma_bf16(tmem + sb * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full + 8 * sb);
+          if (n == nk - 1) umma_commit(q_empty);
+          if (n > 0 && !issue_pv(g - 1, n - 1)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (!issue_pv(g - 1, nk - 1)) { ok = false; break; }
+      }
+      // Drain: wait until every MMA issued above has completed.
+      umma_commit(drain);
+      wait_bar_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const bool rows_active = (R == 128) || (warp < 2);
+    const int row = warp * 32 + lane;                    // = TMEM lane
+    const uint32_t t_lane = tmem + (uint32_t(warp * 32) << 16);
+    uint32_t g = 0;
+    int t = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+      int64_t bh;
+      int i;
+      decode_item(item, bh_np, a.n_p, n_v, bh, i);
+      const bool dense = i < a.n_p;
+      const int nk = dense ? a.T : a.n_p + a.k;
+      // Group barrier of the 128 softmax threads.  A warp that sees the abort
+      // flag leaves instead: the others then also see it before they could
+      // block here (they wait on the same mbarrier phases first).
+      if (*abort_flag) { ok = false; break; }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int x = threadIdx.x; x < nk; x += 128) {
+        const int j = (dense || x < a.n_p) ? x : kept_tile(a, bh, i, x - a.n_p);
+        s_blen[x] = int16_t(__ldg(a.block_len + j));
+      }
+      if (*abort_flag) { ok = false; break; }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int q_live = __ldg(a.block_len + i);
+
+      float m = -INFINITY, l = 0.f;
+      for (int n = 0; n < nk; ++n, ++g) {
+        const uint32_t sb = g & 1;
+        if (!wait_bar(s_full + 8 * sb, (g >> 1) & 1, abort_flag, a.status, 8)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[BN / 32][32];
+        if (rows_active) {
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + sb * BN + 32 * c, r[c]);
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) tmem_wait_ld(r[c]);
+        }
+        tc_fence_before();
+        mbar_arrive(s_empty + 8 * sb);
+
+        float alpha = 1.f;
+        if (rows_active) {
+          const int bl = s_blen[n];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              float x = __uint_as_float(r[c][e]) * a.scale_log2;
+              if (bl < BN && 32 * c + e >= bl) x = -INFINITY;
+              r[c][e] = __float_as_uint(x);
+              mx = fmaxf(mx, x);
+            }
+          const float m_new = fmaxf(m, mx);
+          alpha = ex2(m - m_new);
+          float sum = 0.f;
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float p = ex2(__uint_as_float(r[c][e]) - m_new);
+              sum += p;
+              r[c][e] = __float_as_uint(p);
+            }
+          l = l * alpha + sum;
+          m = m_new;
+        }
+        // PV of the previous tile must be done before P is overwritten and O is touched.
+        if (g > 0 && !wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 9)) { ok = false; break; }
+        tc_fence_after();
+        if (rows_active) {
+#pragma unroll
+          for (int c8 = 0; c8 < BN / 8; ++c8) {
+            const int c = c8 / 4, e = (c8 % 4) * 8;
+            const uint32_t w0 = pack_bf16(__uint_as_float(r[c][e + 0]), __uint_as_float(r[c][e + 1]));
+            const uint32_t w1 = pack_bf16(__uint_as_float(r[c][e + 2]), __uint_as_float(r[c][e + 3]));
+            const uint32_t w2 = pack_bf16(__uint_as_float(r[c][e + 4]), __uint_as_float(r[c][e + 5]));
+            const uint32_t w3 = pack_bf16(__uint_as_float(r[c][e + 6]), __uint_as_float(r[c][e + 7]));
+            const uint32_t addr =
+                sP + (c8 / 8) * kBM * 128 + row * 128 + ((uint32_t(c8 % 8) ^ uint32_t(row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w0), "r"(w1),
+                         "r"(w2), "r"(w3)
+                         : "memory");
+          }
+          if (n > 0 && alpha < 1.f) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(t_lane + 2 * BN + 32 * c, o);
+              tmem_wait_ld(o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(t_lane + 2 * BN + 32 * c, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      // ---- epilogue
+      if (!wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 10)) { ok = false; break; }
+      tc_fence_after();
+      if (rows_active) {
+        const bool live = row < q_live;
+        const float inv_l = live ? 1.0f / l : 0.f;
+        uint16_t* orow = a.out + (bh * a.n_pad + int64_t(i) * R + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + 2 * BN + 32 * c, o);
+          tmem_wait_ld(o);
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+            v.y = pack_bf16(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+            v.z = pack_bf16(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+            v.w = pack_bf16(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+            dst[q] = v;
+          }
+        }
+        if (a.lse != nullptr)
+          a.lse[bh * a.n_pad + int64_t(i) * R + row] = live ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
+      }
+      tc_fence_before();
+      mbar_arrive(o_empty);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a [rows, D] bf16 matrix, box = 64 columns x box_rows rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+  const cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R, int D>
+size_t attn_smem_bytes(int T) {
+  using C = Cfg<R, D>;
+  return size_t(C::OFF_LISTS) + size_t((2 * T + 15) & ~15) + size_t(4) * T + 1024;
+}
+
+template <int R, int D>
+vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, const void* v_t,
+                     const int32_t* topk_idx, int64_t bh, int k, float scale, void* o_fine_t,
+                     float* lse_t, cudaStream_t stream) {
+  const size_t smem = attn_smem_bytes<R, D>(p->n_tiles);
+  if (smem > 227 * 1024)
+    return fail(VSA_ERR_UNSUPPORTED, "too many tiles for the sparse attention kernel's lists");
+  const int64_t rows = bh * p->n_padded;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q_t, rows, D, kBM) || !make_map(&mk, k_t, rows, D, R) ||
+      !make_map(&mv, v_t, rows, D, R))
+    return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<R, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return fail(VSA_ERR_CUDA, cudaGetErrorString(e));
+  AttnArgs a;
+  a.topk = topk_idx;
+  a.block_len = p->d_block_len;
+  a.out = static_cast<uint16_t*>(o_fine_t);
+  a.lse = lse_t;
+  a.status = p->d_status;
+  a.T = p->n_tiles;
+  a.n_p = p->n_prefix_tiles;
+  a.k = k;
+  a.n_pad = p->n_padded;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const int64_t items = bh * p->n_tiles;
+  if (items >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "too many work items");
+  a.n_items = int(items);
+  const int grid = int(std::min<int64_t>(items, p->num_sms > 0 ? p->num_sms : 148));
+  sparse_attn_kernel<R, D><<<grid, kThreadsAttn, smem, stream>>>(mq, mk, mv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(VSA_ERR_CUDA, std::string("sparse_attn launch: ") + cudaGetErrorString(e));
+  return VSA_OK;
+}
+
+}  // namespace
+
+vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* k_t,
+                              const void* v_t, const int32_t* topk_idx, int64_t bh, int D, int k,
+                              float scale, void* o_fine_t, float* lse_t, cudaStream_t stream) {
+  if (p->n_padded * bh >= (int64_t(1) << 31))
+    return fail(VSA_ERR_UNSUPPORTED, "B*H*N_pad rows exceed the 32-bit TMA coordinate range");
+  if (p->R == 128) {
+    if (D == 128) return launch_rd<128, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
+    return launch_rd<128, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
+  }
+  if (D == 128) return launch_rd<64, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
+  return launch_rd<64, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
+}
+
+}  // namespace vsa

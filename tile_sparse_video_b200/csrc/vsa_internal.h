@@ -1,0 +1,64 @@
+// Internal declarations shared by the libvsa translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/vsa.h"
+
+struct vsa_plan_s {
+  // geometry
+  int R = 0;                 // rows per tile
+  int64_t n_tokens = 0;      // N
+  int64_t n_padded = 0;      // N_pad = T * R
+  int n_tiles = 0;           // T
+  int n_prefix_tiles = 0;    // n_p
+  // host tables
+  std::vector<int32_t> untile, row_src, block_len, tile_seg;
+  // device side (device < 0: host-only plan)
+  int device = -1;
+  int num_sms = 0;
+  int32_t* d_untile = nullptr;
+  int32_t* d_row_src = nullptr;
+  int32_t* d_block_len = nullptr;
+  unsigned int* d_status = nullptr;   // device status word (0 = ok)
+};
+
+namespace vsa {
+
+// Thread-local last error message.
+void set_error(const std::string& msg);
+vsa_status fail(vsa_status code, const std::string& msg);
+
+// Host planner (plan.cpp).  Fills tables and sizes; returns VSA_OK or VSA_ERR_PLAN.
+vsa_status build_plan(const vsa_geometry& g, vsa_plan_s* p);
+
+// Kernel launchers (each .cu file); all asynchronous on `stream`.
+cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, const int32_t* map,
+                               int64_t bh, int64_t src_rows, int64_t dst_rows, int D,
+                               int num_sms, cudaStream_t stream);
+cudaError_t launch_pool(const uint16_t* q_t, const uint16_t* k_t, const uint16_t* v_t,
+                        const int32_t* block_len, float* qbar, float* kbar, float* vbar,
+                        int64_t bh, int T, int R, int D, int num_sms, cudaStream_t stream);
+cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float* vbar,
+                               int64_t bh, int T, int n_p, int D, float scale, int k,
+                               float* o_coarse, int32_t* topk_idx, float* topk_score,
+                               cudaStream_t stream);
+cudaError_t launch_gate_combine(const uint16_t* o_fine_t, const uint16_t* gate_t,
+                                const float* o_coarse, uint16_t* out, int out_natural,
+                                const int32_t* row_src, const int32_t* untile,
+                                int64_t bh, int64_t n_tokens, int64_t n_padded, int R, int T,
+                                int D, int num_sms, cudaStream_t stream);
+vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* k_t,
+                              const void* v_t, const int32_t* topk_idx, int64_t bh, int D,
+                              int k, float scale, void* o_fine_t, float* lse_t,
+                              cudaStream_t stream);
+
+// Device status codes written by kernels into vsa_plan_s::d_status.
+enum : unsigned int { kStatusOk = 0, kStatusTimeout = 1, kStatusBadIndex = 2 };
+
+}  // namespace vsa

@@ -1,0 +1,283 @@
+"""Thin Python binding of libvsa (ctypes).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  There is no
+fallback: if ``libvsa.so`` is missing, every call raises.
+
+The names mirror the C ABI in ``include/vsa.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvsa.so")
+_lib = None
+
+VSA_OK = 0
+STATUS_NAMES = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_PLAN",
+                4: "VSA_ERR_WORKSPACE", 5: "VSA_ERR_CUDA", 6: "VSA_ERR_DEVICE_TIMEOUT",
+                7: "VSA_ERR_DEVICE_INDEX"}
+
+# exported C symbols (kept in step with include/vsa.h)
+EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_count",
+           "vsa_plan_destroy", "vsa_workspace_size", "vsa_permute", "vsa_unpermute",
+           "vsa_coarse_topk", "vsa_sparse_attn", "vsa_gate_combine", "vsa_sync_status",
+           "vsa_last_error")
+
+
+class VsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class _Geometry(ctypes.Structure):
+    _fields_ = [("n_prefix_segments", ctypes.c_int32), ("prefix_lens", ctypes.POINTER(ctypes.c_int64)),
+                ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("tile_t", ctypes.c_int32), ("tile_h", ctypes.c_int32), ("tile_w", ctypes.c_int32)]
+
+
+def lib():
+    """Load libvsa.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m tile_sparse_video_b200.build` (no fallback exists)")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, I32, I64, F, D, Z, V = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int32, ctypes.c_int64,
+                                      ctypes.c_float, ctypes.c_double, ctypes.c_size_t, ctypes.c_void_p)
+        sig = {
+            "vsa_plan_create": [ctypes.POINTER(_Geometry), I, ctypes.POINTER(P)],
+            "vsa_plan_info": [P, ctypes.POINTER(I64), ctypes.POINTER(I64), ctypes.POINTER(I32),
+                              ctypes.POINTER(I32), ctypes.POINTER(I32)],
+            "vsa_plan_tables": [P, V, V, V, V],
+            "vsa_keep_count": [P, D, I32, ctypes.POINTER(I32)],
+            "vsa_plan_destroy": [P],
+            "vsa_workspace_size": [P, I, I, I, I, ctypes.POINTER(Z)],
+            "vsa_permute": [P, V, V, I, I, I, V],
+            "vsa_unpermute": [P, V, V, I, I, I, V],
+            "vsa_coarse_topk": [P, V, V, V, I, I, I, F, I, V, V, V, V, Z, V],
+            "vsa_sparse_attn": [P, V, V, V, V, I, I, I, I, F, V, V, V, Z, V],
+            "vsa_gate_combine": [P, V, V, V, V, I, I, I, I, V],
+            "vsa_sync_status": [P, V],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.vsa_last_error.argtypes = []
+        L.vsa_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != VSA_OK:
+        raise VsaError(status, lib().vsa_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class Plan:
+    """Owner of a libvsa plan (step 1 tables).  ``device=-1`` builds a host-only
+    plan (tables and keep counts, no launches)."""
+
+    def __init__(self, prefix_lens: Sequence[int], grid: Sequence[int], tile: Sequence[int],
+                 device: Optional[int] = None):
+        L = lib()
+        if device is None:
+            device = torch.cuda.current_device()
+        self.prefix_lens = tuple(int(x) for x in prefix_lens)
+        self.grid, self.tile = tuple(int(x) for x in grid), tuple(int(x) for x in tile)
+        self._lens = (ctypes.c_int64 * max(1, len(self.prefix_lens)))(*self.prefix_lens)
+        geo = _Geometry(len(self.prefix_lens), ctypes.cast(self._lens, ctypes.POINTER(ctypes.c_int64)),
+                        *self.grid, *self.tile)
+        h = ctypes.c_void_p()
+        _check(L.vsa_plan_create(ctypes.byref(geo), int(device), ctypes.byref(h)))
+        self._h = h
+        self.device = int(device)
+        n_tok, n_pad = ctypes.c_int64(), ctypes.c_int64()
+        T, n_p, R = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(L.vsa_plan_info(h, ctypes.byref(n_tok), ctypes.byref(n_pad), ctypes.byref(T),
+                               ctypes.byref(n_p), ctypes.byref(R)))
+        self.n_tokens, self.n_padded = n_tok.value, n_pad.value
+        self.n_tiles, self.n_prefix_tiles, self.tile_rows = T.value, n_p.value, R.value
+        self.n_video_tiles = self.n_tiles - self.n_prefix_tiles
+
+    @property
+    def handle(self):
+        return self._h
+
+    def tables(self) -> dict:
+        out = {"untile": np.empty(self.n_tokens, np.int32), "row_src": np.empty(self.n_padded, np.int32),
+               "block_len": np.empty(self.n_tiles, np.int32), "tile_seg": np.empty(self.n_tiles, np.int32)}
+        _check(lib().vsa_plan_tables(self._h, *(ctypes.c_void_p(a.ctypes.data) for a in out.values())))
+        return out
+
+    def keep_count(self, keep_ratio: Optional[float] = None, keep_tiles: Optional[int] = None) -> int:
+        k = ctypes.c_int32()
+        _check(lib().vsa_keep_count(self._h, float(keep_ratio if keep_ratio is not None else 0.0),
+                                    int(keep_tiles) if keep_tiles is not None else -1, ctypes.byref(k)))
+        return k.value
+
+    def workspace_size(self, B: int, H: int, D: int, k: int) -> int:
+        n = ctypes.c_size_t()
+        _check(lib().vsa_workspace_size(self._h, B, H, D, k, ctypes.byref(n)))
+        return n.value
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().vsa_plan_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def vsa_plan(prefix_lens, grid, tile, device=None) -> Plan:
+    return Plan(prefix_lens, grid, tile, device)
+
+
+def vsa_permute(plan: Plan, x: torch.Tensor, x_t: Optional[torch.Tensor] = None, stream=None):
+    B, H, N, D = x.shape
+    _need(x, "x", torch.bfloat16, (B, H, plan.n_tokens, D))
+    if x_t is None:
+        x_t = torch.empty(B, H, plan.n_padded, D, dtype=torch.bfloat16, device=x.device)
+    _need(x_t, "x_t", torch.bfloat16, (B, H, plan.n_padded, D))
+    _check(lib().vsa_permute(plan.handle, _ptr(x), _ptr(x_t), B, H, D, _stream(stream)))
+    return x_t
+
+
+def vsa_unpermute(plan: Plan, x_t: torch.Tensor, x: Optional[torch.Tensor] = None, stream=None):
+    B, H, _, D = x_t.shape
+    _need(x_t, "x_t", torch.bfloat16, (B, H, plan.n_padded, D))
+    if x is None:
+        x = torch.empty(B, H, plan.n_tokens, D, dtype=torch.bfloat16, device=x_t.device)
+    _need(x, "x", torch.bfloat16, (B, H, plan.n_tokens, D))
+    _check(lib().vsa_unpermute(plan.handle, _ptr(x_t), _ptr(x), B, H, D, _stream(stream)))
+    return x
+
+
+def vsa_coarse_topk(plan: Plan, q_t, k_t, v_t, k: int, scale: Optional[float] = None, ws=None,
+                    o_coarse=None, topk_idx=None, want_scores: bool = False, stream=None):
+    """Returns (o_coarse fp32 [B,H,T,D], topk_idx int32 [B,H,n_v,k], scores or None, ws)."""
+    B, H, _, D = q_t.shape
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("v_t", v_t)):
+        _need(t, name, torch.bfloat16, (B, H, plan.n_padded, D))
+    dev = q_t.device
+    scale = D ** -0.5 if scale is None else float(scale)
+    T, n_v = plan.n_tiles, plan.n_video_tiles
+    if o_coarse is None:
+        o_coarse = torch.empty(B, H, T, D, dtype=torch.float32, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty(B, H, n_v, max(k, 0), dtype=torch.int32, device=dev)
+    scores = torch.empty(B, H, n_v, max(k, 0), dtype=torch.float32, device=dev) if want_scores else None
+    need = plan.workspace_size(B, H, D, k)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().vsa_coarse_topk(plan.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), B, H, D, scale, k,
+                                 _ptr(o_coarse), _ptr(topk_idx) if topk_idx.numel() else None,
+                                 _ptr(scores) if scores is not None and scores.numel() else None,
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return o_coarse, topk_idx, scores, ws
+
+
+def vsa_sparse_attn(plan: Plan, q_t, k_t, v_t, topk_idx, k: int, scale: Optional[float] = None,
+                    out=None, want_lse: bool = False, stream=None):
+    """Returns (o_fine_t bf16 [B,H,N_pad,D], lse fp32 [B,H,N_pad] or None)."""
+    B, H, _, D = q_t.shape
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("v_t", v_t)):
+        _need(t, name, torch.bfloat16, (B, H, plan.n_padded, D))
+    _need(topk_idx, "topk_idx", torch.int32, (B, H, plan.n_video_tiles, max(k, 0)))
+    scale = D ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q_t)
+    lse = torch.empty(B, H, plan.n_padded, dtype=torch.float32, device=q_t.device) if want_lse else None
+    _check(lib().vsa_sparse_attn(plan.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t),
+                                 _ptr(topk_idx) if topk_idx.numel() else None, B, H, D, k, scale,
+                                 _ptr(out), _ptr(lse), None, 0, _stream(stream)))
+    return out, lse
+
+
+def vsa_gate_combine(plan: Plan, o_fine_t, gate_t, o_coarse, natural: bool = True, out=None,
+                     stream=None):
+    B, H, _, D = o_fine_t.shape
+    _need(o_fine_t, "o_fine_t", torch.bfloat16, (B, H, plan.n_padded, D))
+    _need(gate_t, "gate_t", torch.bfloat16, (B, H, plan.n_padded, D))
+    _need(o_coarse, "o_coarse", torch.float32, (B, H, plan.n_tiles, D))
+    rows = plan.n_tokens if natural else plan.n_padded
+    if out is None:
+        out = torch.empty(B, H, rows, D, dtype=torch.bfloat16, device=o_fine_t.device)
+    _need(out, "out", torch.bfloat16, (B, H, rows, D))
+    _check(lib().vsa_gate_combine(plan.handle, _ptr(o_fine_t), _ptr(gate_t), _ptr(o_coarse), _ptr(out),
+                                  1 if natural else 0, B, H, D, _stream(stream)))
+    return out
+
+
+def vsa_sync_status(plan: Plan, stream=None):
+    _check(lib().vsa_sync_status(plan.handle, _stream(stream)))
+
+
+class Layer:
+    """The five steps in sequence on caller-visible buffers, all launches on
+    one stream: permute Q, K, V, G; coarse + top-k; sparse attention; gated
+    combine writing natural order.  Buffers are allocated once (``reserve``)
+    and reused by every call."""
+
+    def __init__(self, plan: Plan, B: int, H: int, D: int, k: int, scale: Optional[float] = None,
+                 device=None):
+        self.plan, self.B, self.H, self.D, self.k = plan, B, H, D, k
+        self.scale = D ** -0.5 if scale is None else float(scale)
+        dev = torch.device("cuda", plan.device) if device is None else torch.device(device)
+        tiled = (B, H, plan.n_padded, D)
+        self.q_t, self.k_t, self.v_t, self.g_t = (torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+                                                  for _ in range(4))
+        self.o_fine_t = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+        self.o_coarse = torch.empty(B, H, plan.n_tiles, D, dtype=torch.float32, device=dev)
+        self.topk_idx = torch.empty(B, H, plan.n_video_tiles, max(k, 0), dtype=torch.int32, device=dev)
+        self.ws = torch.empty(max(plan.workspace_size(B, H, D, k), 16), dtype=torch.uint8, device=dev)
+        self.out = torch.empty(B, H, plan.n_tokens, D, dtype=torch.bfloat16, device=dev)
+
+    def __call__(self, q, k, v, g, stream=None):
+        p = self.plan
+        vsa_permute(p, q, self.q_t, stream)
+        vsa_permute(p, k, self.k_t, stream)
+        vsa_permute(p, v, self.v_t, stream)
+        vsa_permute(p, g, self.g_t, stream)
+        vsa_coarse_topk(p, self.q_t, self.k_t, self.v_t, self.k, self.scale, ws=self.ws,
+                        o_coarse=self.o_coarse, topk_idx=self.topk_idx, stream=stream)
+        vsa_sparse_attn(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, self.scale,
+                        out=self.o_fine_t, stream=stream)
+        vsa_gate_combine(p, self.o_fine_t, self.g_t, self.o_coarse, natural=True, out=self.out,
+                         stream=stream)
+        return self.out
