@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Benchmark of the VSA tile-sparse attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one whole layer (permute Q/K/V/G, pool + coarse attention + top-k,
+block-sparse attention, gated combine into natural order) on the 104,704-token
+Veda workload: 42 heads x 128, 128-token key tiles (4x8x4), 2 prefix tiles and
+816 video tiles, 90 % sparsity (82 kept video tiles per query tile).
+
+Prints one JSON line (rank 0).  ``value`` is milliseconds per layer over the
+whole job (the timed span, max over ranks, divided by the layers all ranks
+ran), with inputs resident in HBM; ``e2e`` is the same metric through the
+public API with pinned host buffers copied in and the output copied back
+inside the timed region.  Every input tensor (1.1 GB) is larger than L2, so
+each step streams from HBM.  For N > 1 every rank runs its own replica of the
+layer (the layer has no cross-GPU exchange), i.e. weak scaling.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (one head, sampled query tiles),
+extrapolated to ms per layer.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tile_sparse_video_b200.inputs import VEDA_104K, Workload, make_inputs  # noqa: E402
+
+METRIC = "ms/layer & kept-FLOP TFLOP/s (% bf16 peak) at 104k tokens, 90% tile sparsity"
+UNIT = "ms/layer"
+
+
+# ----------------------------------------------------------------- accounting
+
+def geometry_counts(w: Workload, n_p: int, T: int, k: int) -> dict:
+    """Algorithmic work of one layer (only what the method must do)."""
+    R, D, BH = w.tile_rows, w.D, w.B * w.H
+    n_v = T - n_p
+    N, N_pad = w.n_tokens, T * R
+    pairs = n_v * (n_p + k) + n_p * T
+    return dict(
+        pairs=pairs,
+        pair_fraction=pairs / T ** 2,
+        kept_flop=4.0 * D * R * R * pairs * BH,            # QK^T and PV over kept tile pairs
+        dense_flop=4.0 * N * N * D * BH,
+        # bytes: read N real rows, write N_pad padded rows, four tensors
+        permute_bytes=4.0 * BH * (N + N_pad) * D * 2,
+        # pool reads the live rows of Q, K, V
+        pool_bytes=3.0 * BH * N * D * 2,
+        # combine (natural order) reads o_fine and g rows of live tokens, writes the output
+        combine_bytes=3.0 * BH * N * D * 2,
+        # attention: Q, K, V read once and O written once
+        attn_bytes=4.0 * BH * N_pad * D * 2,
+    )
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- oracle sample
+
+def oracle_sample(w: Workload, inp: dict, n_video_tiles: int = 256, n_prefix_tiles: int = 2) -> dict:
+    """Time the fp64 oracle on one head of the workload (pool, coarse, top-k
+    over the whole head; fine attention and combine on sampled query tiles)
+    and extrapolate linearly to one whole layer (cost is linear in heads and
+    in query tiles of each kind)."""
+    import oracle as O
+    p = O.plan(w.prefix, w.grid, w.tile)
+    keep = O.keep_count(p.n_video_tiles, p.n_prefix_tiles, keep_ratio=w.keep_ratio,
+                        keep_tiles=w.keep_tiles)
+    scale = w.D ** -0.5
+    x = {n: inp[n][0, 0].to(torch.float64).numpy() for n in "qkvg"}
+    t0 = time.perf_counter()
+    q_t, k_t, v_t, g_t = (O.permute(x[n], p) for n in "qkvg")
+    qb, kb, vb = O.pool(q_t, p), O.pool(k_t, p), O.pool(v_t, p)
+    s, oc = O.coarse_attention(qb, kb, vb, scale)
+    sel = O.select_topk(s[None], p, keep)[0]
+    t_head = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    vids = p.n_prefix_tiles + rng.choice(p.n_video_tiles, min(n_video_tiles, p.n_video_tiles), replace=False)
+    t0 = time.perf_counter()
+    for i in vids:
+        O.fine_tile(q_t, k_t, v_t, p, int(i), O.key_tiles(p, int(i), sel[int(i) - p.n_prefix_tiles]), scale)
+    t_video = (time.perf_counter() - t0) / max(1, len(vids))
+    t_prefix = 0.0
+    if p.n_prefix_tiles:
+        t0 = time.perf_counter()
+        for i in range(min(n_prefix_tiles, p.n_prefix_tiles)):
+            O.fine_tile(q_t, k_t, v_t, p, i, O.key_tiles(p, i, None), scale)
+        t_prefix = (time.perf_counter() - t0) / min(n_prefix_tiles, p.n_prefix_tiles)
+    t0 = time.perf_counter()
+    O.unpermute(O.gate_combine(q_t[None], g_t[None], oc[None], p), p)
+    t_comb = time.perf_counter() - t0
+    per_head = t_head + p.n_video_tiles * t_video + p.n_prefix_tiles * t_prefix + t_comb
+    ms = per_head * w.B * w.H * 1e3
+    return {"value": ms, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": (f"fp64 numpy oracle on head 0 of {w.name}: permute+pool+coarse+top-k of the "
+                       f"whole head, fine attention of {len(vids)} video and "
+                       f"{min(n_prefix_tiles, p.n_prefix_tiles)} prefix query tiles, combine; "
+                       f"extrapolated linearly to {w.B * w.H} heads x {p.n_tiles} query tiles")}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> None:
+    from tile_sparse_video_b200 import vsa
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = VEDA_104K
+    inp = make_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile, device=local_rank)
+    k = plan.keep_count(keep_ratio=w.keep_ratio, keep_tiles=w.keep_tiles)
+    acct = geometry_counts(w, plan.n_prefix_tiles, plan.n_tiles, k)
+    q, kk, v, g = (inp[n].to(dev) for n in "qkvg")
+    layer = vsa.Layer(plan, w.B, w.H, w.D, k)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 8          # 4 permutes, pool, coarse+top-k, sparse attention, combine
+
+    def step(ev=None):
+        p = plan
+        if ev is not None:
+            ev[0].record(stream)
+        for src, dst in ((q, layer.q_t), (kk, layer.k_t), (v, layer.v_t), (g, layer.g_t)):
+            vsa.vsa_permute(p, src, dst)
+        if ev is not None:
+            ev[1].record(stream)
+        vsa.vsa_coarse_topk(p, layer.q_t, layer.k_t, layer.v_t, k, layer.scale, ws=layer.ws,
+                            o_coarse=layer.o_coarse, topk_idx=layer.topk_idx)
+        if ev is not None:
+            ev[2].record(stream)
+        vsa.vsa_sparse_attn(p, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k, layer.scale,
+                            out=layer.o_fine_t)
+        if ev is not None:
+            ev[3].record(stream)
+        vsa.vsa_gate_combine(p, layer.o_fine_t, layer.g_t, layer.o_coarse, natural=True, out=layer.out)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    vsa.vsa_sync_status(plan)
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.4)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    vsa.vsa_sync_status(plan)
+    elapsed = t_start.elapsed_time(t_end)
+    parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in events])
+    part_ms = parts.mean(axis=0)
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+
+    # end to end through the public API: pinned host inputs in, output back
+    host = {n: inp[n].pin_memory() for n in "qkvg"}
+    out_host = torch.empty(layer.out.shape, dtype=torch.bfloat16, pin_memory=True)
+    dev_in = {"q": q, "k": kk, "v": v, "g": g}
+    e2e_steps = max(1, min(args.steps, 3))
+
+    def e2e_step():
+        for n in "qkvg":
+            dev_in[n].copy_(host[n], non_blocking=True)
+        layer(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"])
+        out_host.copy_(layer.out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_elapsed = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_elapsed = float(t.item())
+    vsa.vsa_sync_status(plan)
+
+    peaks = load_peaks()
+    layers = args.steps * world
+    ms_layer = elapsed / layers
+    attn_ms = float(part_ms[2])
+    achieved = acct["kept_flop"] / (attn_ms * 1e-3) / 1e12
+    res = {
+        "metric": METRIC, "value": round(ms_layer, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; low-rank Q/K field over the tile grid)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "tokens": w.n_tokens,
+                   "tile": "x".join(map(str, w.tile)), "prefix": list(w.prefix),
+                   "grid": list(w.grid), "sparsity": w.sparsity, "kept_video_tiles": k,
+                   "kept_pair_fraction": round(acct["pair_fraction"], 4),
+                   "parallelism": f"replicas x{world}",
+                   "l2": "no flush: every input tensor (1.1 GB) exceeds the 126 MB L2"},
+        "kept_tflops": round(acct["kept_flop"] * layers / (elapsed * 1e-3) / 1e12, 2),
+        "dense_equiv_tflops": round(acct["dense_flop"] * layers / (elapsed * 1e-3) / 1e12, 2),
+        "pct_bf16_peak_layer": round(100 * acct["kept_flop"] * layers / (elapsed * 1e-3) / 1e12 / peaks["bf16"], 2),
+        "kernels_ms": {"permute_x4": round(float(part_ms[0]), 4),
+                       "pool_coarse_topk": round(float(part_ms[1]), 4),
+                       "sparse_attn": round(attn_ms, 4), "gate_combine": round(float(part_ms[3]), 4)},
+        "kernels_hbm_gbs": {"permute_x4": round(acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9, 1),
+                            "gate_combine": round(acct["combine_bytes"] / (part_ms[3] * 1e-3) / 1e9, 1)},
+        "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
+                     "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),
+                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16 burst)",
+                     "traffic": None},
+        "e2e": {"value": round(e2e_elapsed / (e2e_steps * world), 3), "unit": UNIT,
+                "h2d_bytes_per_step": int(sum(host[n].numel() * 2 for n in "qkvg")),
+                "d2h_bytes_per_step": int(out_host.numel() * 2)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = oracle_sample(w, inp)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ----------------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int) -> None:
+    if rank != 0:
+        return
+    w = VEDA_104K
+    inp = make_inputs(w, heads=[0])
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w, inp, n_video_tiles=4, n_prefix_tiles=1)
+        if i >= args.warmup:
+            vals.append(r["value"])
+    v = float(np.median(vals))
+    cb = dict(r)
+    cb["value"] = v
+    res = {"metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(v, 1), "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference",
+           "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "tokens": w.n_tokens,
+                      "tile": "x".join(map(str, w.tile)), "sparsity": w.sparsity},
+           "cpu_baseline": cb,
+           "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

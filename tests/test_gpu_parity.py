@@ -1,0 +1,212 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against
+the fp64 oracle on the same seeded bf16 inputs.
+
+* permutation, tile table and kept-tile sets: bit-exact (a top-k row may
+  differ only by a legal near-tie swap, NEAR_TIE_REL at the k-th score);
+* pooled means and coarse output: fp32 against fp64;
+* o_fine and the layer output: max-abs 2e-2 and mean-abs 2e-3 (bf16 in, fp32
+  accumulation), the oracle evaluated under the GPU's own selection;
+* the full-size workloads in the benchmark's launch configuration, on sampled
+  heads and query tiles the oracle computes one by one.
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests.parity import MAX_ABS, MEAN_ABS, assert_close, check_topk, check_topk_row, f64
+from tile_sparse_video_b200 import vsa
+from tile_sparse_video_b200.inputs import REF2VA, SMALL, TINY, VEDA_104K, Workload, make_inputs, sweep_workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda(libvsa):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.synchronize()
+
+
+_SEEDS = iter(range(9000, 10000, 7))
+
+
+def _w(name, B, H, D, prefix, grid, tile, keep_tiles=None, sparsity=None):
+    return Workload(name, B=B, H=H, D=D, prefix=prefix, grid=grid, tile=tile, keep_tiles=keep_tiles,
+                    sparsity=sparsity, values="iid", gate="marginal", gate_width=64, gate_std=0.2,
+                    seed_base=next(_SEEDS))
+
+
+CASES = [
+    TINY,
+    SMALL,
+    _w("ragged64_b2", 2, 2, 128, (5, 0, 64, 65), (5, 6, 7), (4, 4, 4), keep_tiles=3),
+    _w("ragged128", 1, 2, 128, (256, 3), (8, 17, 9), (4, 8, 4), sparsity=0.9),
+    _w("d64_r128", 1, 3, 64, (100,), (8, 16, 8), (4, 8, 4), keep_tiles=5),
+    _w("noprefix", 1, 2, 128, (), (8, 8, 8), (4, 4, 4), keep_tiles=3),
+    _w("keep_all", 1, 2, 64, (40, 70), (4, 8, 8), (4, 4, 4), sparsity=0.0),
+    _w("keep_none", 1, 2, 128, (40, 70), (4, 8, 8), (4, 4, 4), keep_tiles=0),
+    _w("one_video_tile", 1, 1, 128, (64,), (4, 4, 4), (4, 4, 4), keep_tiles=1),
+    _w("prefix_only", 1, 2, 128, (100, 28), (0, 0, 0), (4, 4, 4), keep_tiles=0),
+]
+# sweep shapes that the oracle finishes quickly (shortest clips, both families)
+CASES += [w for w in sweep_workloads() if w.grid[0] == 16 and ("s90" in w.name or "k24" in w.name)
+          and w.grid[1] == 32]
+
+
+def _keep(plan, w):
+    return plan.keep_count(keep_ratio=w.keep_ratio, keep_tiles=w.keep_tiles)
+
+
+def _run(w: Workload):
+    inp = make_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    q, kk, v, g = (inp[x].cuda() for x in "qkvg")
+    layer = vsa.Layer(plan, w.B, w.H, w.D, k)
+    out = layer(q, kk, v, g)
+    _, _, scores, _ = vsa.vsa_coarse_topk(plan, layer.q_t, layer.k_t, layer.v_t, k, want_scores=True)
+    _, lse = vsa.vsa_sparse_attn(plan, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k, want_lse=True)
+    out_t = vsa.vsa_gate_combine(plan, layer.o_fine_t, layer.g_t, layer.o_coarse, natural=False)
+    vsa.vsa_sync_status(plan)
+    return inp, plan, k, layer, out, scores, lse, out_t
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_layer_parity(w):
+    inp, plan, k, layer, out, scores, lse, out_t = _run(w)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    gpu_idx = layer.topk_idx.cpu().numpy().astype(np.int64)
+    ref = O.layer(*(inp[x] for x in "qkvg"), p, k, kept=gpu_idx)
+
+    # step 1: permutation, bit-exact (pad rows zero)
+    for name in ("q_t", "k_t", "v_t", "g_t"):
+        assert np.array_equal(f64(getattr(layer, name)), ref[name]), name
+    # step 2: pooled means (workspace layout of the header) and coarse output
+    T, D, BH = p.n_tiles, w.D, w.B * w.H
+    pooled = layer.ws[: 3 * BH * T * D * 4].view(torch.float32).view(3, w.B, w.H, T, D)
+    for i, name in enumerate(("qbar", "kbar", "vbar")):
+        np.testing.assert_allclose(f64(pooled[i]), ref[name], rtol=1e-5, atol=1e-6, err_msg=name)
+    np.testing.assert_allclose(f64(layer.o_coarse), ref["o_coarse"], rtol=1e-4, atol=1e-5)
+    # step 3: selection, bit-exact up to legal near-tie swaps
+    near = check_topk(gpu_idx, ref["scores"], p, k)
+    assert near <= max(1, int(np.prod(gpu_idx.shape[:-1])) // 50)
+    if k > 0:
+        gs = f64(scores)
+        want = np.take_along_axis(ref["scores"][..., p.n_prefix_tiles:, :], gpu_idx, axis=-1)
+        np.testing.assert_allclose(gs, want, rtol=1e-4, atol=1e-5)
+    # step 4: fine attention under the GPU's selection
+    assert_close(f64(layer.o_fine_t), ref["o_fine"], what="o_fine")
+    live = p.row_src >= 0
+    np.testing.assert_allclose(f64(lse)[..., live], ref["lse"][..., live], atol=2e-3)
+    assert np.all(f64(lse)[..., ~live] == 0)
+    # step 5: combine, both output layouts
+    assert_close(f64(out), ref["out"], what="out")
+    assert_close(f64(out_t), ref["out_t"], what="out_t")
+    assert np.all(f64(out_t)[..., ~live, :] == 0)
+    assert torch.equal(vsa.vsa_unpermute(plan, out_t), out)
+
+
+def test_keep_all_equals_dense_attention():
+    """k = every video tile: the fine output is plain dense attention over all
+    real tokens (torch's own routine, fp32 on the GPU)."""
+    w = _w("dense_check", 1, 2, 128, (40, 70), (4, 8, 8), (4, 4, 4), sparsity=0.0)
+    inp, plan, k, layer, *_ = _run(w)
+    assert k == plan.n_video_tiles
+    o_nat = vsa.vsa_unpermute(plan, layer.o_fine_t)
+    q, kk, v = (inp[x].cuda().float() for x in "qkv")
+    dense = torch.nn.functional.scaled_dot_product_attention(q, kk, v, scale=w.D ** -0.5)
+    assert_close(f64(o_nat), f64(dense), what="dense")
+
+
+def _sampled(w: Workload, heads, n_video_samples, seed):
+    inp = make_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    dev = torch.device("cuda")
+    q, kk, v, g = (inp[x].to(dev) for x in "qkvg")
+    layer = vsa.Layer(plan, w.B, w.H, w.D, k)
+    out = layer(q, kk, v, g)
+    vsa.vsa_sync_status(plan)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    rng = np.random.default_rng(seed)
+    scale = w.D ** -0.5
+    n_near = 0
+    for b in range(w.B):
+        for h in heads:
+            q_t, k_t, v_t, g_t = (O.permute(inp[x][b, h].to(torch.float64).numpy(), p) for x in "qkvg")
+            qb, kb, vb = O.pool(q_t, p), O.pool(k_t, p), O.pool(v_t, p)
+            s, oc = O.coarse_attention(qb, kb, vb, scale)
+            np.testing.assert_allclose(f64(layer.o_coarse[b, h]), oc, rtol=1e-4, atol=1e-5)
+            idx = layer.topk_idx[b, h].cpu().numpy().astype(np.int64)
+            for r in range(p.n_video_tiles):
+                n_near += check_topk_row(idx[r], s[p.n_prefix_tiles + r], p.n_prefix_tiles, k)
+            tiles = list(range(p.n_prefix_tiles)) + list(
+                p.n_prefix_tiles + rng.choice(p.n_video_tiles, n_video_samples, replace=False))
+            tiles.append(p.n_tiles - 1)
+            out_bh = out[b, h].cpu()
+            o_fine_bh = layer.o_fine_t[b, h].cpu()
+            for i in sorted(set(tiles)):
+                kept = idx[i - p.n_prefix_tiles] if i >= p.n_prefix_tiles else None
+                o, _ = O.fine_tile(q_t, k_t, v_t, p, i, O.key_tiles(p, i, kept), scale)
+                r0, r1 = i * p.R, i * p.R + int(p.block_len[i])
+                want = o + O.sigmoid(g_t[r0:r1]) * oc[i]
+                tok = torch.from_numpy(p.row_src[r0:r1])
+                assert_close(f64(o_fine_bh[r0:r1]), o, what=f"o_fine h{h} tile{i}")
+                assert_close(f64(out_bh[tok]), want, what=f"out h{h} tile{i}")
+    assert n_near <= max(2, w.B * len(heads) * p.n_video_tiles // 50)
+
+
+@pytest.mark.parametrize("w,heads,n", [(REF2VA, (0, 17, 41), 24), (VEDA_104K, (0, 23, 41), 16)],
+                         ids=["ref2va_full", "veda_104k_full"])
+def test_full_size_sampled(w, heads, n):
+    _sampled(w, heads, n, seed=11)
+
+
+def test_error_paths():
+    w = TINY
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    x = torch.zeros(1, 2, plan.n_tokens * 64 + 8, dtype=torch.bfloat16, device="cuda")
+    mis = x.view(-1)[1:1 + 2 * plan.n_tokens * 64].view(1, 2, plan.n_tokens, 64)
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_permute(plan, mis)
+    assert e.value.status == 1
+    q_t = torch.zeros(1, 2, plan.n_padded, 64, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_coarse_topk(plan, q_t, q_t, q_t, 2, ws=ws)
+    assert e.value.status == 4
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_coarse_topk(plan, q_t, q_t, q_t, plan.n_video_tiles + 1)
+    assert e.value.status == 1
+    bad = torch.zeros(1, 2, plan.n_padded, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_permute(plan, torch.zeros(1, 2, plan.n_tokens, 96, dtype=torch.bfloat16, device="cuda"), bad)
+    assert e.value.status == 2
+    vsa.vsa_sync_status(plan)
+
+
+def test_bad_kept_index_is_reported():
+    """An out-of-range kept-tile index is clamped by the kernel and reported
+    through the status word (no fault, no hang)."""
+    w = TINY
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    t = torch.randn(1, 2, plan.n_padded, 64, device="cuda").to(torch.bfloat16)
+    idx = torch.full((1, 2, plan.n_video_tiles, 2), plan.n_prefix_tiles, dtype=torch.int32, device="cuda")
+    idx[0, 1, 2, 1] = plan.n_tiles + 5
+    vsa.vsa_sparse_attn(plan, t, t, t, idx, 2)
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_sync_status(plan)
+    assert e.value.status == 7
+    vsa.vsa_sync_status(plan)       # cleared
+
+
+def test_empty_batch_is_a_no_op():
+    plan = vsa.Plan(TINY.prefix, TINY.grid, TINY.tile)
+    x = torch.empty(0, 2, plan.n_tokens, 64, dtype=torch.bfloat16, device="cuda")
+    assert vsa.vsa_permute(plan, x).shape == (0, 2, plan.n_padded, 64)
+    vsa.vsa_sync_status(plan)

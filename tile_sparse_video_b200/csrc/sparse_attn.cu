@@ -619,10 +619,13 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dynamic shared memory of one CTA.  At least 120 KB, so that two CTAs never
+// share an SM (each allocates its TMEM columns for its whole lifetime).
 template <int R, int D>
 size_t attn_smem_bytes(int T) {
   using C = Cfg<R, D>;
-  return size_t(C::OFF_LISTS) + size_t((2 * T + 15) & ~15) + size_t(4) * T + 1024;
+  const size_t need = size_t(C::OFF_LISTS) + size_t((2 * T + 15) & ~15) + size_t(4) * T + 1024;
+  return need < size_t(120 * 1024) ? size_t(120 * 1024) : need;
 }
 
 template <int R, int D>
