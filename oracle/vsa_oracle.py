@@ -306,6 +306,15 @@ def gate_combine(o_fine, g_t, o_coarse, p: Plan):
 # The whole layer.
 # ---------------------------------------------------------------------------
 
+def as_f64(x) -> np.ndarray:
+    """Exact conversion of an input (numpy array or torch tensor, e.g. bf16)
+    to a float64 numpy array."""
+    if type(x).__module__.split(".")[0] == "torch":
+        import torch
+        return x.detach().to(device="cpu", dtype=torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
 def layer(q, k, v, g, p: Plan, kk: int, scale=None, kept=None):
     """Steps 1-5 on natural-order inputs [B, H, N, D] (any float dtype,
     converted exactly to fp64).  ``kept`` overrides the top-k selection (used
@@ -313,7 +322,7 @@ def layer(q, k, v, g, p: Plan, kk: int, scale=None, kept=None):
     every intermediate, all fp64 except the integer selection."""
     D = q.shape[-1]
     scale = D ** -0.5 if scale is None else scale
-    q_t, k_t, v_t, g_t = (permute(np.asarray(x, dtype=np.float64), p) for x in (q, k, v, g))
+    q_t, k_t, v_t, g_t = (permute(as_f64(x), p) for x in (q, k, v, g))
     qbar, kbar, vbar = pool(q_t, p), pool(k_t, p), pool(v_t, p)
     s, o_coarse = coarse_attention(qbar, kbar, vbar, scale)
     sel = select_topk(s, p, kk) if kept is None else np.asarray(kept, dtype=np.int64)

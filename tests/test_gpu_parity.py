@@ -9,8 +9,6 @@ the fp64 oracle on the same seeded bf16 inputs.
 * the full-size workloads in the benchmark's launch configuration, on sampled
   heads and query tiles the oracle computes one by one.
 """
-from dataclasses import replace
-
 import numpy as np
 import pytest
 import torch
@@ -156,8 +154,11 @@ def _sampled(w: Workload, heads, n_video_samples, seed):
                 r0, r1 = i * p.R, i * p.R + int(p.block_len[i])
                 want = o + O.sigmoid(g_t[r0:r1]) * oc[i]
                 tok = torch.from_numpy(p.row_src[r0:r1])
-                assert_close(f64(o_fine_bh[r0:r1]), o, what=f"o_fine h{h} tile{i}")
-                assert_close(f64(out_bh[tok]), want, what=f"out h{h} tile{i}")
+                # o_fine and out are linear in V: the tolerance (stated for unit-scale
+                # values) scales with the head's value scale s_h where it exceeds 1
+                sv = max(1.0, float(inp["value_scale"][b, h]))
+                assert_close(f64(o_fine_bh[r0:r1]), o, MAX_ABS * sv, MEAN_ABS * sv, what=f"o_fine h{h} tile{i}")
+                assert_close(f64(out_bh[tok]), want, MAX_ABS * sv, MEAN_ABS * sv, what=f"out h{h} tile{i}")
     assert n_near <= max(2, w.B * len(heads) * p.n_video_tiles // 50)
 
 

@@ -47,6 +47,22 @@ constexpr int kThreadsAttn = 192;        // 4 softmax warps + TMA warp + MMA war
 constexpr int kWarpTma = 4, kWarpMma = 5;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
+// Progress trace for debugging builds (-DVSA_TRACE): each role of each CTA
+// publishes its position in the pipeline to a host-visible buffer.  Compiled
+// out otherwise.
+#ifdef VSA_TRACE
+__device__ unsigned int* vsa_trace_buf = nullptr;
+__device__ __forceinline__ void vsa_trace(int slot, unsigned int v) {
+  if (vsa_trace_buf != nullptr) {
+    reinterpret_cast<volatile unsigned int*>(vsa_trace_buf)[blockIdx.x * 8 + slot] = v;
+    __threadfence_system();
+  }
+}
+#define VSA_TR(slot, code, g) vsa_trace((slot), (unsigned(g) << 8) | unsigned(code))
+#else
+#define VSA_TR(slot, code, g) ((void)0)
+#endif
+
 // ---------------------------------------------------------------- PTX wrappers
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -333,6 +349,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) VSA_TR(7, 21, tmem);
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
@@ -350,6 +367,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       __syncwarp();
       if (lane == 0) {
         const int64_t row0 = bh * a.n_pad;
+        VSA_TR(0, 1, g);
         if (t > 0) ok = wait_bar(q_empty, (t - 1) & 1, abort_flag, a.status, 1);
         if (ok) {
           ++q_issued;
@@ -360,6 +378,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         for (int n = 0; n < nk && ok; ++n, ++g) {
           const uint32_t s = g % NS;
+          VSA_TR(0, 3, g);
           if (g >= uint32_t(NS)) {
             ok = wait_bar(kv_empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, 2);
             if (!ok) break;
@@ -372,6 +391,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             tma_load_2d(sK + s * C::KVBYTES + c * BN * 128, &tm_k, kv_full + 8 * s, c * 64, row);
             tma_load_2d(sV + s * C::KVBYTES + c * BN * 128, &tm_v, kv_full + 8 * s, c * 64, row);
           }
+          VSA_TR(0, 4, g);
         }
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -390,8 +410,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       int t = 0;
       bool ok = true;
       auto issue_pv = [&](uint32_t gp, int np_) -> bool {
+        VSA_TR(1, 9, gp);
         if (np_ == 0 && t > 0)
           if (!wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) return false;
+        VSA_TR(1, 10, gp);
         if (!wait_bar(p_full, gp & 1, abort_flag, a.status, 4)) return false;
         tc_fence_after();
         const uint32_t sp = gp % NS;
@@ -403,6 +425,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         umma_commit(pv_done);
         umma_commit(kv_empty + 8 * sp);
+        VSA_TR(1, 11, gp);
         return true;
       };
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
@@ -410,11 +433,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         int i;
         decode_item(item, bh_np, a.n_p, n_v, bh, i);
         const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
+        VSA_TR(1, 5, g);
         if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
         tc_fence_after();
         for (int n = 0; n < nk; ++n, ++g) {
           const uint32_t s = g % NS, sb = g & 1;
+          VSA_TR(1, 6, g);
           if (!wait_bar(kv_full + 8 * s, (g / NS) & 1, abort_flag, a.status, 6)) { ok = false; break; }
+          VSA_TR(1, 7, g);
           if (g >= 2 && !wait_bar(s_empty + 8 * sb, ((g >> 1) - 1) & 1, abort_flag, a.status, 7)) {
             ok = false;
             break;
@@ -428,6 +454,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             umma_bf16(tmem + sb * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
           }
           umma_commit(s_full + 8 * sb);
+          VSA_TR(1, 8, g);
           if (n == nk - 1) umma_commit(q_empty);
           if (n > 0 && !issue_pv(g - 1, n - 1)) { ok = false; break; }
         }
@@ -437,6 +464,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       // Drain: wait until every MMA issued above has completed.
       umma_commit(drain);
       wait_bar_drain(drain, 0);
+      VSA_TR(1, 12, g);
     }
     __syncwarp();
   } else {
@@ -469,7 +497,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       float m = -INFINITY, l = 0.f;
       for (int n = 0; n < nk; ++n, ++g) {
         const uint32_t sb = g & 1;
-        if (!wait_bar(s_full + 8 * sb, (g >> 1) & 1, abort_flag, a.status, 8)) { ok = false; break; }
+        if (lane == 0) VSA_TR(2 + warp, 13, g);
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * sb, (g >> 1) & 1, abort_flag, a.status, 8));
+        if (!ok) break;
         tc_fence_after();
         uint32_t r[BN / 32][32];
         if (rows_active) {
@@ -480,8 +510,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         tc_fence_before();
         mbar_arrive(s_empty + 8 * sb);
+        if (lane == 0) VSA_TR(2 + warp, 14, g);
 
         float alpha = 1.f;
+        bool rescale = false;
         if (rows_active) {
           const int bl = s_blen[n];
           float mx = -INFINITY;
@@ -494,7 +526,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
               r[c][e] = __float_as_uint(x);
               mx = fmaxf(mx, x);
             }
-          const float m_new = fmaxf(m, mx);
+          // Lazy rescale: the reference max moves only when some row of the
+          // warp grew by more than 2^8 (exact math: p <= 256 stays well inside
+          // bf16/fp32 range).  The decision is warp-uniform because the O
+          // rescale below uses warp-collective TMEM loads and stores.
+          const float m_cand = fmaxf(m, mx);
+          rescale = __any_sync(0xFFFFFFFFu, m_cand > m + 8.0f);
+          const float m_new = rescale ? m_cand : m;
           alpha = ex2(m - m_new);
           float sum = 0.f;
 #pragma unroll
@@ -509,7 +547,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           m = m_new;
         }
         // PV of the previous tile must be done before P is overwritten and O is touched.
-        if (g > 0 && !wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 9)) { ok = false; break; }
+        if (lane == 0) VSA_TR(2 + warp, 15, g);
+        if (g > 0) {
+          ok = __all_sync(0xFFFFFFFFu, wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 9));
+          if (!ok) break;
+        }
         tc_fence_after();
         if (rows_active) {
 #pragma unroll
@@ -525,7 +567,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                          "r"(w2), "r"(w3)
                          : "memory");
           }
-          if (n > 0 && alpha < 1.f) {
+          if (n > 0 && rescale) {
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
@@ -541,10 +583,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);
+        if (lane == 0) VSA_TR(2 + warp, 16, g);
       }
       if (!ok) break;
       // ---- epilogue
-      if (!wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 10)) { ok = false; break; }
+      if (lane == 0) VSA_TR(2 + warp, 17, g);
+      ok = __all_sync(0xFFFFFFFFu, wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 10));
+      if (!ok) break;
       tc_fence_after();
       if (rows_active) {
         const bool live = row < q_live;
@@ -571,17 +616,21 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       }
       tc_fence_before();
       mbar_arrive(o_empty);
+      if (lane == 0) VSA_TR(2 + warp, 18, g);
     }
   }
 
   // ---------------------------------------------------------------- teardown
+  if (lane == 0) VSA_TR(warp == kWarpTma ? 0 : (warp == kWarpMma ? 1 : 2 + warp), 19, 0);
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
+    __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(C::TMEM_COLS)
                  : "memory");
+    if (lane == 0) VSA_TR(6, 20, 0);
   }
 }
 

@@ -29,7 +29,8 @@ Recipe (per batch element b, CPU ``torch.Generator`` seeded with
   marginal law of x @ W^T for the two laws above (saves a host GEMM).
 
 Tensors are returned in natural token order, shape [B, H, N, D], bf16,
-contiguous, on the CPU.
+contiguous, on the CPU, under keys "q", "k", "v", "g"; "value_scale" [B, H]
+holds s_h (1.0 without per-head scaling).
 """
 from __future__ import annotations
 
@@ -155,6 +156,9 @@ def make_inputs(w: Workload, batch: Optional[Sequence[int]] = None,
     N, D, P = w.n_tokens, w.D, w.n_prefix
     shape = (len(bsel), len(hsel), N, D)
     out = {k: torch.empty(shape, dtype=torch.bfloat16) for k in ("q", "k", "v", "g")}
+    # per-(b, h) value scale (1 unless values == "head_scaled"); returned so a
+    # comparison can state its tolerance per unit of value scale
+    out["value_scale"] = torch.ones(len(bsel), len(hsel), dtype=torch.float64)
     cells = _video_cells(w) if w.values == "low_rank" else None
     tt, th, tw = w.tile
     n_cells = (-(-w.grid[0] // tt)) * (-(-w.grid[1] // th)) * (-(-w.grid[2] // tw))
@@ -164,6 +168,7 @@ def make_inputs(w: Workload, batch: Optional[Sequence[int]] = None,
         field_ = None
         if w.values == "head_scaled":
             scale = 0.5 + 1.5 * torch.rand(w.H, generator=gen)
+            out["value_scale"][bi] = scale[hsel].double()
         if w.values == "low_rank":
             field_ = torch.randn(w.H, n_cells, 16, generator=gen)
         for name in ("q", "k", "v"):
