@@ -138,6 +138,26 @@ vsa_status vsa_coarse_topk(vsa_plan plan, const void* q_t, const void* k_t, cons
                            float* o_coarse, int32_t* topk_idx, float* topk_score,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of vsa_coarse_topk (the pages have no counterpart:
+ * this is a library convenience).  For callers that cannot call cudaMalloc --
+ * a host application that owns all device memory and gives plugins no
+ * allocator, or a latency-critical loop that cannot afford cudaMalloc's
+ * implicit device-wide synchronisation -- the pooled-mean scratch lives in a
+ * fixed 16 MiB array in the library's device memory, held on every GPU that
+ * loads the library until the process exits.  Same arguments and results as
+ * vsa_coarse_topk, without ws / ws_bytes; allocates nothing.
+ * Limit: the call needs 3*B*H*T*D*4 bytes of scratch and returns
+ * VSA_ERR_WORKSPACE, launching nothing, when that exceeds 16 MiB.
+ * The first call on a device resolves the array's device address with
+ * cudaGetSymbolAddress (once per device, that device current); make that first
+ * call before any stream capture.  All calls share the array, which keeps the
+ * last call's contents (nothing in it needs to start at zero); calls that
+ * overlap on the GPU race on it and must be serialised by the caller. */
+vsa_status vsa_coarse_topk_noalloc(vsa_plan plan, const void* q_t, const void* k_t,
+                                   const void* v_t, int B, int H, int D, float scale, int k,
+                                   float* o_coarse, int32_t* topk_idx, float* topk_score,
+                                   void* stream);
+
 /* Step 4.  For every live query row of tile i and head: softmax over the live
  * key rows of S_i, o_fine = sum p v, with S_i = all T tiles when i < n_p
  * (prefix queries are dense) and S_i = {0..n_p-1} U topk_idx[b,h,i-n_p,:]

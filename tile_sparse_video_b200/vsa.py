@@ -26,8 +26,8 @@ STATUS_NAMES = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED",
 # exported C symbols (kept in step with include/vsa.h)
 EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_count",
            "vsa_plan_destroy", "vsa_workspace_size", "vsa_permute", "vsa_unpermute",
-           "vsa_coarse_topk", "vsa_sparse_attn", "vsa_gate_combine", "vsa_sync_status",
-           "vsa_last_error")
+           "vsa_coarse_topk", "vsa_coarse_topk_noalloc", "vsa_sparse_attn", "vsa_gate_combine",
+           "vsa_sync_status", "vsa_last_error")
 
 
 class VsaError(RuntimeError):
@@ -63,6 +63,7 @@ def lib():
             "vsa_permute": [P, V, V, I, I, I, V],
             "vsa_unpermute": [P, V, V, I, I, I, V],
             "vsa_coarse_topk": [P, V, V, V, I, I, I, F, I, V, V, V, V, Z, V],
+            "vsa_coarse_topk_noalloc": [P, V, V, V, I, I, I, F, I, V, V, V, V],
             "vsa_sparse_attn": [P, V, V, V, V, I, I, I, I, F, V, V, V, Z, V],
             "vsa_gate_combine": [P, V, V, V, V, I, I, I, I, V],
             "vsa_sync_status": [P, V],
@@ -210,6 +211,29 @@ def vsa_coarse_topk(plan: Plan, q_t, k_t, v_t, k: int, scale: Optional[float] = 
                                  _ptr(scores) if scores is not None and scores.numel() else None,
                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
     return o_coarse, topk_idx, scores, ws
+
+
+def vsa_coarse_topk_noalloc(plan: Plan, q_t, k_t, v_t, k: int, scale: Optional[float] = None,
+                            o_coarse=None, topk_idx=None, want_scores: bool = False, stream=None):
+    """Like vsa_coarse_topk, but the library keeps the scratch in its own fixed
+    16 MiB device array (for callers that cannot allocate).  Returns
+    (o_coarse, topk_idx, scores or None)."""
+    B, H, _, D = q_t.shape
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("v_t", v_t)):
+        _need(t, name, torch.bfloat16, (B, H, plan.n_padded, D))
+    dev = q_t.device
+    scale = D ** -0.5 if scale is None else float(scale)
+    if o_coarse is None:
+        o_coarse = torch.empty(B, H, plan.n_tiles, D, dtype=torch.float32, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty(B, H, plan.n_video_tiles, max(k, 0), dtype=torch.int32, device=dev)
+    scores = (torch.empty(B, H, plan.n_video_tiles, max(k, 0), dtype=torch.float32, device=dev)
+              if want_scores else None)
+    _check(lib().vsa_coarse_topk_noalloc(plan.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), B, H, D, scale,
+                                         k, _ptr(o_coarse), _ptr(topk_idx) if topk_idx.numel() else None,
+                                         _ptr(scores) if scores is not None and scores.numel() else None,
+                                         _stream(stream)))
+    return o_coarse, topk_idx, scores
 
 
 def vsa_sparse_attn(plan: Plan, q_t, k_t, v_t, topk_idx, k: int, scale: Optional[float] = None,
