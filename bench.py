@@ -36,7 +36,9 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from tile_sparse_video_b200.inputs import VEDA_104K, Workload, make_inputs  # noqa: E402
+from dataclasses import replace  # noqa: E402
+
+from tile_sparse_video_b200.inputs import VEDA_104K, WORKLOADS, Workload, make_inputs  # noqa: E402
 
 METRIC = "ms/layer & kept-FLOP TFLOP/s (% bf16 peak) at 104k tokens, 90% tile sparsity"
 UNIT = "ms/layer"
@@ -173,13 +175,22 @@ def oracle_sample(w: Workload, inp: dict, n_video_tiles: int = 256, n_prefix_til
 
 # ----------------------------------------------------------------- GPU arm
 
+def pick_workload(args) -> Workload:
+    """The benchmark workload: the 104k-token Veda layer unless a profiling
+    run names another (``--workload``) or fewer heads (``--heads``)."""
+    w = WORKLOADS[args.workload] if args.workload else VEDA_104K
+    if args.heads:
+        w = replace(w, name=f"{w.name}_heads{args.heads}", H=args.heads)
+    return w
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     from tile_sparse_video_b200 import vsa
     import torch.distributed as dist
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = VEDA_104K
+    w = pick_workload(args)
     inp = make_inputs(w)
     plan = vsa.Plan(w.prefix, w.grid, w.tile, device=local_rank)
     k = plan.keep_count(keep_ratio=w.keep_ratio, keep_tiles=w.keep_tiles)
@@ -244,7 +255,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     host = {n: inp[n].pin_memory() for n in "qkvg"}
     out_host = torch.empty(layer.out.shape, dtype=torch.bfloat16, pin_memory=True)
     dev_in = {"q": q, "k": kk, "v": v, "g": g}
-    e2e_steps = max(1, min(args.steps, 3))
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 3))
 
     def e2e_step():
         for n in "qkvg":
@@ -252,7 +263,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         layer(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"])
         out_host.copy_(layer.out, non_blocking=True)
 
-    e2e_step()
+    if e2e_steps:
+        e2e_step()
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -297,7 +309,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                      "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),
                      "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16 burst)",
                      "traffic": None},
-        "e2e": {"value": round(e2e_elapsed / (e2e_steps * world), 3), "unit": UNIT,
+        "e2e": {"value": round(e2e_elapsed / (max(e2e_steps, 1) * world), 3) if e2e_steps else None,
+                "unit": UNIT,
                 "h2d_bytes_per_step": int(sum(host[n].numel() * 2 for n in "qkvg")),
                 "d2h_bytes_per_step": int(out_host.numel() * 2)},
         "gpu_launches": launches_per_step * args.steps,
@@ -342,6 +355,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
+                    help="profiling runs only: another named workload")
+    ap.add_argument("--heads", type=int, default=0, help="profiling runs only: fewer heads")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", "0"))

@@ -12,22 +12,27 @@
 //   work item = (b*h, query tile i); prefix items (n_p of them per head, each
 //   T key tiles long) come first, then the video items head by head, so the
 //   CTAs share one or two heads' K/V in L2 at any time.
-//   warp 4  (TMA)    loads Q once per item and K_j, V_j per kept tile into an
-//                    NS-stage ring (128-byte swizzled boxes of 64 columns).
-//   warp 5  (MMA)    one elected lane issues S = Q K_j^T (M=128, N=R, K=D) into
-//                    one of two TMEM S buffers, then O += P V_{j-1} (M=128,
-//                    N=D, K=R) once the softmax has written P_{j-1}; every
-//                    completion is signalled with tcgen05.commit on an mbarrier.
-//   warps 0-3        thread t owns query row t = TMEM lane t: it loads its S
-//                    row from TMEM, applies the block_len mask and the running
-//                    max, writes P = exp2(S*scale*log2e - m) as bf16 into a
-//                    swizzled shared-memory tile (the A operand of the PV MMA),
-//                    rescales its O row in TMEM when the max grew, and in the
-//                    epilogue divides by the row sum and stores bf16 rows.
-// TMEM columns: S0 [0,R), S1 [R,2R), O [2R, 2R+D).
+//   warp 8  (TMA K)  loads Q once per item and K_j per kept tile into a K ring,
+//                    and prefetches K/V tiles a few steps ahead into L2.
+//   warp 9  (TMA V)  loads V_j into its own ring (V is needed later than K).
+//   warp 10 (MMA)    one lane issues S_n = Q K_n^T (M=128, N=R, K=D) into the
+//                    TMEM S buffer of warpgroup n & 1, and O_w += P_n V_n
+//                    (M=128, N=D, K=R) once P_n is written; order per item:
+//                    S0, S1, then S_{n+2}, PV_n for every n.
+//   warps 0-7        two softmax warpgroups; warpgroup w takes the tiles
+//                    n = w (mod 2) of an item (a split of the key set inside the
+//                    CTA).  Thread = query row = TMEM lane: it loads its S row,
+//                    masks past block_len, keeps a running max (moved only when
+//                    a row grew by more than 2^8, exact), writes P = exp2(.) as
+//                    bf16 into the single 128-byte-swizzled shared P tile (the
+//                    A operand of the PV MMA; the two warpgroups take turns in
+//                    tile order) and rescales its O_w row in TMEM when the max
+//                    moved.  The epilogue merges the two partial (m, l, O)
+//                    states and stores bf16 rows (and the LSE).
+// TMEM columns: S_0 [0,R), S_1 [R,2R), O_0 [2R,2R+D), O_1 [2R+D,2R+2D).
 // With R = 64 the MMA still runs with M = 128 (rows 64..127 of the Q box are
 // the next rows of the tensor, or zero past its end); their results are never
-// stored and warps 2-3 skip the softmax work for them.
+// stored and the warps of those rows skip the softmax work.
 //
 // Every mbarrier wait is bounded (kWaitLimitNs of wall time); on expiry the
 // CTA raises an abort flag, records VSA_ERR_DEVICE_TIMEOUT in the status word,
@@ -43,18 +48,18 @@ namespace vsa {
 namespace {
 
 constexpr int kBM = 128;                 // MMA M (query rows per item)
-constexpr int kThreadsAttn = 192;        // 4 softmax warps + TMA warp + MMA warp
-constexpr int kWarpTma = 4, kWarpMma = 5;
+constexpr int kThreadsAttn = 352;        // 8 softmax warps + TMA K + TMA V + MMA
+constexpr int kWarpTmaK = 8, kWarpTmaV = 9, kWarpMma = 10;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
 // Progress trace for debugging builds (-DVSA_TRACE): each role of each CTA
-// publishes its position in the pipeline to a host-visible buffer.  Compiled
-// out otherwise.
+// publishes its position in the pipeline to a host-visible buffer (16 slots
+// per CTA).  Compiled out otherwise.
 #ifdef VSA_TRACE
 __device__ unsigned int* vsa_trace_buf = nullptr;
 __device__ __forceinline__ void vsa_trace(int slot, unsigned int v) {
   if (vsa_trace_buf != nullptr) {
-    reinterpret_cast<volatile unsigned int*>(vsa_trace_buf)[blockIdx.x * 8 + slot] = v;
+    reinterpret_cast<volatile unsigned int*>(vsa_trace_buf)[blockIdx.x * 16 + slot] = v;
     __threadfence_system();
   }
 }
@@ -103,6 +108,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
+}
+// L2 prefetch of one tensor-map box (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -214,21 +226,25 @@ struct AttnArgs {
 template <int R, int D>
 struct Cfg {
   static constexpr int BN = R;
-  static constexpr int NS = (R == 128) ? 2 : 4;         // K/V pipeline stages
+  static constexpr int NSK = (R == 128) ? 2 : 4;        // K ring stages
+  static constexpr int NSV = (R == 128) ? 2 : 4;        // V ring stages
   static constexpr int QBYTES = kBM * D * 2;
-  static constexpr int KVBYTES = BN * D * 2;             // one K (or V) tile
+  static constexpr int TBYTES = BN * D * 2;              // one K (or V) tile
   static constexpr int PBYTES = kBM * BN * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBYTES;
-  static constexpr int OFF_V = OFF_K + NS * KVBYTES;
-  static constexpr int OFF_P = OFF_V + NS * KVBYTES;
+  static constexpr int OFF_V = OFF_K + NSK * TBYTES;
+  static constexpr int OFF_P = OFF_V + NSV * TBYTES;
   static constexpr int OFF_BAR = OFF_P + PBYTES;
-  // barriers: q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], s_empty[2],
-  //           p_full, pv_done, o_empty, drain
-  static constexpr int NBAR = 2 + 2 * NS + 4 + 4;
+  // barriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV],
+  //           s_full[2], s_empty[2], p_full, pv_done[2], o_empty, drain
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 4 + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag
-  static constexpr int OFF_LISTS = OFF_MISC + 16;
-  static constexpr uint32_t TMEM_COLS = (2 * BN + D) <= 256 ? 256u : 512u;
+  static constexpr int OFF_ML = OFF_MISC + 16;           // float m[2][128], l[2][128]
+  static constexpr int OFF_LISTS = OFF_ML + 4 * 128 * 4;
+  static constexpr uint32_t TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256u : 512u;
+  static constexpr uint32_t COL_S = 0;                   // S_w at COL_S + w*BN
+  static constexpr uint32_t COL_O = 2 * BN;              // O_w at COL_O + w*D
   static constexpr uint32_t IDESC_QK = idesc_bf16(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, false, true);
 };
@@ -287,13 +303,84 @@ __device__ __forceinline__ int kept_tile(const AttnArgs& a, int64_t bh, int i, i
   return j;
 }
 
+// Producer loop shared by the K and the V warp: lane 0 issues one TMA tile per
+// kept key tile into an NS-stage ring; the K warp also loads Q per item and
+// prefetches K/V tiles kPrefetch ahead into L2.
+template <int R, int D, int NS, bool kIsK>
+__device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* tm_q,
+                                         const CUtensorMap* tm_t, const CUtensorMap* tm_other,
+                                         uint32_t sQ, uint32_t sT, uint32_t full, uint32_t empty,
+                                         uint32_t q_full, uint32_t q_empty, int32_t* s_list,
+                                         volatile int* abort_flag, int lane, int bh_np, int n_v) {
+  using C = Cfg<R, D>;
+  constexpr int kPrefetch = 4;
+  uint32_t g = 0, q_issued = 0;
+  int t = 0;
+  bool ok = true;
+  for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+    int64_t bh;
+    int i;
+    decode_item(item, bh_np, a.n_p, n_v, bh, i);
+    const bool dense = i < a.n_p;
+    const int nk = dense ? a.T : a.n_p + a.k;
+    if (!dense)
+      for (int x = lane; x < a.k; x += 32) s_list[x] = kept_tile(a, bh, i, x);
+    __syncwarp();
+    if (lane == 0) {
+      const int64_t row0 = bh * a.n_pad;
+      if (kIsK) {
+        VSA_TR(8, 1, g);
+        if (t > 0) ok = wait_bar(q_empty, (t - 1) & 1, abort_flag, a.status, 1);
+        if (ok) {
+          ++q_issued;
+          mbar_expect_tx(q_full, C::QBYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sQ + c * kBM * 128, tm_q, q_full, c * 64, int(row0 + int64_t(i) * R));
+        }
+      }
+      for (int n = 0; n < nk && ok; ++n, ++g) {
+        const uint32_t s = g % NS;
+        if (g >= uint32_t(NS)) {
+          ok = wait_bar(empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, kIsK ? 2 : 11);
+          if (!ok) break;
+        }
+        const int j = (dense || n < a.n_p) ? n : s_list[n - a.n_p];
+        const int row = int(row0 + int64_t(j) * R);
+        mbar_expect_tx(full + 8 * s, C::TBYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(sT + s * C::TBYTES + c * C::BN * 128, tm_t, full + 8 * s, c * 64, row);
+        if (kIsK && n + kPrefetch < nk) {
+          const int jp = (dense || n + kPrefetch < a.n_p) ? n + kPrefetch : s_list[n + kPrefetch - a.n_p];
+          const int rp = int(row0 + int64_t(jp) * R);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_prefetch_l2(tm_t, c * 64, rp);
+            tma_prefetch_l2(tm_other, c * 64, rp);
+          }
+        }
+        VSA_TR(kIsK ? 8 : 9, 4, g);
+      }
+    }
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+  }
+  if (lane == 0 && !ok) {
+    // Abort: make sure none of our TMA writes is still in flight.
+    for (uint32_t x = (g > uint32_t(NS) ? g - NS : 0); x < g; ++x)
+      wait_bar_drain(full + 8 * (x % NS), (x / NS) & 1);
+    if (kIsK && q_issued > 0) wait_bar_drain(q_full, (q_issued - 1) & 1);
+  }
+}
+
 template <int R, int D>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   using C = Cfg<R, D>;
-  constexpr int BN = C::BN, NS = C::NS;
+  constexpr int BN = C::BN, NSK = C::NSK, NSV = C::NSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -302,14 +389,22 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                  sP = s_base + C::OFF_P;
   const uint32_t bar0 = s_base + C::OFF_BAR;
   const uint32_t q_full = bar0, q_empty = bar0 + 8;
-  const uint32_t kv_full = bar0 + 16, kv_empty = kv_full + 8 * NS;
-  const uint32_t s_full = kv_empty + 8 * NS, s_empty = s_full + 16;
-  const uint32_t p_full = s_empty + 16, pv_done = p_full + 8, o_empty = pv_done + 8,
+  const uint32_t k_full = bar0 + 16, k_empty = k_full + 8 * NSK;
+  const uint32_t v_full = k_empty + 8 * NSK, v_empty = v_full + 8 * NSV;
+  const uint32_t s_full = v_empty + 8 * NSV, s_empty = s_full + 16;
+  // pv_done[w] completes once per PV of warpgroup w's tiles.  A waiter never
+  // lags a barrier by two phases (which would alias in the parity test): a
+  // warpgroup waits for the other's PV of tile n-1 only after it has seen the
+  // other's PV of tile n-3.
+  const uint32_t p_full = s_empty + 16, pv_done = p_full + 8, o_empty = pv_done + 16,
                  drain = o_empty + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  int16_t* s_blen = reinterpret_cast<int16_t*>(smem + C::OFF_LISTS);         // [T]
-  int32_t* s_plist = reinterpret_cast<int32_t*>(smem + C::OFF_LISTS + ((2 * a.T + 15) & ~15));
+  float* s_m = reinterpret_cast<float*>(smem + C::OFF_ML);          // [2][128]
+  float* s_l = s_m + 2 * 128;                                        // [2][128]
+  uint8_t* s_blen = smem + C::OFF_LISTS;                             // [T]
+  int32_t* s_klist = reinterpret_cast<int32_t*>(smem + C::OFF_LISTS + ((a.T + 15) & ~15));
+  int32_t* s_vlist = s_klist + ((a.k + 3) & ~3);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_v = a.T - a.n_p;
@@ -318,22 +413,27 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(kv_full + 8 * s, 1);
-      mbar_init(kv_empty + 8 * s, 1);
+    for (int s = 0; s < NSK; ++s) {
+      mbar_init(k_full + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(s_full + 8 * s, 1);
-      mbar_init(s_empty + 8 * s, 128);
+    for (int s = 0; s < NSV; ++s) {
+      mbar_init(v_full + 8 * s, 1);
+      mbar_init(v_empty + 8 * s, 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(s_full + 8 * w, 1);
+      mbar_init(s_empty + 8 * w, 128);
     }
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
-    mbar_init(o_empty, 128);
+    mbar_init(pv_done + 8, 1);
+    mbar_init(o_empty, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == kWarpTma && lane == 0) {
+  if (warp == kWarpTmaK && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -349,83 +449,61 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) VSA_TR(7, 21, tmem);
+  if (threadIdx.x == 0) VSA_TR(10, 21, tmem);
 
-  if (warp == kWarpTma) {
-    // ------------------------------------------------------------ TMA producer
-    uint32_t g = 0, q_issued = 0;
-    int t = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
-      int64_t bh;
-      int i;
-      decode_item(item, bh_np, a.n_p, n_v, bh, i);
-      const bool dense = i < a.n_p;
-      const int nk = dense ? a.T : a.n_p + a.k;
-      if (!dense)
-        for (int x = lane; x < a.k; x += 32) s_plist[x] = kept_tile(a, bh, i, x);
-      __syncwarp();
-      if (lane == 0) {
-        const int64_t row0 = bh * a.n_pad;
-        VSA_TR(0, 1, g);
-        if (t > 0) ok = wait_bar(q_empty, (t - 1) & 1, abort_flag, a.status, 1);
-        if (ok) {
-          ++q_issued;
-          mbar_expect_tx(q_full, C::QBYTES);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sQ + c * kBM * 128, &tm_q, q_full, c * 64, int(row0 + int64_t(i) * R));
-        }
-        for (int n = 0; n < nk && ok; ++n, ++g) {
-          const uint32_t s = g % NS;
-          VSA_TR(0, 3, g);
-          if (g >= uint32_t(NS)) {
-            ok = wait_bar(kv_empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, 2);
-            if (!ok) break;
-          }
-          const int j = (dense || n < a.n_p) ? n : s_plist[n - a.n_p];
-          const int row = int(row0 + int64_t(j) * R);
-          mbar_expect_tx(kv_full + 8 * s, 2 * C::KVBYTES);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(sK + s * C::KVBYTES + c * BN * 128, &tm_k, kv_full + 8 * s, c * 64, row);
-            tma_load_2d(sV + s * C::KVBYTES + c * BN * 128, &tm_v, kv_full + 8 * s, c * 64, row);
-          }
-          VSA_TR(0, 4, g);
-        }
-      }
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      __syncwarp();
-    }
-    if (lane == 0 && !ok) {
-      // Abort: make sure none of our TMA writes is still in flight.
-      for (uint32_t x = (g > uint32_t(NS) ? g - NS : 0); x < g; ++x)
-        wait_bar_drain(kv_full + 8 * (x % NS), (x / NS) & 1);
-      if (q_issued > 0) wait_bar_drain(q_full, (q_issued - 1) & 1);
-    }
+  if (warp == kWarpTmaK) {
+    producer<R, D, NSK, true>(a, &tm_q, &tm_k, &tm_v, sQ, sK, k_full, k_empty, q_full, q_empty,
+                              s_klist, abort_flag, lane, bh_np, n_v);
+  } else if (warp == kWarpTmaV) {
+    producer<R, D, NSV, false>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full, q_empty,
+                               s_vlist, abort_flag, lane, bh_np, n_v);
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
+    // Order per item: S(0), S(1), then for every tile n: S(n+2), PV(n).
+    // Tile n belongs to softmax warpgroup w = n & 1 (S_w, O_w in TMEM); the
+    // single P buffer in shared memory is written in tile order.
     if (lane == 0) {
-      uint32_t g = 0;
+      uint32_t g = 0;            // global tile counter (K/V rings, p_full, pv_done)
+      uint32_t si[2] = {0, 0};   // S issues per warpgroup (s_full / s_empty phases)
       int t = 0;
       bool ok = true;
-      auto issue_pv = [&](uint32_t gp, int np_) -> bool {
-        VSA_TR(1, 9, gp);
-        if (np_ == 0 && t > 0)
-          if (!wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) return false;
-        VSA_TR(1, 10, gp);
-        if (!wait_bar(p_full, gp & 1, abort_flag, a.status, 4)) return false;
+      auto issue_s = [&](uint32_t gt, int w) -> bool {
+        const uint32_t s = gt % NSK;
+        VSA_TR(11, 6, gt);
+        if (!wait_bar(k_full + 8 * s, (gt / NSK) & 1, abort_flag, a.status, 6)) return false;
+        if (si[w] > 0 && !wait_bar(s_empty + 8 * w, (si[w] - 1) & 1, abort_flag, a.status, 7))
+          return false;
         tc_fence_after();
-        const uint32_t sp = gp % NS;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ad = sdesc_sw128(sQ + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
+          const uint64_t bd =
+              sdesc_sw128(sK + s * C::TBYTES + (ks / 4) * BN * 128 + (ks % 4) * 32, 16, 1024);
+          umma_bf16(tmem + C::COL_S + w * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + 8 * w);
+        umma_commit(k_empty + 8 * s);
+        ++si[w];
+        VSA_TR(11, 8, gt);
+        return true;
+      };
+      auto issue_pv = [&](uint32_t gt, int n) -> bool {
+        const int w = n & 1;
+        if (n == 0 && t > 0 && !wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) return false;
+        VSA_TR(11, 10, gt);
+        if (!wait_bar(p_full, gt & 1, abort_flag, a.status, 4)) return false;
+        const uint32_t sv = gt % NSV;
+        if (!wait_bar(v_full + 8 * sv, (gt / NSV) & 1, abort_flag, a.status, 12)) return false;
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
           const uint64_t ad = sdesc_sw128(sP + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sV + sp * C::KVBYTES + ks * 16 * 128, BN * 128, 1024);
-          umma_bf16(tmem + 2 * BN, ad, bd, C::IDESC_PV, (np_ > 0 || ks > 0) ? 1u : 0u);
+          const uint64_t bd = sdesc_sw128(sV + sv * C::TBYTES + ks * 16 * 128, BN * 128, 1024);
+          umma_bf16(tmem + C::COL_O + w * D, ad, bd, C::IDESC_PV, (n >= 2 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(pv_done);
-        umma_commit(kv_empty + 8 * sp);
-        VSA_TR(1, 11, gp);
+        umma_commit(pv_done + 8 * w);
+        umma_commit(v_empty + 8 * sv);
+        VSA_TR(11, 11, gt);
         return true;
       };
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
@@ -433,46 +511,38 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         int i;
         decode_item(item, bh_np, a.n_p, n_v, bh, i);
         const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
-        VSA_TR(1, 5, g);
+        VSA_TR(11, 5, g);
         if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
         tc_fence_after();
-        for (int n = 0; n < nk; ++n, ++g) {
-          const uint32_t s = g % NS, sb = g & 1;
-          VSA_TR(1, 6, g);
-          if (!wait_bar(kv_full + 8 * s, (g / NS) & 1, abort_flag, a.status, 6)) { ok = false; break; }
-          VSA_TR(1, 7, g);
-          if (g >= 2 && !wait_bar(s_empty + 8 * sb, ((g >> 1) - 1) & 1, abort_flag, a.status, 7)) {
-            ok = false;
-            break;
+        for (int n = 0; n < 2 && n < nk && ok; ++n) ok = issue_s(g + n, n);
+        if (ok && nk <= 2) umma_commit(q_empty);
+        for (int n = 0; n < nk && ok; ++n) {
+          if (n + 2 < nk) {
+            ok = issue_s(g + n + 2, n & 1);
+            if (ok && n + 3 == nk) umma_commit(q_empty);
           }
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ad = sdesc_sw128(sQ + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
-            const uint64_t bd =
-                sdesc_sw128(sK + s * C::KVBYTES + (ks / 4) * BN * 128 + (ks % 4) * 32, 16, 1024);
-            umma_bf16(tmem + sb * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
-          }
-          umma_commit(s_full + 8 * sb);
-          VSA_TR(1, 8, g);
-          if (n == nk - 1) umma_commit(q_empty);
-          if (n > 0 && !issue_pv(g - 1, n - 1)) { ok = false; break; }
+          if (ok) ok = issue_pv(g + n, n);
         }
-        if (!ok) break;
-        if (!issue_pv(g - 1, nk - 1)) { ok = false; break; }
+        g += nk;
       }
       // Drain: wait until every MMA issued above has completed.
       umma_commit(drain);
       wait_bar_drain(drain, 0);
-      VSA_TR(1, 12, g);
+      VSA_TR(11, 12, g);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const bool rows_active = (R == 128) || (warp < 2);
-    const int row = warp * 32 + lane;                    // = TMEM lane
-    const uint32_t t_lane = tmem + (uint32_t(warp * 32) << 16);
-    uint32_t g = 0;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;                            // 0 or 1
+    const int quad = warp & 3;
+    const bool rows_active = (R == 128) || (quad < 2);
+    const int row = quad * 32 + lane;                    // = TMEM lane
+    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
+    const uint32_t col_s = C::COL_S + wg * BN;
+    const uint32_t col_o = C::COL_O + wg * D;
+    uint32_t g = 0;              // global tile counter (trace only)
+    uint32_t cnt[2] = {0, 0};    // tiles of each warpgroup in earlier items
+    uint32_t cw = 0;             // tiles processed by this warpgroup (s_full phases)
     int t = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
@@ -481,75 +551,90 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       decode_item(item, bh_np, a.n_p, n_v, bh, i);
       const bool dense = i < a.n_p;
       const int nk = dense ? a.T : a.n_p + a.k;
-      // Group barrier of the 128 softmax threads.  A warp that sees the abort
+      // Group barrier of the 256 softmax threads.  A warp that sees the abort
       // flag leaves instead: the others then also see it before they could
       // block here (they wait on the same mbarrier phases first).
       if (*abort_flag) { ok = false; break; }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int x = threadIdx.x; x < nk; x += 128) {
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      for (int x = threadIdx.x; x < nk; x += 256) {
         const int j = (dense || x < a.n_p) ? x : kept_tile(a, bh, i, x - a.n_p);
-        s_blen[x] = int16_t(__ldg(a.block_len + j));
+        s_blen[x] = uint8_t(__ldg(a.block_len + j) - 1);
       }
       if (*abort_flag) { ok = false; break; }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       const int q_live = __ldg(a.block_len + i);
 
       float m = -INFINITY, l = 0.f;
-      for (int n = 0; n < nk; ++n, ++g) {
-        const uint32_t sb = g & 1;
-        if (lane == 0) VSA_TR(2 + warp, 13, g);
-        ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * sb, (g >> 1) & 1, abort_flag, a.status, 8));
+      for (int n = wg; n < nk; n += 2, ++cw) {
+        const uint32_t gn = g + n;
+        if (lane == 0) VSA_TR(quad + 4 * wg, 13, gn);
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * wg, cw & 1, abort_flag, a.status, 8));
         if (!ok) break;
         tc_fence_after();
         uint32_t r[BN / 32][32];
         if (rows_active) {
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + sb * BN + 32 * c, r[c]);
+          for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + col_s + 32 * c, r[c]);
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c) tmem_wait_ld(r[c]);
         }
         tc_fence_before();
-        mbar_arrive(s_empty + 8 * sb);
-        if (lane == 0) VSA_TR(2 + warp, 14, g);
+        mbar_arrive(s_empty + 8 * wg);
 
-        float alpha = 1.f;
         bool rescale = false;
+        float alpha = 1.f;
         if (rows_active) {
-          const int bl = s_blen[n];
-          float mx = -INFINITY;
+          // Row max over raw scores (scale > 0 commutes with max), four
+          // independent chains so the warp is not latency-bound.
+          const int bl = int(s_blen[n]) + 1;
+          if (bl < BN) {
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (32 * c + e >= bl) r[c][e] = __float_as_uint(-INFINITY);
+          }
+          float mx4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mx4[q] = -INFINITY;
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              float x = __uint_as_float(r[c][e]) * a.scale_log2;
-              if (bl < BN && 32 * c + e >= bl) x = -INFINITY;
-              r[c][e] = __float_as_uint(x);
-              mx = fmaxf(mx, x);
-            }
+            for (int e = 0; e < 32; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(r[c][e]));
+          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
           // Lazy rescale: the reference max moves only when some row of the
           // warp grew by more than 2^8 (exact math: p <= 256 stays well inside
           // bf16/fp32 range).  The decision is warp-uniform because the O
           // rescale below uses warp-collective TMEM loads and stores.
-          const float m_cand = fmaxf(m, mx);
+          const float m_cand = fmaxf(m, mx * a.scale_log2);
           rescale = __any_sync(0xFFFFFFFFu, m_cand > m + 8.0f);
           const float m_new = rescale ? m_cand : m;
           alpha = ex2(m - m_new);
-          float sum = 0.f;
+          const float neg_m = -m_new;
+          float sum4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) sum4[q] = 0.f;
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float p = ex2(__uint_as_float(r[c][e]) - m_new);
-              sum += p;
+              const float p = ex2(fmaf(__uint_as_float(r[c][e]), a.scale_log2, neg_m));
+              sum4[e & 3] += p;
               r[c][e] = __float_as_uint(p);
             }
+          const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
           l = l * alpha + sum;
           m = m_new;
         }
-        // PV of the previous tile must be done before P is overwritten and O is touched.
-        if (lane == 0) VSA_TR(2 + warp, 15, g);
-        if (g > 0) {
-          ok = __all_sync(0xFFFFFFFFu, wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 9));
+        // The previous tile's PV (the other warpgroup's) must be done before
+        // the shared P buffer is overwritten; it also orders this
+        // warpgroup's own earlier PV into O_w before the rescale below.  For
+        // n = 0 the previous item's epilogue already waited for all its PVs.
+        if (lane == 0) VSA_TR(quad + 4 * wg, 15, gn);
+        if (n > 0) {
+          const uint32_t idx = cnt[1 - wg] + uint32_t((n - 1) >> 1);
+          ok = __all_sync(0xFFFFFFFFu,
+                          wait_bar(pv_done + 8 * (1 - wg), idx & 1, abort_flag, a.status, 9));
           if (!ok) break;
         }
         tc_fence_after();
@@ -567,15 +652,15 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                          "r"(w2), "r"(w3)
                          : "memory");
           }
-          if (n > 0 && rescale) {
+          if (n >= 2 && rescale) {
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
-              tmem_ld32(t_lane + 2 * BN + 32 * c, o);
+              tmem_ld32(t_lane + col_o + 32 * c, o);
               tmem_wait_ld(o);
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(t_lane + 2 * BN + 32 * c, o);
+              tmem_st32(t_lane + col_o + 32 * c, o);
             }
             tmem_wait_st();
           }
@@ -583,45 +668,78 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);
-        if (lane == 0) VSA_TR(2 + warp, 16, g);
+        if (lane == 0) VSA_TR(quad + 4 * wg, 16, gn);
       }
       if (!ok) break;
-      // ---- epilogue
-      if (lane == 0) VSA_TR(2 + warp, 17, g);
-      ok = __all_sync(0xFFFFFFFFu, wait_bar(pv_done, (g - 1) & 1, abort_flag, a.status, 10));
+      // ---- epilogue: merge the two warpgroups' partial softmax states once
+      // the last PV of each warpgroup in this item is complete.
+      const uint32_t g_last = g + nk - 1;
+      if (lane == 0) VSA_TR(quad + 4 * wg, 17, g_last);
+      for (int w = 0; w < 2 && ok; ++w) {
+        const uint32_t nw = uint32_t((nk - w + 1) / 2);
+        if (nw > 0)
+          ok = __all_sync(0xFFFFFFFFu, wait_bar(pv_done + 8 * w, (cnt[w] + nw - 1) & 1, abort_flag,
+                                                a.status, 10));
+      }
       if (!ok) break;
+      cnt[0] += uint32_t((nk + 1) / 2);
+      cnt[1] += uint32_t(nk / 2);
       tc_fence_after();
+      s_m[wg * 128 + row] = m;
+      s_l[wg * 128 + row] = l;
+      if (*abort_flag) { ok = false; break; }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       if (rows_active) {
+        const float m0 = s_m[row], m1 = s_m[128 + row];
+        const float l0 = s_l[row], l1 = s_l[128 + row];
+        const float mm = fmaxf(m0, m1);
+        const float a0 = l0 > 0.f ? ex2(m0 - mm) : 0.f;
+        const float a1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
+        const float lt = a0 * l0 + a1 * l1;
         const bool live = row < q_live;
-        const float inv_l = live ? 1.0f / l : 0.f;
-        uint16_t* orow = a.out + (bh * a.n_pad + int64_t(i) * R + row) * D;
+        const float inv = live ? 1.0f / lt : 0.f;
+        const float f0 = a0 * inv, f1 = a1 * inv;
+        // warpgroup wg stores columns [wg*D/2, (wg+1)*D/2) of the row
+        uint16_t* orow = a.out + (bh * a.n_pad + int64_t(i) * R + row) * D + wg * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_lane + 2 * BN + 32 * c, o);
-          tmem_wait_ld(o);
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(t_lane + C::COL_O + wg * (D / 2) + 32 * c, o0);
+          tmem_ld32(t_lane + C::COL_O + D + wg * (D / 2) + 32 * c, o1);
+          tmem_wait_ld(o0);
+          tmem_wait_ld(o1);
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
-            v.y = pack_bf16(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
-            v.z = pack_bf16(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
-            v.w = pack_bf16(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
-            dst[q] = v;
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              // a warpgroup that saw no tile left its O columns unwritten
+              const float x0 = l0 > 0.f ? __uint_as_float(o0[8 * q + e]) * f0 : 0.f;
+              const float x1 = l1 > 0.f ? __uint_as_float(o1[8 * q + e]) * f1 : 0.f;
+              v[e] = x0 + x1;
+            }
+            uint4 u;
+            u.x = pack_bf16(v[0], v[1]);
+            u.y = pack_bf16(v[2], v[3]);
+            u.z = pack_bf16(v[4], v[5]);
+            u.w = pack_bf16(v[6], v[7]);
+            dst[q] = u;
           }
         }
-        if (a.lse != nullptr)
-          a.lse[bh * a.n_pad + int64_t(i) * R + row] = live ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
+        if (a.lse != nullptr && wg == 0)
+          a.lse[bh * a.n_pad + int64_t(i) * R + row] =
+              live ? (mm + __log2f(lt)) * 0.69314718055994531f : 0.f;
       }
       tc_fence_before();
       mbar_arrive(o_empty);
-      if (lane == 0) VSA_TR(2 + warp, 18, g);
+      if (lane == 0) VSA_TR(quad + 4 * wg, 18, g_last);
+      g += nk;
     }
   }
 
   // ---------------------------------------------------------------- teardown
-  if (lane == 0) VSA_TR(warp == kWarpTma ? 0 : (warp == kWarpMma ? 1 : 2 + warp), 19, 0);
+  if (lane == 0) VSA_TR(warp, 19, 0);
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
@@ -630,7 +748,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(C::TMEM_COLS)
                  : "memory");
-    if (lane == 0) VSA_TR(6, 20, 0);
+    if (lane == 0) VSA_TR(12, 20, 0);
   }
 }
 
@@ -671,9 +789,10 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows
 // Dynamic shared memory of one CTA.  At least 120 KB, so that two CTAs never
 // share an SM (each allocates its TMEM columns for its whole lifetime).
 template <int R, int D>
-size_t attn_smem_bytes(int T) {
+size_t attn_smem_bytes(int T, int k) {
   using C = Cfg<R, D>;
-  const size_t need = size_t(C::OFF_LISTS) + size_t((2 * T + 15) & ~15) + size_t(4) * T + 1024;
+  const size_t lists = size_t((T + 15) & ~15) + size_t(8) * ((k + 3) & ~3);
+  const size_t need = size_t(C::OFF_LISTS) + lists + 1024;
   return need < size_t(120 * 1024) ? size_t(120 * 1024) : need;
 }
 
@@ -681,7 +800,7 @@ template <int R, int D>
 vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, const void* v_t,
                      const int32_t* topk_idx, int64_t bh, int k, float scale, void* o_fine_t,
                      float* lse_t, cudaStream_t stream) {
-  const size_t smem = attn_smem_bytes<R, D>(p->n_tiles);
+  const size_t smem = attn_smem_bytes<R, D>(p->n_tiles, k);
   if (smem > 227 * 1024)
     return fail(VSA_ERR_UNSUPPORTED, "too many tiles for the sparse attention kernel's lists");
   const int64_t rows = bh * p->n_padded;
