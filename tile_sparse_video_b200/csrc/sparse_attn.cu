@@ -68,6 +68,30 @@ __device__ __forceinline__ void vsa_trace(int slot, unsigned int v) {
 #define VSA_TR(slot, code, g) ((void)0)
 #endif
 
+// Event timeline for debugging builds (-DVSA_TIMELINE): CTA 0 records
+// (role, event, tile, SM clock) into a device buffer, 4096 entries per role.
+#ifdef VSA_TIMELINE
+__device__ unsigned long long* vsa_tl_buf = nullptr;
+__device__ __forceinline__ void vsa_tl(int role, unsigned int ev, unsigned int tile,
+                                       unsigned int& k) {
+  if (vsa_tl_buf != nullptr && blockIdx.x == 0) {
+    if (k < 4096u) {
+      long long c;
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+      vsa_tl_buf[role * 4096 + k] = (unsigned long long)(c & 0xFFFFFFFFFFull) |
+                                    ((unsigned long long)(ev & 0xFFu) << 40) |
+                                    ((unsigned long long)(tile & 0xFFFFu) << 48);
+      ++k;
+    }
+  }
+}
+#define VSA_TL(role, ev, tile) vsa_tl((role), (ev), (tile), tl_k)
+#define VSA_TL_DECL unsigned int tl_k = 0
+#else
+#define VSA_TL(role, ev, tile) ((void)0)
+#define VSA_TL_DECL ((void)0)
+#endif
+
 // ---------------------------------------------------------------- PTX wrappers
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -219,6 +243,7 @@ struct AttnArgs {
   float* lse;                 // [BH, N_pad] or null
   unsigned int* status;       // device status word
   int T, n_p, k, n_items;
+  int two_p;                  // 1: one P tile per softmax warpgroup, 0: one shared P tile
   int64_t n_pad;
   float scale_log2;           // scale * log2(e)
 };
@@ -234,23 +259,38 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_V = OFF_K + NSK * TBYTES;
-  static constexpr int OFF_P = OFF_V + NSV * TBYTES;
-  static constexpr int OFF_BAR = OFF_P + PBYTES;
+  static constexpr int OFF_P = OFF_V + NSV * TBYTES;     // P_0, then P_1 when two_p
   // barriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV],
-  //           s_full[2], s_empty[2], p_full, pv_done[2], o_empty, drain
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 4 + 5;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag
-  static constexpr int OFF_ML = OFF_MISC + 16;           // float m[2][128], l[2][128]
-  static constexpr int OFF_LISTS = OFF_ML + 4 * 128 * 4;
+  //           s_full[2], s_empty[2], p_full[2], pv_done[2], o_full, o_empty, drain
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 11;
+  static constexpr int TAIL = NBAR * 8 + 16;              // barriers + tmem slot + abort flag
   static constexpr uint32_t TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256u : 512u;
   static constexpr uint32_t COL_S = 0;                   // S_w at COL_S + w*BN
   static constexpr uint32_t COL_O = 2 * BN;              // O_w at COL_O + w*D
   static constexpr uint32_t IDESC_QK = idesc_bf16(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, false, true);
+  // bytes after OFF_P: P tiles, barriers/misc, then the lists (blen uint8[T],
+  // two int32[k] kept-tile lists)
+  static size_t bytes(int two_p, int T, int k) {
+    return size_t(OFF_P) + size_t(two_p ? 2 : 1) * PBYTES + TAIL + size_t((T + 15) & ~15) +
+           size_t(8) * ((k + 3) & ~3);
+  }
 };
 
 __device__ __forceinline__ void record(unsigned int* status, unsigned int code, unsigned int info) {
   if (atomicCAS(status, 0u, code) == 0u) atomicExch(status + 1, info);
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
 // Bounded wait; false when the CTA is aborting (flag already set, or this wait
@@ -314,6 +354,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
                                          volatile int* abort_flag, int lane, int bh_np, int n_v) {
   using C = Cfg<R, D>;
   constexpr int kPrefetch = 4;
+  VSA_TL_DECL;
   uint32_t g = 0, q_issued = 0;
   int t = 0;
   bool ok = true;
@@ -341,10 +382,12 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
       }
       for (int n = 0; n < nk && ok; ++n, ++g) {
         const uint32_t s = g % NS;
+        VSA_TL(kIsK ? 3 : 4, 'x', g);
         if (g >= uint32_t(NS)) {
           ok = wait_bar(empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, kIsK ? 2 : 11);
           if (!ok) break;
         }
+        VSA_TL(kIsK ? 3 : 4, kIsK ? 'K' : 'V', g);
         const int j = (dense || n < a.n_p) ? n : s_list[n - a.n_p];
         const int row = int(row0 + int64_t(j) * R);
         mbar_expect_tx(full + 8 * s, C::TBYTES);
@@ -374,6 +417,33 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
   }
 }
 
+// Position in this CTA's stream of (item, tile) pairs.
+struct Cursor {
+  int item, t, n, nk;
+  uint32_t g;          // global tile counter
+  int64_t bh;
+  int i;
+};
+
+__device__ __forceinline__ void cursor_load(Cursor& c, const AttnArgs& a, int bh_np, int n_v) {
+  c.nk = 0;
+  if (c.item < a.n_items) {
+    decode_item(c.item, bh_np, a.n_p, n_v, c.bh, c.i);
+    c.nk = (c.i < a.n_p) ? a.T : a.n_p + a.k;
+  }
+}
+
+__device__ __forceinline__ void cursor_next(Cursor& c, const AttnArgs& a, int bh_np, int n_v) {
+  ++c.n;
+  ++c.g;
+  if (c.n == c.nk) {
+    c.n = 0;
+    ++c.t;
+    c.item += gridDim.x;
+    cursor_load(c, a, bh_np, n_v);
+  }
+}
+
 template <int R, int D>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -387,23 +457,26 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const uint32_t s_base = smem_u32(smem);
   const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V,
                  sP = s_base + C::OFF_P;
-  const uint32_t bar0 = s_base + C::OFF_BAR;
+  const int n_ptiles = a.two_p ? 2 : 1;
+  const uint32_t off_bar = C::OFF_P + n_ptiles * C::PBYTES;
+  const uint32_t bar0 = s_base + off_bar;
   const uint32_t q_full = bar0, q_empty = bar0 + 8;
   const uint32_t k_full = bar0 + 16, k_empty = k_full + 8 * NSK;
   const uint32_t v_full = k_empty + 8 * NSK, v_empty = v_full + 8 * NSV;
   const uint32_t s_full = v_empty + 8 * NSV, s_empty = s_full + 16;
-  // pv_done[w] completes once per PV of warpgroup w's tiles.  A waiter never
-  // lags a barrier by two phases (which would alias in the parity test): a
-  // warpgroup waits for the other's PV of tile n-1 only after it has seen the
-  // other's PV of tile n-3.
-  const uint32_t p_full = s_empty + 16, pv_done = p_full + 8, o_empty = pv_done + 16,
-                 drain = o_empty + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  float* s_m = reinterpret_cast<float*>(smem + C::OFF_ML);          // [2][128]
-  float* s_l = s_m + 2 * 128;                                        // [2][128]
-  uint8_t* s_blen = smem + C::OFF_LISTS;                             // [T]
-  int32_t* s_klist = reinterpret_cast<int32_t*>(smem + C::OFF_LISTS + ((a.T + 15) & ~15));
+  // p_full[w] / pv_done[w] complete once per tile of warpgroup w, o_full and
+  // o_empty once per item.  Every wait below targets a phase whose predecessor
+  // is already complete and whose successor cannot complete before the waiter
+  // has observed it, so the parity test never aliases.
+  const uint32_t p_full = s_empty + 16, pv_done = p_full + 16, o_full = pv_done + 16,
+                 o_empty = o_full + 8, drain = o_empty + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + off_bar + C::NBAR * 8 + 4);
+  // merge exchange of (m, l) lives in P_0 (free once an item's PVs are done)
+  float* s_m = reinterpret_cast<float*>(smem + C::OFF_P);         // [2][128]
+  float* s_l = s_m + 2 * 128;                                      // [2][128]
+  uint8_t* s_blen = smem + off_bar + C::TAIL;                      // [T]
+  int32_t* s_klist = reinterpret_cast<int32_t*>(s_blen + ((a.T + 15) & ~15));
   int32_t* s_vlist = s_klist + ((a.k + 3) & ~3);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -424,10 +497,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     for (int w = 0; w < 2; ++w) {
       mbar_init(s_full + 8 * w, 1);
       mbar_init(s_empty + 8 * w, 128);
+      mbar_init(p_full + 8 * w, 128);
+      mbar_init(pv_done + 8 * w, 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
-    mbar_init(pv_done + 8, 1);
+    mbar_init(o_full, 1);
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -459,80 +532,95 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                s_vlist, abort_flag, lane, bh_np, n_v);
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    // Order per item: S(0), S(1), then for every tile n: S(n+2), PV(n).
-    // Tile n belongs to softmax warpgroup w = n & 1 (S_w, O_w in TMEM); the
-    // single P buffer in shared memory is written in tile order.
+    // Two independent streams over this CTA's (item, tile) sequence, issued
+    // as soon as each is ready (non-blocking barrier tests, PV first):
+    //   S stream:  S_n = Q K_n^T into S_{n&1}; needs Q of the item, K_n, and
+    //              warpgroup n&1 done reading its previous S.
+    //   PV stream: O_{n&1} += P_n V_n; needs P_n written, V_n, and at an
+    //              item's first tile the previous item's epilogue done.
     if (lane == 0) {
-      uint32_t g = 0;            // global tile counter (K/V rings, p_full, pv_done)
-      uint32_t si[2] = {0, 0};   // S issues per warpgroup (s_full / s_empty phases)
-      int t = 0;
+      VSA_TL_DECL;
+      Cursor cs{int(blockIdx.x), 0, 0, 0, 0u, 0, 0};
+      cursor_load(cs, a, bh_np, n_v);
+      Cursor cp = cs;
+      uint32_t si[2] = {0, 0};   // S issues into S_w
+      uint32_t pc[2] = {0, 0};   // PV issues from warpgroup w
+      unsigned long long t_idle = 0;
       bool ok = true;
-      auto issue_s = [&](uint32_t gt, int w) -> bool {
-        const uint32_t s = gt % NSK;
-        VSA_TR(11, 6, gt);
-        if (!wait_bar(k_full + 8 * s, (gt / NSK) & 1, abort_flag, a.status, 6)) return false;
-        if (si[w] > 0 && !wait_bar(s_empty + 8 * w, (si[w] - 1) & 1, abort_flag, a.status, 7))
-          return false;
-        tc_fence_after();
+      while (cp.nk > 0 && ok) {
+        bool progressed = false;
+        // ---- PV stream
+        if (cp.g < cs.g) {
+          const int w = cp.n & 1;
+          const uint32_t sv = cp.g % NSV;
+          if ((cp.n != 0 || cp.t == 0 || mbar_test(o_empty, (cp.t - 1) & 1)) &&
+              mbar_test(p_full + 8 * w, pc[w] & 1) && mbar_test(v_full + 8 * sv, (cp.g / NSV) & 1)) {
+            VSA_TL(0, 'P', cp.g);
+            tc_fence_after();
+            const uint32_t sp = sP + (a.two_p ? w * C::PBYTES : 0);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(sQ + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
-          const uint64_t bd =
-              sdesc_sw128(sK + s * C::TBYTES + (ks / 4) * BN * 128 + (ks % 4) * 32, 16, 1024);
-          umma_bf16(tmem + C::COL_S + w * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full + 8 * w);
-        umma_commit(k_empty + 8 * s);
-        ++si[w];
-        VSA_TR(11, 8, gt);
-        return true;
-      };
-      auto issue_pv = [&](uint32_t gt, int n) -> bool {
-        const int w = n & 1;
-        if (n == 0 && t > 0 && !wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) return false;
-        VSA_TR(11, 10, gt);
-        if (!wait_bar(p_full, gt & 1, abort_flag, a.status, 4)) return false;
-        const uint32_t sv = gt % NSV;
-        if (!wait_bar(v_full + 8 * sv, (gt / NSV) & 1, abort_flag, a.status, 12)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t ad = sdesc_sw128(sP + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sV + sv * C::TBYTES + ks * 16 * 128, BN * 128, 1024);
-          umma_bf16(tmem + C::COL_O + w * D, ad, bd, C::IDESC_PV, (n >= 2 || ks > 0) ? 1u : 0u);
-        }
-        umma_commit(pv_done + 8 * w);
-        umma_commit(v_empty + 8 * sv);
-        VSA_TR(11, 11, gt);
-        return true;
-      };
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
-        int64_t bh;
-        int i;
-        decode_item(item, bh_np, a.n_p, n_v, bh, i);
-        const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
-        VSA_TR(11, 5, g);
-        if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
-        tc_fence_after();
-        for (int n = 0; n < 2 && n < nk && ok; ++n) ok = issue_s(g + n, n);
-        if (ok && nk <= 2) umma_commit(q_empty);
-        for (int n = 0; n < nk && ok; ++n) {
-          if (n + 2 < nk) {
-            ok = issue_s(g + n + 2, n & 1);
-            if (ok && n + 3 == nk) umma_commit(q_empty);
+            for (int ks = 0; ks < BN / 16; ++ks) {
+              const uint64_t ad = sdesc_sw128(sp + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(sV + sv * C::TBYTES + ks * 16 * 128, BN * 128, 1024);
+              umma_bf16(tmem + C::COL_O + w * D, ad, bd, C::IDESC_PV, (cp.n >= 2 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(pv_done + 8 * w);
+            umma_commit(v_empty + 8 * sv);
+            if (cp.n == cp.nk - 1) umma_commit(o_full);
+            ++pc[w];
+            cursor_next(cp, a, bh_np, n_v);
+            progressed = true;
           }
-          if (ok) ok = issue_pv(g + n, n);
         }
-        g += nk;
+        // ---- S stream
+        if (cs.nk > 0) {
+          const int w = cs.n & 1;
+          const uint32_t s = cs.g % NSK;
+          if ((cs.n != 0 || mbar_test(q_full, cs.t & 1)) &&
+              mbar_test(k_full + 8 * s, (cs.g / NSK) & 1) &&
+              (si[w] == 0 || mbar_test(s_empty + 8 * w, (si[w] - 1) & 1))) {
+            VSA_TL(0, 'S', cs.g);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint64_t ad = sdesc_sw128(sQ + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
+              const uint64_t bd =
+                  sdesc_sw128(sK + s * C::TBYTES + (ks / 4) * BN * 128 + (ks % 4) * 32, 16, 1024);
+              umma_bf16(tmem + C::COL_S + w * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(s_full + 8 * w);
+            umma_commit(k_empty + 8 * s);
+            ++si[w];
+            if (cs.n == cs.nk - 1) umma_commit(q_empty);
+            cursor_next(cs, a, bh_np, n_v);
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_idle = 0;
+        } else {
+          // bounded idle time, as for every other wait
+          const unsigned long long now = globaltimer();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (*abort_flag) {
+            ok = false;
+          } else if (now - t_idle > kWaitLimitNs) {
+            *abort_flag = 1;
+            record(a.status, kStatusTimeout, 6);
+            ok = false;
+          }
+        }
       }
       // Drain: wait until every MMA issued above has completed.
       umma_commit(drain);
       wait_bar_drain(drain, 0);
-      VSA_TR(11, 12, g);
+      VSA_TR(11, 12, cp.g);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warpgroups
+    VSA_TL_DECL;
     const int wg = warp >> 2;                            // 0 or 1
     const int quad = warp & 3;
     const bool rows_active = (R == 128) || (quad < 2);
@@ -540,6 +628,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
     const uint32_t col_s = C::COL_S + wg * BN;
     const uint32_t col_o = C::COL_O + wg * D;
+    const uint32_t my_p = sP + (a.two_p ? wg * C::PBYTES : 0);
     uint32_t g = 0;              // global tile counter (trace only)
     uint32_t cnt[2] = {0, 0};    // tiles of each warpgroup in earlier items
     uint32_t cw = 0;             // tiles processed by this warpgroup (s_full phases)
@@ -551,9 +640,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       decode_item(item, bh_np, a.n_p, n_v, bh, i);
       const bool dense = i < a.n_p;
       const int nk = dense ? a.T : a.n_p + a.k;
-      // Group barrier of the 256 softmax threads.  A warp that sees the abort
-      // flag leaves instead: the others then also see it before they could
-      // block here (they wait on the same mbarrier phases first).
+      // Group barrier of the 256 softmax threads (it also keeps the next P
+      // write behind the previous item's (m, l) exchange in P_0).  A warp that
+      // sees the abort flag leaves instead: the others then also see it before
+      // they could block here (they wait on the same mbarrier phases first).
       if (*abort_flag) { ok = false; break; }
       asm volatile("bar.sync 1, 256;" ::: "memory");
       for (int x = threadIdx.x; x < nk; x += 256) {
@@ -567,9 +657,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       float m = -INFINITY, l = 0.f;
       for (int n = wg; n < nk; n += 2, ++cw) {
         const uint32_t gn = g + n;
+        (void)gn;
         if (lane == 0) VSA_TR(quad + 4 * wg, 13, gn);
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'a', gn);
         ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * wg, cw & 1, abort_flag, a.status, 8));
         if (!ok) break;
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 's', gn);
         tc_fence_after();
         uint32_t r[BN / 32][32];
         if (rows_active) {
@@ -626,15 +719,18 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           l = l * alpha + sum;
           m = m_new;
         }
-        // The previous tile's PV (the other warpgroup's) must be done before
-        // the shared P buffer is overwritten; it also orders this
-        // warpgroup's own earlier PV into O_w before the rescale below.  For
-        // n = 0 the previous item's epilogue already waited for all its PVs.
+        // Before P_n is written (and O_w possibly rescaled): with one P tile per
+        // warpgroup, this warpgroup's own PV of tile n-2 must be done; with one
+        // shared P tile, the other warpgroup's PV of tile n-1 (which orders our
+        // own n-2 before it).  At an item's first tiles the previous item's
+        // epilogue already waited for every PV.
         if (lane == 0) VSA_TR(quad + 4 * wg, 15, gn);
-        if (n > 0) {
-          const uint32_t idx = cnt[1 - wg] + uint32_t((n - 1) >> 1);
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'w', gn);
+        if (a.two_p ? n >= 2 : n >= 1) {
+          const int ow = a.two_p ? wg : 1 - wg;
+          const uint32_t idx = cnt[ow] + uint32_t(a.two_p ? (n - 2) >> 1 : (n - 1) >> 1);
           ok = __all_sync(0xFFFFFFFFu,
-                          wait_bar(pv_done + 8 * (1 - wg), idx & 1, abort_flag, a.status, 9));
+                          wait_bar(pv_done + 8 * ow, idx & 1, abort_flag, a.status, 9));
           if (!ok) break;
         }
         tc_fence_after();
@@ -647,7 +743,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             const uint32_t w2 = pack_bf16(__uint_as_float(r[c][e + 4]), __uint_as_float(r[c][e + 5]));
             const uint32_t w3 = pack_bf16(__uint_as_float(r[c][e + 6]), __uint_as_float(r[c][e + 7]));
             const uint32_t addr =
-                sP + (c8 / 8) * kBM * 128 + row * 128 + ((uint32_t(c8 % 8) ^ uint32_t(row & 7)) << 4);
+                my_p + (c8 / 8) * kBM * 128 + row * 128 + ((uint32_t(c8 % 8) ^ uint32_t(row & 7)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w0), "r"(w1),
                          "r"(w2), "r"(w3)
                          : "memory");
@@ -667,20 +763,17 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(p_full + 8 * wg);
         if (lane == 0) VSA_TR(quad + 4 * wg, 16, gn);
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'W', gn);
       }
       if (!ok) break;
       // ---- epilogue: merge the two warpgroups' partial softmax states once
-      // the last PV of each warpgroup in this item is complete.
+      // every PV of the item is complete (o_full).
       const uint32_t g_last = g + nk - 1;
+      (void)g_last;
       if (lane == 0) VSA_TR(quad + 4 * wg, 17, g_last);
-      for (int w = 0; w < 2 && ok; ++w) {
-        const uint32_t nw = uint32_t((nk - w + 1) / 2);
-        if (nw > 0)
-          ok = __all_sync(0xFFFFFFFFu, wait_bar(pv_done + 8 * w, (cnt[w] + nw - 1) & 1, abort_flag,
-                                                a.status, 10));
-      }
+      ok = __all_sync(0xFFFFFFFFu, wait_bar(o_full, t & 1, abort_flag, a.status, 10));
       if (!ok) break;
       cnt[0] += uint32_t((nk + 1) / 2);
       cnt[1] += uint32_t(nk / 2);
@@ -788,11 +881,15 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows
 
 // Dynamic shared memory of one CTA.  At least 120 KB, so that two CTAs never
 // share an SM (each allocates its TMEM columns for its whole lifetime).
+// Dynamic shared memory of one CTA (+1 KB so the kernel can align its base to
+// 1024 bytes), at least 120 KB so that two CTAs never share an SM (each holds
+// its TMEM columns for its whole lifetime).  Two P tiles when they fit.
+constexpr size_t kMaxSmem = 227 * 1024;
 template <int R, int D>
-size_t attn_smem_bytes(int T, int k) {
+size_t attn_smem_bytes(int T, int k, int* two_p) {
   using C = Cfg<R, D>;
-  const size_t lists = size_t((T + 15) & ~15) + size_t(8) * ((k + 3) & ~3);
-  const size_t need = size_t(C::OFF_LISTS) + lists + 1024;
+  *two_p = (C::bytes(1, T, k) + 1024 <= kMaxSmem) ? 1 : 0;
+  const size_t need = C::bytes(*two_p, T, k) + 1024;
   return need < size_t(120 * 1024) ? size_t(120 * 1024) : need;
 }
 
@@ -800,8 +897,9 @@ template <int R, int D>
 vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, const void* v_t,
                      const int32_t* topk_idx, int64_t bh, int k, float scale, void* o_fine_t,
                      float* lse_t, cudaStream_t stream) {
-  const size_t smem = attn_smem_bytes<R, D>(p->n_tiles, k);
-  if (smem > 227 * 1024)
+  int two_p = 0;
+  const size_t smem = attn_smem_bytes<R, D>(p->n_tiles, k, &two_p);
+  if (smem > kMaxSmem)
     return fail(VSA_ERR_UNSUPPORTED, "too many tiles for the sparse attention kernel's lists");
   const int64_t rows = bh * p->n_padded;
   CUtensorMap mq, mk, mv;
@@ -821,6 +919,7 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   a.n_p = p->n_prefix_tiles;
   a.k = k;
   a.n_pad = p->n_padded;
+  a.two_p = two_p;
   a.scale_log2 = scale * 1.4426950408889634f;
   const int64_t items = bh * p->n_tiles;
   if (items >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "too many work items");
