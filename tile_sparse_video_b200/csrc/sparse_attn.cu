@@ -15,10 +15,11 @@
 //   warp 8  (TMA K)  loads Q once per item and K_j per kept tile into a K ring,
 //                    and prefetches K/V tiles a few steps ahead into L2.
 //   warp 9  (TMA V)  loads V_j into its own ring (V is needed later than K).
-//   warp 10 (MMA)    one lane issues S_n = Q K_n^T (M=128, N=R, K=D) into the
-//                    TMEM S buffer of warpgroup n & 1, and O_w += P_n V_n
-//                    (M=128, N=D, K=R) once P_n is written; order per item:
-//                    S0, S1, then S_{n+2}, PV_n for every n.
+//   warp 10 (MMA S)  one lane issues S_n = Q K_n^T (M=128, N=R, K=D) into the
+//                    TMEM S buffer of warpgroup n & 1 as soon as K_n is in and
+//                    the warpgroup has read its previous S.
+//   warp 11 (MMA PV) one lane issues O_w += P_n V_n (M=128, N=D, K=R) as soon
+//                    as P_n is written; the two issuers run independently.
 //   warps 0-7        two softmax warpgroups; warpgroup w takes the tiles
 //                    n = w (mod 2) of an item (a split of the key set inside the
 //                    CTA).  Thread = query row = TMEM lane: it loads its S row,
@@ -30,6 +31,9 @@
 //                    moved.  The epilogue merges the two partial (m, l, O)
 //                    states and stores bf16 rows (and the LSE).
 // TMEM columns: S_0 [0,R), S_1 [R,2R), O_0 [2R,2R+D), O_1 [2R+D,2R+2D).
+// P tiles live in shared memory: one per warpgroup when they fit (then a
+// warpgroup only waits for its own PV of tile n-2 before rewriting its P),
+// else one shared tile written in tile order.
 // With R = 64 the MMA still runs with M = 128 (rows 64..127 of the Q box are
 // the next rows of the tensor, or zero past its end); their results are never
 // stored and the warps of those rows skip the softmax work.
@@ -48,9 +52,16 @@ namespace vsa {
 namespace {
 
 constexpr int kBM = 128;                 // MMA M (query rows per item)
-constexpr int kThreadsAttn = 352;        // 8 softmax warps + TMA K + TMA V + MMA
-constexpr int kWarpTmaK = 8, kWarpTmaV = 9, kWarpMma = 10;
+constexpr int kThreadsAttn = 384;        // 8 softmax warps + TMA K + TMA V + MMA S + MMA PV
+constexpr int kWarpTmaK = 8, kWarpTmaV = 9, kWarpMmaS = 10, kWarpMmaPV = 11;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+
+// K ring depth for 128-row tiles (a tuning knob: 2 stages leave room for one
+// P tile per softmax warpgroup, which measured faster on B200 than 3 stages
+// with one shared P tile: 27.4 vs 32.2 ms at the 104k-token Veda layer).
+#ifndef VSA_NSK128
+#define VSA_NSK128 2
+#endif
 
 // Progress trace for debugging builds (-DVSA_TRACE): each role of each CTA
 // publishes its position in the pipeline to a host-visible buffer (16 slots
@@ -251,7 +262,7 @@ struct AttnArgs {
 template <int R, int D>
 struct Cfg {
   static constexpr int BN = R;
-  static constexpr int NSK = (R == 128) ? 2 : 4;        // K ring stages
+  static constexpr int NSK = (R == 128) ? VSA_NSK128 : 4;   // K ring stages
   static constexpr int NSV = (R == 128) ? 2 : 4;        // V ring stages
   static constexpr int QBYTES = kBM * D * 2;
   static constexpr int TBYTES = BN * D * 2;              // one K (or V) tile
@@ -261,8 +272,9 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + NSK * TBYTES;
   static constexpr int OFF_P = OFF_V + NSV * TBYTES;     // P_0, then P_1 when two_p
   // barriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV],
-  //           s_full[2], s_empty[2], p_full[2], pv_done[2], o_full, o_empty, drain
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 11;
+  //           s_full[2], s_empty[2], p_full[2], pv_done[2], o_full, o_empty, drain,
+  //           drain2
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 12;
   static constexpr int TAIL = NBAR * 8 + 16;              // barriers + tmem slot + abort flag
   static constexpr uint32_t TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256u : 512u;
   static constexpr uint32_t COL_S = 0;                   // S_w at COL_S + w*BN
@@ -279,18 +291,6 @@ struct Cfg {
 
 __device__ __forceinline__ void record(unsigned int* status, unsigned int code, unsigned int info) {
   if (atomicCAS(status, 0u, code) == 0u) atomicExch(status + 1, info);
-}
-
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
 }
 
 // Bounded wait; false when the CTA is aborting (flag already set, or this wait
@@ -417,33 +417,6 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
   }
 }
 
-// Position in this CTA's stream of (item, tile) pairs.
-struct Cursor {
-  int item, t, n, nk;
-  uint32_t g;          // global tile counter
-  int64_t bh;
-  int i;
-};
-
-__device__ __forceinline__ void cursor_load(Cursor& c, const AttnArgs& a, int bh_np, int n_v) {
-  c.nk = 0;
-  if (c.item < a.n_items) {
-    decode_item(c.item, bh_np, a.n_p, n_v, c.bh, c.i);
-    c.nk = (c.i < a.n_p) ? a.T : a.n_p + a.k;
-  }
-}
-
-__device__ __forceinline__ void cursor_next(Cursor& c, const AttnArgs& a, int bh_np, int n_v) {
-  ++c.n;
-  ++c.g;
-  if (c.n == c.nk) {
-    c.n = 0;
-    ++c.t;
-    c.item += gridDim.x;
-    cursor_load(c, a, bh_np, n_v);
-  }
-}
-
 template <int R, int D>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -469,7 +442,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   // is already complete and whose successor cannot complete before the waiter
   // has observed it, so the parity test never aliases.
   const uint32_t p_full = s_empty + 16, pv_done = p_full + 16, o_full = pv_done + 16,
-                 o_empty = o_full + 8, drain = o_empty + 8;
+                 o_empty = o_full + 8, drain = o_empty + 8, drain2 = drain + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + off_bar + C::NBAR * 8 + 4);
   // merge exchange of (m, l) lives in P_0 (free once an item's PVs are done)
@@ -503,6 +476,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     mbar_init(o_full, 1);
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
+    mbar_init(drain2, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -511,7 +485,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == kWarpMma) {
+  if (warp == kWarpMmaS) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(C::TMEM_COLS)
@@ -530,92 +504,91 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   } else if (warp == kWarpTmaV) {
     producer<R, D, NSV, false>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full, q_empty,
                                s_vlist, abort_flag, lane, bh_np, n_v);
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
-    // Two independent streams over this CTA's (item, tile) sequence, issued
-    // as soon as each is ready (non-blocking barrier tests, PV first):
-    //   S stream:  S_n = Q K_n^T into S_{n&1}; needs Q of the item, K_n, and
-    //              warpgroup n&1 done reading its previous S.
-    //   PV stream: O_{n&1} += P_n V_n; needs P_n written, V_n, and at an
-    //              item's first tile the previous item's epilogue done.
+  } else if (warp == kWarpMmaS) {
+    // ------------------------------------------------------------ S issuer
+    // S_n = Q K_n^T into S_{n&1} (tile n of an item belongs to softmax
+    // warpgroup n & 1); needs Q of the item, K_n, and the warpgroup done
+    // reading its previous S.  Runs ahead across items.
     if (lane == 0) {
       VSA_TL_DECL;
-      Cursor cs{int(blockIdx.x), 0, 0, 0, 0u, 0, 0};
-      cursor_load(cs, a, bh_np, n_v);
-      Cursor cp = cs;
-      uint32_t si[2] = {0, 0};   // S issues into S_w
-      uint32_t pc[2] = {0, 0};   // PV issues from warpgroup w
-      unsigned long long t_idle = 0;
+      uint32_t g = 0, si[2] = {0, 0};
+      int t = 0;
       bool ok = true;
-      while (cp.nk > 0 && ok) {
-        bool progressed = false;
-        // ---- PV stream
-        if (cp.g < cs.g) {
-          const int w = cp.n & 1;
-          const uint32_t sv = cp.g % NSV;
-          if ((cp.n != 0 || cp.t == 0 || mbar_test(o_empty, (cp.t - 1) & 1)) &&
-              mbar_test(p_full + 8 * w, pc[w] & 1) && mbar_test(v_full + 8 * sv, (cp.g / NSV) & 1)) {
-            VSA_TL(0, 'P', cp.g);
-            tc_fence_after();
-            const uint32_t sp = sP + (a.two_p ? w * C::PBYTES : 0);
-#pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks) {
-              const uint64_t ad = sdesc_sw128(sp + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sV + sv * C::TBYTES + ks * 16 * 128, BN * 128, 1024);
-              umma_bf16(tmem + C::COL_O + w * D, ad, bd, C::IDESC_PV, (cp.n >= 2 || ks > 0) ? 1u : 0u);
-            }
-            umma_commit(pv_done + 8 * w);
-            umma_commit(v_empty + 8 * sv);
-            if (cp.n == cp.nk - 1) umma_commit(o_full);
-            ++pc[w];
-            cursor_next(cp, a, bh_np, n_v);
-            progressed = true;
-          }
-        }
-        // ---- S stream
-        if (cs.nk > 0) {
-          const int w = cs.n & 1;
-          const uint32_t s = cs.g % NSK;
-          if ((cs.n != 0 || mbar_test(q_full, cs.t & 1)) &&
-              mbar_test(k_full + 8 * s, (cs.g / NSK) & 1) &&
-              (si[w] == 0 || mbar_test(s_empty + 8 * w, (si[w] - 1) & 1))) {
-            VSA_TL(0, 'S', cs.g);
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint64_t ad = sdesc_sw128(sQ + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
-              const uint64_t bd =
-                  sdesc_sw128(sK + s * C::TBYTES + (ks / 4) * BN * 128 + (ks % 4) * 32, 16, 1024);
-              umma_bf16(tmem + C::COL_S + w * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
-            }
-            umma_commit(s_full + 8 * w);
-            umma_commit(k_empty + 8 * s);
-            ++si[w];
-            if (cs.n == cs.nk - 1) umma_commit(q_empty);
-            cursor_next(cs, a, bh_np, n_v);
-            progressed = true;
-          }
-        }
-        if (progressed) {
-          t_idle = 0;
-        } else {
-          // bounded idle time, as for every other wait
-          const unsigned long long now = globaltimer();
-          if (t_idle == 0) {
-            t_idle = now;
-          } else if (*abort_flag) {
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+        int64_t bh;
+        int i;
+        decode_item(item, bh_np, a.n_p, n_v, bh, i);
+        const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
+        if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
+        for (int n = 0; n < nk; ++n, ++g) {
+          const int w = n & 1;
+          const uint32_t s = g % NSK;
+          if (!wait_bar(k_full + 8 * s, (g / NSK) & 1, abort_flag, a.status, 6)) { ok = false; break; }
+          if (si[w] > 0 && !wait_bar(s_empty + 8 * w, (si[w] - 1) & 1, abort_flag, a.status, 7)) {
             ok = false;
-          } else if (now - t_idle > kWaitLimitNs) {
-            *abort_flag = 1;
-            record(a.status, kStatusTimeout, 6);
-            ok = false;
+            break;
           }
+          VSA_TL(0, 'S', g);
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ad = sdesc_sw128(sQ + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
+            const uint64_t bd =
+                sdesc_sw128(sK + s * C::TBYTES + (ks / 4) * BN * 128 + (ks % 4) * 32, 16, 1024);
+            umma_bf16(tmem + C::COL_S + w * BN, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full + 8 * w);
+          umma_commit(k_empty + 8 * s);
+          ++si[w];
+          if (n == nk - 1) umma_commit(q_empty);
         }
       }
       // Drain: wait until every MMA issued above has completed.
       umma_commit(drain);
       wait_bar_drain(drain, 0);
-      VSA_TR(11, 12, cp.g);
+    }
+    __syncwarp();
+  } else if (warp == kWarpMmaPV) {
+    // ------------------------------------------------------------ PV issuer
+    // O_{n&1} += P_n V_n; needs P_n written, V_n, and at an item's first tile
+    // the previous item's epilogue done reading O.
+    if (lane == 0) {
+      VSA_TL_DECL;
+      uint32_t g = 0, pc[2] = {0, 0};
+      int t = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+        int64_t bh;
+        int i;
+        decode_item(item, bh_np, a.n_p, n_v, bh, i);
+        const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
+        for (int n = 0; n < nk; ++n, ++g) {
+          const int w = n & 1;
+          const uint32_t sv = g % NSV;
+          if (n == 0 && t > 0 && !wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) {
+            ok = false;
+            break;
+          }
+          if (!wait_bar(p_full + 8 * w, pc[w] & 1, abort_flag, a.status, 4)) { ok = false; break; }
+          if (!wait_bar(v_full + 8 * sv, (g / NSV) & 1, abort_flag, a.status, 12)) { ok = false; break; }
+          VSA_TL(5, 'P', g);
+          tc_fence_after();
+          const uint32_t sp = sP + (a.two_p ? w * C::PBYTES : 0);
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t ad = sdesc_sw128(sp + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sV + sv * C::TBYTES + ks * 16 * 128, BN * 128, 1024);
+            umma_bf16(tmem + C::COL_O + w * D, ad, bd, C::IDESC_PV, (n >= 2 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(pv_done + 8 * w);
+          umma_commit(v_empty + 8 * sv);
+          if (n == nk - 1) umma_commit(o_full);
+          ++pc[w];
+        }
+      }
+      umma_commit(drain2);
+      wait_bar_drain(drain2, 0);
+      VSA_TR(11, 12, g);
     }
     __syncwarp();
   } else {
@@ -835,7 +808,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   if (lane == 0) VSA_TR(warp, 19, 0);
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == kWarpMmaS) {
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
