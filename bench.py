@@ -43,6 +43,11 @@ from tile_sparse_video_b200.inputs import VEDA_104K, WORKLOADS, Workload, make_i
 METRIC = "ms/layer & kept-FLOP TFLOP/s (% bf16 peak) at 104k tokens, 90% tile sparsity"
 UNIT = "ms/layer"
 
+# DRAM bytes (read + write) of one full-size sparse_attn launch, from the ncu
+# capture summarised in profiles/sparse_attn_veda_h8.md (8 heads, scaled by
+# 42/8), valid only for the kernel source it was taken on.
+ATTN_TRAFFIC = {"source_sha256_16": "0db0ee252c210a2a", "bytes": 23.42e9}
+
 
 # ----------------------------------------------------------------- accounting
 
@@ -66,6 +71,18 @@ def geometry_counts(w: Workload, n_p: int, T: int, k: int) -> dict:
         # attention: Q, K, V read once and O written once
         attn_bytes=4.0 * BH * N_pad * D * 2,
     )
+
+
+def attn_traffic():
+    """Measured DRAM traffic of the attention kernel, or None once its source
+    has changed since the counters were taken."""
+    import hashlib
+    src = os.path.join(ROOT, "tile_sparse_video_b200", "csrc", "sparse_attn.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return ATTN_TRAFFIC["bytes"] if h == ATTN_TRAFFIC["source_sha256_16"] else None
 
 
 def load_peaks() -> dict:
@@ -308,7 +325,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
                      "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),
                      "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16 burst)",
-                     "traffic": None},
+                     "traffic": attn_traffic()},
         "e2e": {"value": round(e2e_elapsed / (max(e2e_steps, 1) * world), 3) if e2e_steps else None,
                 "unit": UNIT,
                 "h2d_bytes_per_step": int(sum(host[n].numel() * 2 for n in "qkvg")),
