@@ -213,6 +213,8 @@ vsa_status vsa_coarse_topk(vsa_plan p, const void* q_t, const void* k_t, const v
   if (topk_score != nullptr && !aligned16(topk_score))
     return fail(VSA_ERR_INVALID_ARG, "topk_score is not 16-byte aligned");
   if (!std::isfinite(scale)) return fail(VSA_ERR_INVALID_ARG, "scale is not finite");
+  if (p->n_tiles > 4096)
+    return fail(VSA_ERR_UNSUPPORTED, "coarse attention supports at most 4096 tiles");
   size_t need = 0;
   vsa_workspace_size(p, B, H, D, k, &need);
   if (ws == nullptr || ws_bytes < need)

@@ -1,25 +1,28 @@
 // Coarse attention over pooled tiles and the per-head top-k of video key tiles.
 //
-// One CTA of kQB warps handles kQB query tiles of one (b, h); warp w owns query
-// tile i0 + w.  Pooled key (then value) tiles are staged through shared memory
-// in chunks of 32, shared by the kQB warps.  Per warp:
-//   1. s[j] = scale * <qbar_i, kbar_j> for all T key tiles (lane = key tile of
-//      the chunk; the staging buffer has a padded row stride so the 32 lanes
-//      read 32 different banks), kept in shared memory in fp32;
-//   2. o_coarse_i = sum_j softmax(s)_j vbar_j (lane = 4 output columns);
-//   3. for a video query tile, a radix select over the 32-bit order-preserving
-//      image of s[j], j in [n_p, T): four 8-bit digit passes with a per-warp
-//      256-bin histogram find the k-th largest key K*; then one ascending sweep
-//      over j keeps every key > K* and the lowest-index keys == K* until k are
-//      kept, which writes the result already sorted by tile index and breaks
-//      ties towards the lower index.  Bit-exact for given fp32 scores.
+// One CTA handles QB = 8*RW query tiles of one (b, h); warp w owns the RW
+// query tiles i0 + w*RW ...  The work is three register-tiled fp32 passes:
+//   1. scores: s[r][j] = scale * <qbar_r, kbar_j> for all T key tiles.  Key
+//      tiles are staged 64 at a time in shared memory (padded rows, so the 32
+//      lanes read 32 banks); lane l computes keys l and l+32 for the warp's RW
+//      rows, reading the RW query values of one dimension as one broadcast
+//      vector load (q is stored transposed).  Scores stay in shared memory.
+//   2. top-k (video query tiles only): a radix select over the 32-bit
+//      order-preserving image of s[r][j], j in [n_p, T): four 8-bit digit
+//      passes with a per-warp 256-bin histogram find the k-th largest key K*;
+//      one ascending sweep over j keeps every key > K* and the lowest-index
+//      keys == K* until k are kept, which writes the result already sorted by
+//      tile index with ties broken towards the lower index.  Bit-exact for
+//      given fp32 scores.
+//   3. softmax and o_coarse = sum_j p[r][j] vbar_j: the scores become
+//      probabilities in place, value tiles are staged 64 at a time, lane l
+//      accumulates columns l, l+32, ... for the warp's RW rows.
 #include "vsa_internal.h"
 
 namespace vsa {
 namespace {
 
-constexpr int kQB = 8;                 // query tiles (= warps) per CTA
-constexpr int kKC = 32;                // key tiles per staged chunk
+constexpr int kKC = 64;                // key / value tiles per staged chunk
 constexpr int kMaxTiles = 4096;        // bound on T (shared-memory budget)
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -28,178 +31,329 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kQB * 32) coarse_topk_kernel(
+template <int RW>
+struct QVec;
+template <>
+struct QVec<1> {
+  __device__ static void load(const float* p, float (&q)[1]) { q[0] = p[0]; }
+};
+template <>
+struct QVec<2> {
+  __device__ static void load(const float* p, float (&q)[2]) {
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    q[0] = v.x;
+    q[1] = v.y;
+  }
+};
+template <>
+struct QVec<4> {
+  __device__ static void load(const float* p, float (&q)[4]) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    q[0] = v.x;
+    q[1] = v.y;
+    q[2] = v.z;
+    q[3] = v.w;
+  }
+};
+
+// Asynchronous copy of nj rows of a [*, D] fp32 matrix into a shared-memory
+// stage with a padded row stride (D + 4 floats: rows stay 16-byte aligned and
+// 128-bit reads of 8 consecutive rows hit 8 distinct bank groups).  One
+// commit group per call; the caller waits with cp_async_wait<N>.
+template <int D, int kWarps>
+__device__ __forceinline__ void stage_rows_async(float* stage, const float* src, int nj) {
+  constexpr int kStride = D + 4;
+  constexpr int kVecPerRow = D / 4;
+  constexpr int kPerThread = (kKC * kVecPerRow) / (kWarps * 32);
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int idx = threadIdx.x + u * kWarps * 32;
+    if (idx < nj * kVecPerRow) {
+      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(
+          stage + (idx / kVecPerRow) * kStride + (idx % kVecPerRow) * 4));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + idx * 4)
+                   : "memory");
+    }
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int D, int NW, int RW>
+__global__ void __launch_bounds__(NW * 32) coarse_topk_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ vbar,
     int T, int n_p, float scale, int k, float* __restrict__ o_coarse, int32_t* __restrict__ topk_idx,
     float* __restrict__ topk_score) {
-  constexpr int kStride = D + 1;
-  extern __shared__ float smem[];
-  float* stage = smem;                           // [kKC][kStride]
-  float* qrow = stage + kKC * kStride;           // [kQB][D]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(qrow + kQB * D);   // [kQB][256]
-  float* srow = reinterpret_cast<float*>(hist + kQB * 256);       // [kQB][Tpad]
-  const int Tpad = (T + 31) & ~31;
+  constexpr int kWarps = NW;
+  constexpr int QB = kWarps * RW;
+  constexpr int kStride = D + 4;
+  extern __shared__ float4 smem4[];
+  float* smem = reinterpret_cast<float*>(smem4);
+  float* qT = smem;                                   // [D][QB]
+  float* stage0 = qT + D * QB;                        // [2][kKC][kStride]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(stage0 + 2 * kKC * kStride);  // [kWarps][256]
+  float* sc = reinterpret_cast<float*>(hist + kWarps * 256);            // [QB][Tpad]
+  const int Tpad = (T + 3) & ~3;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bh = blockIdx.y;
-  const int i = blockIdx.x * kQB + warp;
-  const bool active = i < T;
+  const int i0 = blockIdx.x * QB;
   const float* kb = kbar + bh * int64_t(T) * D;
   const float* vb = vbar + bh * int64_t(T) * D;
-  float* s = srow + warp * Tpad;
 
-  for (int d = lane; d < D; d += 32) qrow[warp * D + d] = active ? qbar[(bh * T + i) * D + d] : 0.f;
-
-  // 1. scores
-  for (int j0 = 0; j0 < T; j0 += kKC) {
-    __syncthreads();
-    const int nj = min(kKC, T - j0);
-    for (int x = threadIdx.x; x < nj * D; x += kQB * 32) {
-      const int jj = x / D, d = x % D;
-      stage[jj * kStride + d] = kb[int64_t(j0 + jj) * D + d];
+  {
+    // transposed query block: qT[d][r]; batched loads as in stage_rows
+    constexpr int kNVec = QB * D / 4;
+    constexpr int kVec = (kNVec + kWarps * 32 - 1) / (kWarps * 32);
+    const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * T + i0) * D);
+    float4 v[kVec];
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int idx = threadIdx.x + u * kWarps * 32;
+      v[u] = (idx < kNVec && i0 + idx / (D / 4) < T) ? __ldg(q4 + idx)
+                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
-    if (active && lane < nj) {
-      float acc = 0.f;
-      const float* kr = stage + lane * kStride;
-      const float* qr = qrow + warp * D;
-#pragma unroll 16
-      for (int d = 0; d < D; ++d) acc = fmaf(qr[d], kr[d], acc);
-      s[j0 + lane] = scale * acc;
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int idx = threadIdx.x + u * kWarps * 32;
+      if (idx >= kNVec) continue;
+      const int r = idx / (D / 4), d = (idx % (D / 4)) * 4;
+      qT[(d + 0) * QB + r] = v[u].x;
+      qT[(d + 1) * QB + r] = v[u].y;
+      qT[(d + 2) * QB + r] = v[u].z;
+      qT[(d + 3) * QB + r] = v[u].w;
     }
   }
-  __syncwarp();
 
-  // 2. softmax and o_coarse
-  float m = -INFINITY;
-  for (int j = lane; j < T; j += 32) m = fmaxf(m, s[j]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-  float l = 0.f;
-  for (int j = lane; j < T; j += 32) l += __expf(s[j] - m);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-  float acc[D / 32];
-#pragma unroll
-  for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
-  for (int j0 = 0; j0 < T; j0 += kKC) {
-    __syncthreads();
+  // ---- 1. scores (double-buffered key stages)
+  const int n_chunks = (T + kKC - 1) / kKC;
+  stage_rows_async<D, NW>(stage0, kb, min(kKC, T));
+  for (int c = 0; c < n_chunks; ++c) {
+    const int j0 = c * kKC;
     const int nj = min(kKC, T - j0);
-    for (int x = threadIdx.x; x < nj * D; x += kQB * 32) {
-      const int jj = x / D, d = x % D;
-      stage[jj * kStride + d] = vb[int64_t(j0 + jj) * D + d];
+    float* stage = stage0 + (c & 1) * kKC * kStride;
+    if (c + 1 < n_chunks) {
+      stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, kb + int64_t(j0 + kKC) * D,
+                          min(kKC, T - j0 - kKC));
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
-    if (active) {
-      for (int jj = 0; jj < nj; ++jj) {
-        const float p = __expf(s[j0 + jj] - m);
+    float acc[RW][2];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(p, stage[jj * kStride + lane + 32 * c], acc[c]);
+    for (int r = 0; r < RW; ++r) acc[r][0] = acc[r][1] = 0.f;
+    const float4* k0 = reinterpret_cast<const float4*>(stage + lane * kStride);
+    const float4* k1 = reinterpret_cast<const float4*>(stage + (lane + 32) * kStride);
+    const float* qw = qT + warp * RW;
+#pragma unroll 4
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      const float4 a0 = k0[d4], a1 = k1[d4];
+      const float a0v[4] = {a0.x, a0.y, a0.z, a0.w};
+      const float a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float q[RW];
+        QVec<RW>::load(qw + (4 * d4 + e) * QB, q);
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+          acc[r][0] = fmaf(q[r], a0v[e], acc[r][0]);
+          acc[r][1] = fmaf(q[r], a1v[e], acc[r][1]);
+        }
       }
     }
-  }
-  if (!active) return;
-  {
-    const float inv = 1.0f / l;
-    float* oc = o_coarse + (bh * T + i) * D;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) oc[lane + 32 * c] = acc[c] * inv;
+    for (int r = 0; r < RW; ++r) {
+      float* row = sc + (warp * RW + r) * Tpad + j0;
+      if (lane < nj) row[lane] = scale * acc[r][0];
+      if (lane + 32 < nj) row[lane + 32] = scale * acc[r][1];
+    }
+    __syncthreads();     // stage (c & 1) is refilled two chunks later
   }
 
-  // 3. top-k over video key tiles (video query tiles only)
-  if (i < n_p || k <= 0) return;
+  // ---- 2. top-k over video key tiles (video query tiles only), raw scores
   const int n_v = T - n_p;
   uint32_t* h = hist + warp * 256;
-  uint32_t prefix = 0u, mask = 0u;
-  int remaining = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int r = 0; r < RW; ++r) {
+    const int i = i0 + warp * RW + r;
+    if (i >= T || i < n_p || k <= 0) continue;
+    const float* s = sc + (warp * RW + r) * Tpad;
+    uint32_t prefix = 0u, mask = 0u;
+    int remaining = k;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
 #pragma unroll
-    for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
-    __syncwarp();
-    for (int j = n_p + lane; j < T; j += 32) {
-      const uint32_t key = order_key(s[j]);
-      if ((key & mask) == prefix) atomicAdd(h + ((key >> shift) & 255u), 1u);
-    }
-    __syncwarp();
-    // lane L holds bins 255-8L .. 248-8L (lane 0 = highest digits)
-    uint32_t cnt = 0;
+      for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
+      __syncwarp();
+      for (int jb = n_p; jb < T; jb += 32) {
+        const int j = jb + lane;
+        const uint32_t key = j < T ? order_key(s[j]) : 0u;
+        const bool in = j < T && (key & mask) == prefix;
+        // lanes with the same digit add once (scores cluster in few bins)
+        const uint32_t bin = in ? ((key >> shift) & 255u) : 256u;
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+        if (in && (__ffs(peers) - 1) == lane) atomicAdd(h + bin, uint32_t(__popc(peers)));
+      }
+      __syncwarp();
+      // lane L holds bins 255-8L .. 248-8L (lane 0 = highest digits)
+      uint32_t cnt = 0;
 #pragma unroll
-    for (int b = 0; b < 8; ++b) cnt += h[255 - 8 * lane - b];
-    uint32_t incl = cnt;
+      for (int b = 0; b < 8; ++b) cnt += h[255 - 8 * lane - b];
+      uint32_t incl = cnt;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, incl >= uint32_t(remaining));
-    const int L = __ffs(ballot) - 1;
-    uint32_t digit = 0;
-    int rem_new = 0;
-    if (lane == L) {
-      uint32_t run = incl - cnt;                      // keys with a higher digit
-      for (int b = 0; b < 8; ++b) {
-        const uint32_t bin = 255 - 8 * L - b;
-        if (run + h[bin] >= uint32_t(remaining)) {
-          digit = bin;
-          rem_new = remaining - int(run);
-          break;
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, incl >= uint32_t(remaining));
+      const int L = __ffs(ballot) - 1;
+      uint32_t digit = 0;
+      int rem_new = 0;
+      if (lane == L) {
+        uint32_t run = incl - cnt;                      // keys with a higher digit
+        for (int b = 0; b < 8; ++b) {
+          const uint32_t bin = 255 - 8 * L - b;
+          if (run + h[bin] >= uint32_t(remaining)) {
+            digit = bin;
+            rem_new = remaining - int(run);
+            break;
+          }
+          run += h[bin];
         }
-        run += h[bin];
+      }
+      digit = __shfl_sync(0xFFFFFFFFu, digit, L);
+      remaining = __shfl_sync(0xFFFFFFFFu, rem_new, L);
+      prefix |= digit << shift;
+      mask |= 255u << shift;
+      __syncwarp();
+    }
+    // prefix = K*, remaining = number of keys equal to K* to keep (lowest j first)
+    int32_t* out_idx = topk_idx + ((bh * n_v) + (i - n_p)) * int64_t(k);
+    float* out_s = topk_score ? topk_score + ((bh * n_v) + (i - n_p)) * int64_t(k) : nullptr;
+    int pos = 0, eq_seen = 0;
+    for (int base = n_p; base < T; base += 32) {
+      const int j = base + lane;
+      const bool valid = j < T;
+      const float sv = valid ? s[j] : 0.f;
+      const uint32_t key = valid ? order_key(sv) : 0u;
+      const bool gt = valid && key > prefix;
+      const bool eq = valid && key == prefix;
+      const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
+      const int eq_rank = eq_seen + __popc(eqb & lt_mask);
+      const bool sel = gt || (eq && eq_rank < remaining);
+      const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
+      if (sel) {
+        const int o = pos + __popc(selb & lt_mask);
+        out_idx[o] = j;
+        if (out_s) out_s[o] = sv;
+      }
+      pos += __popc(selb);
+      eq_seen += __popc(eqb);
+    }
+  }
+
+  // ---- 3. softmax in place, then o_coarse
+  float inv_l[RW];
+#pragma unroll
+  for (int r = 0; r < RW; ++r) {
+    float* s = sc + (warp * RW + r) * Tpad;
+    float m = -INFINITY;
+    for (int j = lane; j < T; j += 32) m = fmaxf(m, s[j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    float l = 0.f;
+    for (int j = lane; j < T; j += 32) {
+      const float p = __expf(s[j] - m);
+      s[j] = p;
+      l += p;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
+    inv_l[r] = 1.0f / l;
+  }
+  float acc[RW][D / 32];
+#pragma unroll
+  for (int r = 0; r < RW; ++r)
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) acc[r][c] = 0.f;
+  __syncthreads();
+  stage_rows_async<D, NW>(stage0, vb, min(kKC, T));
+  for (int c = 0; c < n_chunks; ++c) {
+    const int j0 = c * kKC;
+    const int nj = min(kKC, T - j0);
+    const float* stage = stage0 + (c & 1) * kKC * kStride;
+    if (c + 1 < n_chunks) {
+      stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, vb + int64_t(j0 + kKC) * D,
+                          min(kKC, T - j0 - kKC));
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    for (int jj = 0; jj < nj; ++jj) {
+      float v[D / 32];
+#pragma unroll
+      for (int c2 = 0; c2 < D / 32; ++c2) v[c2] = stage[jj * kStride + lane + 32 * c2];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const float p = sc[(warp * RW + r) * Tpad + j0 + jj];
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2) acc[r][c2] = fmaf(p, v[c2], acc[r][c2]);
       }
     }
-    digit = __shfl_sync(0xFFFFFFFFu, digit, L);
-    remaining = __shfl_sync(0xFFFFFFFFu, rem_new, L);
-    prefix |= digit << shift;
-    mask |= 255u << shift;
-    __syncwarp();
+    __syncthreads();
   }
-  // prefix = K*, remaining = number of keys equal to K* to keep (lowest j first)
-  int32_t* out_idx = topk_idx + ((bh * n_v) + (i - n_p)) * int64_t(k);
-  float* out_s = topk_score ? topk_score + ((bh * n_v) + (i - n_p)) * int64_t(k) : nullptr;
-  int pos = 0, eq_seen = 0;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int base = n_p; base < T; base += 32) {
-    const int j = base + lane;
-    const bool valid = j < T;
-    const float sv = valid ? s[j] : 0.f;
-    const uint32_t key = valid ? order_key(sv) : 0u;
-    const bool gt = valid && key > prefix;
-    const bool eq = valid && key == prefix;
-    const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
-    const int eq_rank = eq_seen + __popc(eqb & lt_mask);
-    const bool sel = gt || (eq && eq_rank < remaining);
-    const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
-    if (sel) {
-      const int o = pos + __popc(selb & lt_mask);
-      out_idx[o] = j;
-      if (out_s) out_s[o] = sv;
-    }
-    pos += __popc(selb);
-    eq_seen += __popc(eqb);
+#pragma unroll
+  for (int r = 0; r < RW; ++r) {
+    const int i = i0 + warp * RW + r;
+    if (i >= T) continue;
+    float* oc = o_coarse + (bh * T + i) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) oc[lane + 32 * c] = acc[r][c] * inv_l[r];
   }
 }
 
-template <int D>
+template <int D, int NW, int RW>
 size_t coarse_smem_bytes(int T) {
-  const int Tpad = (T + 31) & ~31;
-  return sizeof(float) * (size_t(kKC) * (D + 1) + size_t(kQB) * D + size_t(kQB) * 256 +
-                          size_t(kQB) * Tpad);
+  const int Tpad = (T + 3) & ~3;
+  return sizeof(float) * (size_t(D) * NW * RW + size_t(2) * kKC * (D + 4) + size_t(NW) * 256 +
+                          size_t(NW) * RW * Tpad);
+}
+
+template <int D, int NW, int RW>
+cudaError_t launch_coarse_cfg(const float* qbar, const float* kbar, const float* vbar, int64_t bh,
+                              int T, int n_p, float scale, int k, float* o_coarse,
+                              int32_t* topk_idx, float* topk_score, cudaStream_t stream) {
+  const size_t smem = coarse_smem_bytes<D, NW, RW>(T);
+  cudaError_t e = cudaFuncSetAttribute(coarse_topk_kernel<D, NW, RW>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  constexpr int QB = NW * RW;
+  const dim3 grid(unsigned((T + QB - 1) / QB), unsigned(bh), 1);
+  coarse_topk_kernel<D, NW, RW><<<grid, NW * 32, smem, stream>>>(
+      qbar, kbar, vbar, T, n_p, scale, k, o_coarse, topk_idx, topk_score);
+  return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_coarse_d(const float* qbar, const float* kbar, const float* vbar, int64_t bh,
                             int T, int n_p, float scale, int k, float* o_coarse, int32_t* topk_idx,
                             float* topk_score, cudaStream_t stream) {
-  const size_t smem = coarse_smem_bytes<D>(T);
-  cudaError_t e = cudaFuncSetAttribute(coarse_topk_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  const dim3 grid(unsigned((T + kQB - 1) / kQB), unsigned(bh), 1);
-  coarse_topk_kernel<D><<<grid, kQB * 32, smem, stream>>>(qbar, kbar, vbar, T, n_p, scale, k,
-                                                          o_coarse, topk_idx, topk_score);
-  return cudaGetLastError();
+  // 16 warps per CTA (one CTA fills an SM's shared memory), and as many query
+  // tiles per CTA as the score rows leave room for
+  if (T <= 960)
+    return launch_coarse_cfg<D, 16, 2>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
+                                       topk_score, stream);
+  if (T <= 1920)
+    return launch_coarse_cfg<D, 16, 1>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
+                                       topk_score, stream);
+  return launch_coarse_cfg<D, 8, 1>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
+                                    topk_score, stream);
 }
 
 }  // namespace

@@ -113,53 +113,59 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const uint4* __restrict_
   }
 }
 
-__device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + __expf(-g)); }
+// sigmoid(g) = (1 + tanh(g/2)) / 2: one hardware tanh instead of exp + reciprocal.
+__device__ __forceinline__ float sigmoidf_(float g) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * g));
+  return fmaf(0.5f, t, 0.5f);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
-// out = o_fine + sigmoid(g) * o_coarse[tile].  kNatural: destination rows are
-// natural tokens n (source row untile[n]); otherwise padded rows r (pad -> 0).
+// out = o_fine + sigmoid(g) * o_coarse[tile].  The walk is over the padded
+// (tiled) rows, so o_fine and g are read contiguously; with kNatural the live
+// row r is written to natural token row_src[r] (whole 16-byte chunks of a
+// 128/256-byte row), otherwise to row r with pad rows set to 0.
 template <int kCpr, bool kNatural>
 __global__ void __launch_bounds__(kThreads) gate_combine_kernel(
     const uint4* __restrict__ o_fine, const uint4* __restrict__ gate,
-    const float* __restrict__ o_coarse, uint4* __restrict__ out, const int32_t* __restrict__ map,
+    const float* __restrict__ o_coarse, uint4* __restrict__ out, const int32_t* __restrict__ row_src,
     int64_t n_tokens, int64_t n_padded, int R, int T) {
   const int64_t bh = blockIdx.y;
   const uint4* of = o_fine + bh * n_padded * kCpr;
   const uint4* gg = gate + bh * n_padded * kCpr;
   const float* oc = o_coarse + bh * int64_t(T) * (kCpr * 8);
-  const int64_t dst_rows = kNatural ? n_tokens : n_padded;
-  uint4* d = out + bh * dst_rows * kCpr;
-  const int64_t total = dst_rows * kCpr;
+  uint4* d = out + bh * (kNatural ? n_tokens : n_padded) * kCpr;
+  const int64_t total = n_padded * kCpr;
   const int64_t stride = int64_t(gridDim.x) * kThreads;
-  for (int64_t c0 = int64_t(blockIdx.x) * kThreads + threadIdx.x; c0 < total;
-       c0 += stride * kUnroll) {
-    uint4 a[kUnroll], g[kUnroll];
-    int64_t row[kUnroll];
+  constexpr int kU = 2 * kUnroll;
+  for (int64_t c0 = int64_t(blockIdx.x) * kThreads + threadIdx.x; c0 < total; c0 += stride * kU) {
+    // The data loads do not wait for row_src (pad rows are readable memory),
+    // so every load of the step is in flight at once.
+    uint4 a[kU], g[kU];
+    int32_t src[kU];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < kU; ++u) {
       const int64_t c = c0 + u * stride;
-      row[u] = -1;
+      src[u] = -2;
       if (c < total) {
-        const int32_t m = __ldg(map + c / kCpr);
-        row[u] = kNatural ? int64_t(m) : (m >= 0 ? c / kCpr : -1);
-        if (row[u] >= 0) {
-          a[u] = ldg_nc(of + row[u] * kCpr + (c % kCpr));
-          g[u] = ldg_nc(gg + row[u] * kCpr + (c % kCpr));
-        }
+        src[u] = __ldg(row_src + c / kCpr);
+        a[u] = ldg_nc(of + c);
+        g[u] = ldg_nc(gg + c);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < kU; ++u) {
       const int64_t c = c0 + u * stride;
-      if (c >= total) continue;
+      if (src[u] == -2) continue;                 // past the end
+      const int64_t r = c / kCpr;
+      const int col = int(c % kCpr);
       uint4 res = make_uint4(0u, 0u, 0u, 0u);
-      if (row[u] >= 0) {
-        const int col = int(c % kCpr);
-        const float4* cp = reinterpret_cast<const float4*>(oc + (row[u] / R) * (kCpr * 8) + col * 8);
+      if (src[u] >= 0) {
+        const float4* cp = reinterpret_cast<const float4*>(oc + (r / R) * (kCpr * 8) + col * 8);
         const float4 c0v = __ldg(cp), c1v = __ldg(cp + 1);
         const float cv[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
         const uint32_t aw[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
@@ -169,11 +175,16 @@ __global__ void __launch_bounds__(kThreads) gate_combine_kernel(
         for (int i = 0; i < 4; ++i) {
           const float f0 = __uint_as_float(aw[i] << 16), f1 = __uint_as_float(aw[i] & 0xFFFF0000u);
           const float g0 = __uint_as_float(gw[i] << 16), g1 = __uint_as_float(gw[i] & 0xFFFF0000u);
-          ow[i] = pack_bf16x2(f0 + sigmoidf_(g0) * cv[2 * i], f1 + sigmoidf_(g1) * cv[2 * i + 1]);
+          ow[i] = pack_bf16x2(fmaf(sigmoidf_(g0), cv[2 * i], f0), fmaf(sigmoidf_(g1), cv[2 * i + 1], f1));
         }
         res = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      } else if (kNatural) {
+        continue;                                  // pad rows have no natural token
       }
-      d[c] = res;
+      if (kNatural)
+        d[int64_t(src[u]) * kCpr + col] = res;
+      else
+        d[c] = res;
     }
   }
 }
@@ -232,16 +243,17 @@ cudaError_t launch_gate_combine(const uint16_t* o_fine_t, const uint16_t* gate_t
   const uint4* of = reinterpret_cast<const uint4*>(o_fine_t);
   const uint4* g = reinterpret_cast<const uint4*>(gate_t);
   uint4* o = reinterpret_cast<uint4*>(out);
+  (void)untile;
   if (D == 128) {
     if (out_natural)
-      gate_combine_kernel<16, true><<<grid, kThreads, 0, stream>>>(of, g, o_coarse, o, untile,
+      gate_combine_kernel<16, true><<<grid, kThreads, 0, stream>>>(of, g, o_coarse, o, row_src,
                                                                    n_tokens, n_padded, R, T);
     else
       gate_combine_kernel<16, false><<<grid, kThreads, 0, stream>>>(of, g, o_coarse, o, row_src,
                                                                     n_tokens, n_padded, R, T);
   } else {
     if (out_natural)
-      gate_combine_kernel<8, true><<<grid, kThreads, 0, stream>>>(of, g, o_coarse, o, untile,
+      gate_combine_kernel<8, true><<<grid, kThreads, 0, stream>>>(of, g, o_coarse, o, row_src,
                                                                   n_tokens, n_padded, R, T);
     else
       gate_combine_kernel<8, false><<<grid, kThreads, 0, stream>>>(of, g, o_coarse, o, row_src,
