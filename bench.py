@@ -3,8 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one whole layer (permute Q/K/V/G, pool + coarse attention + top-k,
-block-sparse attention, gated combine into natural order) on the 104,704-token
+One step = one whole layer (permute Q/K/V, pool + coarse attention + top-k,
+block-sparse attention with the gated combine fused into its epilogue, writing
+natural order) on the 104,704-token
 Veda workload: 42 heads x 128, 128-token key tiles (4x8x4), 2 prefix tiles and
 816 video tiles, 90 % sparsity (82 kept video tiles per query tile).
 
@@ -62,14 +63,14 @@ def geometry_counts(w: Workload, n_p: int, T: int, k: int) -> dict:
         pair_fraction=pairs / T ** 2,
         kept_flop=4.0 * D * R * R * pairs * BH,            # QK^T and PV over kept tile pairs
         dense_flop=4.0 * N * N * D * BH,
-        # bytes: read N real rows, write N_pad padded rows, four tensors
-        permute_bytes=4.0 * BH * (N + N_pad) * D * 2,
+        # bytes: read N real rows, write N_pad padded rows; Q, K and V (the gate
+        # is read in natural order by the fused attention + combine)
+        permute_bytes=3.0 * BH * (N + N_pad) * D * 2,
         # pool reads the live rows of Q, K, V
         pool_bytes=3.0 * BH * N * D * 2,
-        # combine (natural order) reads o_fine and g rows of live tokens, writes the output
-        combine_bytes=3.0 * BH * N * D * 2,
-        # attention: Q, K, V read once and O written once
-        attn_bytes=4.0 * BH * N_pad * D * 2,
+        # attention + combine: Q, K, V read once, the gate read and the output
+        # written once (natural order)
+        attn_bytes=3.0 * BH * N_pad * D * 2 + 2.0 * BH * N * D * 2,
     )
 
 
@@ -215,13 +216,13 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     q, kk, v, g = (inp[n].to(dev) for n in "qkvg")
     layer = vsa.Layer(plan, w.B, w.H, w.D, k)
     stream = torch.cuda.current_stream()
-    launches_per_step = 8          # 4 permutes, pool, coarse+top-k, sparse attention, combine
+    launches_per_step = 6          # 3 permutes, pool, coarse+top-k, attention with fused combine
 
     def step(ev=None):
         p = plan
         if ev is not None:
             ev[0].record(stream)
-        for src, dst in ((q, layer.q_t), (kk, layer.k_t), (v, layer.v_t), (g, layer.g_t)):
+        for src, dst in ((q, layer.q_t), (kk, layer.k_t), (v, layer.v_t)):
             vsa.vsa_permute(p, src, dst)
         if ev is not None:
             ev[1].record(stream)
@@ -229,13 +230,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                             o_coarse=layer.o_coarse, topk_idx=layer.topk_idx)
         if ev is not None:
             ev[2].record(stream)
-        vsa.vsa_sparse_attn(p, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k, layer.scale,
-                            out=layer.o_fine_t)
+        vsa.vsa_sparse_attn_combine(p, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k, g,
+                                    layer.o_coarse, layer.scale, out=layer.out)
         if ev is not None:
             ev[3].record(stream)
-        vsa.vsa_gate_combine(p, layer.o_fine_t, layer.g_t, layer.o_coarse, natural=True, out=layer.out)
-        if ev is not None:
-            ev[4].record(stream)
 
     def barrier():
         if world > 1:
@@ -245,7 +243,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         step()
     vsa.vsa_sync_status(plan)
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
@@ -261,7 +259,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     barrier()
     vsa.vsa_sync_status(plan)
     elapsed = t_start.elapsed_time(t_end)
-    parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in events])
+    parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in events])
     part_ms = parts.mean(axis=0)
     if world > 1:
         t = torch.tensor([elapsed], device=dev)
@@ -316,12 +314,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "kept_tflops": round(acct["kept_flop"] * layers / (elapsed * 1e-3) / 1e12, 2),
         "dense_equiv_tflops": round(acct["dense_flop"] * layers / (elapsed * 1e-3) / 1e12, 2),
         "pct_bf16_peak_layer": round(100 * acct["kept_flop"] * layers / (elapsed * 1e-3) / 1e12 / peaks["bf16"], 2),
-        "kernels_ms": {"permute_x4": round(float(part_ms[0]), 4),
+        "kernels_ms": {"permute_q_k_v": round(float(part_ms[0]), 4),
                        "pool_coarse_topk": round(float(part_ms[1]), 4),
-                       "sparse_attn": round(attn_ms, 4), "gate_combine": round(float(part_ms[3]), 4)},
-        "kernels_hbm_gbs": {"permute_x4": round(acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9, 1),
-                            "gate_combine": round(acct["combine_bytes"] / (part_ms[3] * 1e-3) / 1e9, 1)},
-        "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
+                       "sparse_attn_combine": round(attn_ms, 4)},
+        "kernels_hbm_gbs": {"permute_q_k_v": round(acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9, 1)},
+        "roofline": {"kernel": "sparse_attn_combine", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
                      "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),
                      "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16 burst)",

@@ -174,6 +174,20 @@ vsa_status vsa_sparse_attn(vsa_plan plan, const void* q_t, const void* k_t, cons
                            void* o_fine_t, float* lse_t, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* Steps 4 and 5 fused: the attention of vsa_sparse_attn, with the gated combine
+ * of vsa_gate_combine applied in its epilogue to the fp32 attention output (no
+ * bf16 rounding of o_fine in between) and the result written in natural token
+ * order: out[b,h,n,:] = o_fine + sigmoid(gate[b,h,n,:]) * o_coarse[b,h,tile(n),:].
+ * gate: bf16 [B,H,N,D] in NATURAL order (the to_gate_compress projection split
+ * into heads, no permute needed); o_coarse: fp32 [B,H,T,D] from
+ * vsa_coarse_topk; out: bf16 [B,H,N,D]; lse_t as for vsa_sparse_attn.  Sources
+ * as for the two unfused calls; fusing them saves the o_fine round trip
+ * through HBM, the permute of the gate and one launch. */
+vsa_status vsa_sparse_attn_combine(vsa_plan plan, const void* q_t, const void* k_t,
+                                   const void* v_t, const int32_t* topk_idx, int B, int H, int D,
+                                   int k, float scale, const void* gate, const float* o_coarse,
+                                   void* out, float* lse_t, void* stream);
+
 /* Step 5.  out = o_fine + sigmoid(g) * o_coarse[tile(row)], element-wise over
  * D, fp32 arithmetic, bf16 round-to-nearest-even store.  o_fine_t and gate_t:
  * bf16 [B,H,N_pad,D] (the gate is the bias-free to_gate_compress projection of

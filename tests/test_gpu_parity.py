@@ -61,16 +61,22 @@ def _keep(plan, w):
 
 
 def _run(w: Workload):
+    """The unfused chain (every intermediate visible), plus the fused
+    attention + combine entry point on the same inputs."""
     inp = make_inputs(w)
     plan = vsa.Plan(w.prefix, w.grid, w.tile)
     k = _keep(plan, w)
     q, kk, v, g = (inp[x].cuda() for x in "qkvg")
-    layer = vsa.Layer(plan, w.B, w.H, w.D, k)
+    layer = vsa.Layer(plan, w.B, w.H, w.D, k, fused=False)
     out = layer(q, kk, v, g)
     _, _, scores, _ = vsa.vsa_coarse_topk(plan, layer.q_t, layer.k_t, layer.v_t, k, want_scores=True)
     _, lse = vsa.vsa_sparse_attn(plan, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k, want_lse=True)
     out_t = vsa.vsa_gate_combine(plan, layer.o_fine_t, layer.g_t, layer.o_coarse, natural=False)
+    fused, lse_f = vsa.vsa_sparse_attn_combine(plan, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k,
+                                               g, layer.o_coarse, want_lse=True)
     vsa.vsa_sync_status(plan)
+    assert torch.equal(lse_f, lse)
+    layer.fused_out = fused
     return inp, plan, k, layer, out, scores, lse, out_t
 
 
@@ -102,8 +108,9 @@ def test_layer_parity(w):
     live = p.row_src >= 0
     np.testing.assert_allclose(f64(lse)[..., live], ref["lse"][..., live], atol=2e-3)
     assert np.all(f64(lse)[..., ~live] == 0)
-    # step 5: combine, both output layouts
+    # step 5: combine, both output layouts, and the fused attention + combine
     assert_close(f64(out), ref["out"], what="out")
+    assert_close(f64(layer.fused_out), ref["out"], what="fused out")
     assert_close(f64(out_t), ref["out_t"], what="out_t")
     assert np.all(f64(out_t)[..., ~live, :] == 0)
     assert torch.equal(vsa.vsa_unpermute(plan, out_t), out)
@@ -113,7 +120,7 @@ def test_keep_all_equals_dense_attention():
     """k = every video tile: the fine output is plain dense attention over all
     real tokens (torch's own routine, fp32 on the GPU)."""
     w = _w("dense_check", 1, 2, 128, (40, 70), (4, 8, 8), (4, 4, 4), sparsity=0.0)
-    inp, plan, k, layer, *_ = _run(w)
+    inp, plan, k, layer, *_ = _run(w)      # unfused layer: o_fine_t is kept
     assert k == plan.n_video_tiles
     o_nat = vsa.vsa_unpermute(plan, layer.o_fine_t)
     q, kk, v = (inp[x].cuda().float() for x in "qkv")
@@ -127,8 +134,9 @@ def _sampled(w: Workload, heads, n_video_samples, seed):
     k = _keep(plan, w)
     dev = torch.device("cuda")
     q, kk, v, g = (inp[x].to(dev) for x in "qkvg")
-    layer = vsa.Layer(plan, w.B, w.H, w.D, k)
+    layer = vsa.Layer(plan, w.B, w.H, w.D, k)          # the fused chain the benchmark times
     out = layer(q, kk, v, g)
+    o_fine_t, _ = vsa.vsa_sparse_attn(plan, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k)
     vsa.vsa_sync_status(plan)
     p = O.plan(w.prefix, w.grid, w.tile)
     rng = np.random.default_rng(seed)
@@ -147,7 +155,7 @@ def _sampled(w: Workload, heads, n_video_samples, seed):
                 p.n_prefix_tiles + rng.choice(p.n_video_tiles, n_video_samples, replace=False))
             tiles.append(p.n_tiles - 1)
             out_bh = out[b, h].cpu()
-            o_fine_bh = layer.o_fine_t[b, h].cpu()
+            o_fine_bh = o_fine_t[b, h].cpu()
             for i in sorted(set(tiles)):
                 kept = idx[i - p.n_prefix_tiles] if i >= p.n_prefix_tiles else None
                 o, _ = O.fine_tile(q_t, k_t, v_t, p, i, O.key_tiles(p, i, kept), scale)

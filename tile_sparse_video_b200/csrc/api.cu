@@ -255,7 +255,31 @@ vsa_status vsa_sparse_attn(vsa_plan p, const void* q_t, const void* k_t, const v
   if (!(scale > 0.0f) || !std::isfinite(scale))
     return fail(VSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   return launch_sparse_attn(p, q_t, k_t, v_t, topk_idx, int64_t(B) * H, D, k, scale, o_fine_t,
-                            lse_t, static_cast<cudaStream_t>(stream));
+                            lse_t, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_sparse_attn_combine(vsa_plan p, const void* q_t, const void* k_t, const void* v_t,
+                                   const int32_t* topk_idx, int B, int H, int D, int k, float scale,
+                                   const void* gate, const float* o_coarse, void* out,
+                                   float* lse_t, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  VSA_TRY(check_k(p, k));
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(q_t, "q_t"));
+  VSA_TRY(check_ptr(k_t, "k_t"));
+  VSA_TRY(check_ptr(v_t, "v_t"));
+  VSA_TRY(check_ptr(gate, "gate"));
+  VSA_TRY(check_ptr(o_coarse, "o_coarse"));
+  VSA_TRY(check_ptr(out, "out"));
+  const int n_v = p->n_tiles - p->n_prefix_tiles;
+  if (k > 0 && n_v > 0) VSA_TRY(check_ptr(topk_idx, "topk_idx"));
+  if (lse_t != nullptr && !aligned16(lse_t))
+    return fail(VSA_ERR_INVALID_ARG, "lse_t is not 16-byte aligned");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  return launch_sparse_attn(p, q_t, k_t, v_t, topk_idx, int64_t(B) * H, D, k, scale, out, lse_t,
+                            gate, o_coarse, static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_gate_combine(vsa_plan p, const void* o_fine_t, const void* gate_t,

@@ -250,14 +250,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 struct AttnArgs {
   const int32_t* topk;        // [BH, n_v, k]
   const int32_t* block_len;   // [T]
-  uint16_t* out;              // bf16 [BH, N_pad, D]
+  uint16_t* out;              // bf16 [BH, N_pad, D], or [BH, N, D] natural when fused
   float* lse;                 // [BH, N_pad] or null
   unsigned int* status;       // device status word
+  // fused gated combine (step 5) in the epilogue: out[row_src[r]] =
+  // o_fine[r] + sigmoid(gate[row_src[r]]) * o_coarse[tile(r)]
+  const uint16_t* gate;       // bf16 [BH, N, D] natural order, or null (unfused)
+  const float* o_coarse;      // fp32 [BH, T, D]
+  const int32_t* row_src;     // [N_pad] padded row -> token, -1 for a pad row
   int T, n_p, k, n_items;
   int two_p;                  // 1: one P tile per softmax warpgroup, 0: one shared P tile
-  int64_t n_pad;
+  int64_t n_pad, n_tok;
   float scale_log2;           // scale * log2(e)
 };
+
+// sigmoid(g) = (1 + tanh(g/2)) / 2 with the hardware tanh.
+__device__ __forceinline__ float sigmoid_fast(float g) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * g));
+  return fmaf(0.5f, t, 0.5f);
+}
 
 template <int R, int D>
 struct Cfg {
@@ -765,8 +777,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         const bool live = row < q_live;
         const float inv = live ? 1.0f / lt : 0.f;
         const float f0 = a0 * inv, f1 = a1 * inv;
-        // warpgroup wg stores columns [wg*D/2, (wg+1)*D/2) of the row
-        uint16_t* orow = a.out + (bh * a.n_pad + int64_t(i) * R + row) * D + wg * (D / 2);
+        // warpgroup wg stores columns [wg*D/2, (wg+1)*D/2) of the row; fused:
+        // the gated combine, written to the row's natural token position
+        const bool fused = a.gate != nullptr;
+        const int64_t tok = (fused && live) ? int64_t(__ldg(a.row_src + int64_t(i) * R + row)) : 0;
+        uint16_t* orow = fused ? a.out + (bh * a.n_tok + tok) * D + wg * (D / 2)
+                               : a.out + (bh * a.n_pad + int64_t(i) * R + row) * D + wg * (D / 2);
+        const uint16_t* grow = fused ? a.gate + (bh * a.n_tok + tok) * D + wg * (D / 2) : nullptr;
+        const float* ocrow = fused ? a.o_coarse + (bh * a.T + i) * D + wg * (D / 2) : nullptr;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t o0[32], o1[32];
@@ -784,6 +802,20 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
               const float x0 = l0 > 0.f ? __uint_as_float(o0[8 * q + e]) * f0 : 0.f;
               const float x1 = l1 > 0.f ? __uint_as_float(o1[8 * q + e]) * f1 : 0.f;
               v[e] = x0 + x1;
+            }
+            if (fused) {
+              if (!live) continue;                  // pad rows have no natural token
+              const uint4 gv = __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
+              const float4 c0v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q));
+              const float4 c1v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q + 4));
+              const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+              const float cv[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                v[2 * e] = fmaf(sigmoid_fast(__uint_as_float(gw[e] << 16)), cv[2 * e], v[2 * e]);
+                v[2 * e + 1] =
+                    fmaf(sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u)), cv[2 * e + 1], v[2 * e + 1]);
+              }
             }
             uint4 u;
             u.x = pack_bf16(v[0], v[1]);
@@ -868,8 +900,8 @@ size_t attn_smem_bytes(int T, int k, int* two_p) {
 
 template <int R, int D>
 vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, const void* v_t,
-                     const int32_t* topk_idx, int64_t bh, int k, float scale, void* o_fine_t,
-                     float* lse_t, cudaStream_t stream) {
+                     const int32_t* topk_idx, int64_t bh, int k, float scale, void* out,
+                     float* lse_t, const void* gate, const float* o_coarse, cudaStream_t stream) {
   int two_p = 0;
   const size_t smem = attn_smem_bytes<R, D>(p->n_tiles, k, &two_p);
   if (smem > kMaxSmem)
@@ -885,7 +917,11 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   AttnArgs a;
   a.topk = topk_idx;
   a.block_len = p->d_block_len;
-  a.out = static_cast<uint16_t*>(o_fine_t);
+  a.out = static_cast<uint16_t*>(out);
+  a.gate = static_cast<const uint16_t*>(gate);
+  a.o_coarse = o_coarse;
+  a.row_src = p->d_row_src;
+  a.n_tok = p->n_tokens;
   a.lse = lse_t;
   a.status = p->d_status;
   a.T = p->n_tiles;
@@ -908,15 +944,22 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
 
 vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* k_t,
                               const void* v_t, const int32_t* topk_idx, int64_t bh, int D, int k,
-                              float scale, void* o_fine_t, float* lse_t, cudaStream_t stream) {
+                              float scale, void* out, float* lse_t, const void* gate,
+                              const float* o_coarse, cudaStream_t stream) {
   if (p->n_padded * bh >= (int64_t(1) << 31))
     return fail(VSA_ERR_UNSUPPORTED, "B*H*N_pad rows exceed the 32-bit TMA coordinate range");
   if (p->R == 128) {
-    if (D == 128) return launch_rd<128, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
-    return launch_rd<128, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
+    if (D == 128)
+      return launch_rd<128, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate,
+                                 o_coarse, stream);
+    return launch_rd<128, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate, o_coarse,
+                              stream);
   }
-  if (D == 128) return launch_rd<64, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
-  return launch_rd<64, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, o_fine_t, lse_t, stream);
+  if (D == 128)
+    return launch_rd<64, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate, o_coarse,
+                              stream);
+  return launch_rd<64, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate, o_coarse,
+                           stream);
 }
 
 }  // namespace vsa

@@ -53,10 +53,12 @@ cudaError_t launch_gate_combine(const uint16_t* o_fine_t, const uint16_t* gate_t
                                 const int32_t* row_src, const int32_t* untile,
                                 int64_t bh, int64_t n_tokens, int64_t n_padded, int R, int T,
                                 int D, int num_sms, cudaStream_t stream);
+// gate == nullptr: o_fine in the padded layout; otherwise the fused gated
+// combine writing natural order (gate natural [BH,N,D], o_coarse [BH,T,D]).
 vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* k_t,
                               const void* v_t, const int32_t* topk_idx, int64_t bh, int D,
-                              int k, float scale, void* o_fine_t, float* lse_t,
-                              cudaStream_t stream);
+                              int k, float scale, void* out, float* lse_t, const void* gate,
+                              const float* o_coarse, cudaStream_t stream);
 
 // Device status codes written by kernels into vsa_plan_s::d_status.
 enum : unsigned int { kStatusOk = 0, kStatusTimeout = 1, kStatusBadIndex = 2 };

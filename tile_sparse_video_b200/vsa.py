@@ -26,8 +26,8 @@ STATUS_NAMES = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED",
 # exported C symbols (kept in step with include/vsa.h)
 EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_count",
            "vsa_plan_destroy", "vsa_workspace_size", "vsa_permute", "vsa_unpermute",
-           "vsa_coarse_topk", "vsa_coarse_topk_noalloc", "vsa_sparse_attn", "vsa_gate_combine",
-           "vsa_sync_status", "vsa_last_error")
+           "vsa_coarse_topk", "vsa_coarse_topk_noalloc", "vsa_sparse_attn",
+           "vsa_sparse_attn_combine", "vsa_gate_combine", "vsa_sync_status", "vsa_last_error")
 
 
 class VsaError(RuntimeError):
@@ -65,6 +65,7 @@ def lib():
             "vsa_coarse_topk": [P, V, V, V, I, I, I, F, I, V, V, V, V, Z, V],
             "vsa_coarse_topk_noalloc": [P, V, V, V, I, I, I, F, I, V, V, V, V],
             "vsa_sparse_attn": [P, V, V, V, V, I, I, I, I, F, V, V, V, Z, V],
+            "vsa_sparse_attn_combine": [P, V, V, V, V, I, I, I, I, F, V, V, V, V, V],
             "vsa_gate_combine": [P, V, V, V, V, I, I, I, I, V],
             "vsa_sync_status": [P, V],
         }
@@ -253,6 +254,29 @@ def vsa_sparse_attn(plan: Plan, q_t, k_t, v_t, topk_idx, k: int, scale: Optional
     return out, lse
 
 
+def vsa_sparse_attn_combine(plan: Plan, q_t, k_t, v_t, topk_idx, k: int, gate, o_coarse,
+                            scale: Optional[float] = None, out=None, want_lse: bool = False,
+                            stream=None):
+    """Attention with the gated combine fused into its epilogue; ``gate`` is in
+    natural order.  Returns (out bf16 [B,H,N,D] natural order, lse or None)."""
+    B, H, _, D = q_t.shape
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("v_t", v_t)):
+        _need(t, name, torch.bfloat16, (B, H, plan.n_padded, D))
+    _need(topk_idx, "topk_idx", torch.int32, (B, H, plan.n_video_tiles, max(k, 0)))
+    _need(gate, "gate", torch.bfloat16, (B, H, plan.n_tokens, D))
+    _need(o_coarse, "o_coarse", torch.float32, (B, H, plan.n_tiles, D))
+    scale = D ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty(B, H, plan.n_tokens, D, dtype=torch.bfloat16, device=q_t.device)
+    _need(out, "out", torch.bfloat16, (B, H, plan.n_tokens, D))
+    lse = torch.empty(B, H, plan.n_padded, dtype=torch.float32, device=q_t.device) if want_lse else None
+    _check(lib().vsa_sparse_attn_combine(plan.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t),
+                                         _ptr(topk_idx) if topk_idx.numel() else None, B, H, D, k,
+                                         scale, _ptr(gate), _ptr(o_coarse), _ptr(out), _ptr(lse),
+                                         _stream(stream)))
+    return out, lse
+
+
 def vsa_gate_combine(plan: Plan, o_fine_t, gate_t, o_coarse, natural: bool = True, out=None,
                      stream=None):
     B, H, _, D = o_fine_t.shape
@@ -274,19 +298,22 @@ def vsa_sync_status(plan: Plan, stream=None):
 
 class Layer:
     """The five steps in sequence on caller-visible buffers, all launches on
-    one stream: permute Q, K, V, G; coarse + top-k; sparse attention; gated
-    combine writing natural order.  Buffers are allocated once (``reserve``)
-    and reused by every call."""
+    one stream.  ``fused=True`` (default): permute Q, K, V; coarse + top-k;
+    attention with the gated combine fused into its epilogue, writing natural
+    order (the gate is read in natural order).  ``fused=False``: the unfused
+    chain (permute Q, K, V, G; coarse + top-k; attention; combine).  Buffers
+    are allocated once and reused by every call."""
 
     def __init__(self, plan: Plan, B: int, H: int, D: int, k: int, scale: Optional[float] = None,
-                 device=None):
-        self.plan, self.B, self.H, self.D, self.k = plan, B, H, D, k
+                 device=None, fused: bool = True):
+        self.plan, self.B, self.H, self.D, self.k, self.fused = plan, B, H, D, k, fused
         self.scale = D ** -0.5 if scale is None else float(scale)
         dev = torch.device("cuda", plan.device) if device is None else torch.device(device)
         tiled = (B, H, plan.n_padded, D)
-        self.q_t, self.k_t, self.v_t, self.g_t = (torch.empty(tiled, dtype=torch.bfloat16, device=dev)
-                                                  for _ in range(4))
-        self.o_fine_t = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+        self.q_t, self.k_t, self.v_t = (torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+                                        for _ in range(3))
+        self.g_t = None if fused else torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+        self.o_fine_t = None if fused else torch.empty(tiled, dtype=torch.bfloat16, device=dev)
         self.o_coarse = torch.empty(B, H, plan.n_tiles, D, dtype=torch.float32, device=dev)
         self.topk_idx = torch.empty(B, H, plan.n_video_tiles, max(k, 0), dtype=torch.int32, device=dev)
         self.ws = torch.empty(max(plan.workspace_size(B, H, D, k), 16), dtype=torch.uint8, device=dev)
@@ -297,9 +324,13 @@ class Layer:
         vsa_permute(p, q, self.q_t, stream)
         vsa_permute(p, k, self.k_t, stream)
         vsa_permute(p, v, self.v_t, stream)
-        vsa_permute(p, g, self.g_t, stream)
         vsa_coarse_topk(p, self.q_t, self.k_t, self.v_t, self.k, self.scale, ws=self.ws,
                         o_coarse=self.o_coarse, topk_idx=self.topk_idx, stream=stream)
+        if self.fused:
+            vsa_sparse_attn_combine(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, g,
+                                    self.o_coarse, self.scale, out=self.out, stream=stream)
+            return self.out
+        vsa_permute(p, g, self.g_t, stream)
         vsa_sparse_attn(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, self.scale,
                         out=self.o_fine_t, stream=stream)
         vsa_gate_combine(p, self.o_fine_t, self.g_t, self.o_coarse, natural=True, out=self.out,
