@@ -239,6 +239,62 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit.
+// Cody-Waite range reduction: j = round(x) through the 1.5*2^23 magic constant
+// (the fp32 add rounds to nearest and leaves j in the low mantissa bits), f =
+// x - j in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted to minimise the
+// relative error on that interval (max 2.2e-4, far below bf16's 2^-9); 2^j is
+// added to the exponent field.  x is clamped at -125 so the exponent stays
+// normal (the result is then ~2.4e-38, nothing for any sum it enters).
+#ifndef VSA_STAGGER
+#define VSA_STAGGER 1
+#endif
+constexpr bool kStagger = VSA_STAGGER != 0;
+
+#ifndef VSA_EXP2_FMA_SHARE
+#define VSA_EXP2_FMA_SHARE 0
+#endif
+// One exponential in kExp2FmaShare runs on the FMA pipe (0: all on MUFU).  On
+// B200 every share measured slower (the softmax is issue-bound, not MUFU-bound:
+// 27.6 ms with none, 28.6 / 30.7 / 31.6 ms with 1 in 8 / 4 / 2), so it is off.
+constexpr int kExp2FmaShare = VSA_EXP2_FMA_SHARE;
+constexpr float kExp2C0 = 0.99996275f;
+constexpr float kExp2C1 = 0.69358679f;
+constexpr float kExp2C2 = 0.24215202f;
+constexpr float kExp2C3 = 0.05286738f;
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes of work).
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t u;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(hi), "f"(lo));
@@ -540,6 +596,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             ok = false;
             break;
           }
+          // Stagger the two softmax warpgroups by half a tile: warpgroup 1's
+          // first S of an item waits until warpgroup 0 has written its first P,
+          // so their exponential phases alternate on the MUFU unit instead of
+          // colliding.  (p_full[0] cannot move on meanwhile: warpgroup 0's next
+          // arrival needs an S that is not issued yet.)
+          if (kStagger && n == 1 &&
+              !wait_bar(p_full, (si[0] - 1) & 1, abort_flag, a.status, 13)) {
+            ok = false;
+            break;
+          }
           VSA_TL(0, 'S', g);
           tc_fence_after();
 #pragma unroll
@@ -658,9 +724,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         tc_fence_before();
         mbar_arrive(s_empty + 8 * wg);
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'l', gn);
 
         bool rescale = false;
         float alpha = 1.f;
+        uint32_t pw[BN / 2];                               // P as packed bf16 pairs
         if (rows_active) {
           // Row max over raw scores (scale > 0 commutes with max), four
           // independent chains so the warp is not latency-bound.
@@ -678,37 +746,51 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(r[c][e]));
-          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            for (int e = 0; e < 32; e += 2)
+              mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(r[c][e]),
+                                        __uint_as_float(r[c][e + 1]));
+          const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
           // Lazy rescale: the reference max moves only when some row of the
           // warp grew by more than 2^8 (exact math: p <= 256 stays well inside
           // bf16/fp32 range).  The decision is warp-uniform because the O
           // rescale below uses warp-collective TMEM loads and stores.
+          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'm', gn);
           const float m_cand = fmaxf(m, mx * a.scale_log2);
           rescale = __any_sync(0xFFFFFFFFu, m_cand > m + 8.0f);
           const float m_new = rescale ? m_cand : m;
           alpha = ex2(m - m_new);
           const float neg_m = -m_new;
-          float sum4[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) sum4[q] = 0.f;
+          // exponentials on pairs: packed scale-and-subtract, two exp2, packed
+          // row sums, and P packed to bf16 right away (one in kExp2FmaShare on
+          // the FMA pipe)
+          const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(neg_m, neg_m);
+          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float p = ex2(fmaf(__uint_as_float(r[c][e]), a.scale_log2, neg_m));
-              sum4[e & 3] += p;
-              r[c][e] = __float_as_uint(p);
+            for (int e = 0; e < 32; e += 2) {
+              float x0, x1;
+              f2unpack(ffma2(f2pack(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), sc2, nm2),
+                       x0, x1);
+              const bool fma0 = kExp2FmaShare > 0 && e % kExp2FmaShare == kExp2FmaShare - 1;
+              const bool fma1 = kExp2FmaShare > 0 && (e + 1) % kExp2FmaShare == kExp2FmaShare - 1;
+              const float p0 = fma0 ? exp2_fma(x0) : ex2(x0);
+              const float p1 = fma1 ? exp2_fma(x1) : ex2(x1);
+              acc2[(e >> 1) & 3] = fadd2(acc2[(e >> 1) & 3], f2pack(p0, p1));
+              pw[16 * c + (e >> 1)] = pack_bf16(p0, p1);
             }
-          const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-          l = l * alpha + sum;
+          float s0, s1, s2, s3;
+          f2unpack(fadd2(acc2[0], acc2[1]), s0, s1);
+          f2unpack(fadd2(acc2[2], acc2[3]), s2, s3);
+          l = l * alpha + ((s0 + s1) + (s2 + s3));
           m = m_new;
         }
         // Before P_n is written (and O_w possibly rescaled): with one P tile per
         // warpgroup, this warpgroup's own PV of tile n-2 must be done; with one
         // shared P tile, the other warpgroup's PV of tile n-1 (which orders our
         // own n-2 before it).  At an item's first tiles the previous item's
-        // epilogue already waited for every PV.
+        // epilogue already waited for every PV.  The exponentials above overlap
+        // that PV.
         if (lane == 0) VSA_TR(quad + 4 * wg, 15, gn);
         if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'w', gn);
         if (a.two_p ? n >= 2 : n >= 1) {
@@ -722,17 +804,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         if (rows_active) {
 #pragma unroll
           for (int c8 = 0; c8 < BN / 8; ++c8) {
-            const int c = c8 / 4, e = (c8 % 4) * 8;
-            const uint32_t w0 = pack_bf16(__uint_as_float(r[c][e + 0]), __uint_as_float(r[c][e + 1]));
-            const uint32_t w1 = pack_bf16(__uint_as_float(r[c][e + 2]), __uint_as_float(r[c][e + 3]));
-            const uint32_t w2 = pack_bf16(__uint_as_float(r[c][e + 4]), __uint_as_float(r[c][e + 5]));
-            const uint32_t w3 = pack_bf16(__uint_as_float(r[c][e + 6]), __uint_as_float(r[c][e + 7]));
             const uint32_t addr =
                 my_p + (c8 / 8) * kBM * 128 + row * 128 + ((uint32_t(c8 % 8) ^ uint32_t(row & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w0), "r"(w1),
-                         "r"(w2), "r"(w3)
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pw[4 * c8]),
+                         "r"(pw[4 * c8 + 1]), "r"(pw[4 * c8 + 2]), "r"(pw[4 * c8 + 3])
                          : "memory");
           }
+          // O_w rescale after the S registers are dead (PV(n) is not issued
+          // before the p_full arrival below).
           if (n >= 2 && rescale) {
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
