@@ -202,6 +202,31 @@ def pick_workload(args) -> Workload:
     return w
 
 
+# ----------------------------------------------------------------- ranks
+
+def rank_workload(w: Workload, rank: int) -> Workload:
+    """Rank ``rank``'s replica: the same shapes, its own seeded batch (rank 0
+    keeps the workload's own seed, so a 1-GPU run is unchanged)."""
+    return w if rank == 0 else replace(w, seed_base=w.seed_base + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value of ``x`` over all ranks (the slowest rank's time).
+    Every rank must call it, in the same order as the other collectives."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(elapsed_max_ms: float, steps: int, world: int) -> float:
+    """Whole-job time per layer: the slowest rank's span over every layer that
+    all ranks ran (each rank runs ``steps`` layers of its own)."""
+    return elapsed_max_ms / (steps * world)
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     from tile_sparse_video_b200 import vsa
     import torch.distributed as dist
@@ -209,7 +234,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = pick_workload(args)
-    inp = make_inputs(w)
+    inp = make_inputs(rank_workload(w, rank))
     plan = vsa.Plan(w.prefix, w.grid, w.tile, device=local_rank)
     k = plan.keep_count(keep_ratio=w.keep_ratio, keep_tiles=w.keep_tiles)
     acct = geometry_counts(w, plan.n_prefix_tiles, plan.n_tiles, k)
@@ -261,10 +286,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     elapsed = t_start.elapsed_time(t_end)
     parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in events])
     part_ms = parts.mean(axis=0)
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, world, dev)
 
     # end to end through the public API: pinned host inputs in, output back
     host = {n: inp[n].pin_memory() for n in "qkvg"}
@@ -289,15 +311,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_elapsed = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_elapsed = float(t.item())
+    e2e_elapsed = max_over_ranks(e2e_elapsed, world, dev)
     vsa.vsa_sync_status(plan)
 
     peaks = load_peaks()
     layers = args.steps * world
-    ms_layer = elapsed / layers
+    ms_layer = job_ms_per_layer(elapsed, args.steps, world)
     attn_ms = float(part_ms[2])
     achieved = acct["kept_flop"] / (attn_ms * 1e-3) / 1e12
     res = {
@@ -323,7 +342,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                      "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),
                      "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16 burst)",
                      "traffic": attn_traffic()},
-        "e2e": {"value": round(e2e_elapsed / (max(e2e_steps, 1) * world), 3) if e2e_steps else None,
+        "e2e": {"value": round(job_ms_per_layer(e2e_elapsed, e2e_steps, world), 3) if e2e_steps else None,
                 "unit": UNIT,
                 "h2d_bytes_per_step": int(sum(host[n].numel() * 2 for n in "qkvg")),
                 "d2h_bytes_per_step": int(out_host.numel() * 2)},
