@@ -9,11 +9,14 @@
 // masked; o = softmax(scale * q k^T) v per live query row.
 //
 // Design (one persistent CTA per SM, static round-robin over work items):
-//   work item = (b*h, query tile i); prefix items (n_p of them per head, each
-//   T key tiles long) come first, then the video items head by head, so the
-//   CTAs share one or two heads' K/V in L2 at any time.
-//   warp 8  (TMA K)  loads Q once per item and K_j per kept tile into a K ring,
-//                    and prefetches K/V tiles a few steps ahead into L2.
+//   work item = (b*h, query tile i); the video items come first, head by
+//   head, so the CTAs share one or two heads' K/V in L2 at any time, and the
+//   prefix items (n_p per head, each T key tiles long, streaming a whole
+//   head's K/V) come last.  Run first, the prefix items kept their CTAs about
+//   a millisecond behind the others for the rest of the launch, spreading the
+//   concurrent items over three heads whose K/V no longer fit in L2.
+//   warp 8  (TMA K)  loads Q once per item (evict-first: it is read once) and
+//                    K_j per kept tile into a K ring.
 //   warp 9  (TMA V)  loads V_j into its own ring (V is needed later than K).
 //   warp 10 (MMA S)  one lane issues S_n = Q K_n^T (M=128, N=R, K=D) into the
 //                    TMEM S buffer of warpgroup n & 1 as soon as K_n is in and
@@ -62,6 +65,33 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 #ifndef VSA_NSK128
 #define VSA_NSK128 2
 #endif
+
+// Tuning knobs (compile-time).  L2 prefetch distance of the K producer in
+// key tiles (0: none), work item order (see decode_item), an evict-first L2
+// policy on the Q loads (each Q tile is read once) and an evict-last policy
+// on the K/V loads (each K/V tile is read by many query tiles).  Measured on
+// B200 at the 104k-token Veda layer (sparse attention + combine): item order
+// 0 -> 1 took 27.0 to 25.6 ms; a 4-tile L2 prefetch cost 0.5-0.9 ms (it
+// doubles the L2 lookups, and the co-resident CTAs already share most K/V
+// tiles); the K/V evict-last policy and streaming epilogue accesses changed
+// nothing measurable or cost a little.
+#ifndef VSA_PREFETCH
+#define VSA_PREFETCH 0
+#endif
+#ifndef VSA_ORDER
+#define VSA_ORDER 1
+#endif
+#ifndef VSA_QHINT
+#define VSA_QHINT 1
+#endif
+#ifndef VSA_KVHINT
+#define VSA_KVHINT 0
+#endif
+// Streaming (evict-first) gate loads and output stores in the fused epilogue.
+#ifndef VSA_STREAM_IO
+#define VSA_STREAM_IO 0
+#endif
+constexpr int kItemOrder = VSA_ORDER;
 
 // Progress trace for debugging builds (-DVSA_TRACE): each role of each CTA
 // publishes its position in the pipeline to a host-visible buffer (16 slots
@@ -143,6 +173,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
+}
+// Same with an L2 cache policy (from createpolicy).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 // L2 prefetch of one tensor-map box (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int c0, int c1) {
@@ -388,13 +437,24 @@ __device__ __noinline__ void wait_bar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void decode_item(int item, int bh_np, int n_p, int n_v, int64_t& bh,
+// Work item -> (b*h, query tile i).  kItemOrder 0: every head's prefix query
+// tiles first, then the video query tiles head by head; 1: the video tiles
+// head by head, then every head's prefix tiles; 2: head by head, each head's
+// tiles in tile order.
+__device__ __forceinline__ void decode_item(int item, int BH, int n_p, int n_v, int64_t& bh,
                                             int& i) {
-  if (item < bh_np) {
-    bh = item / n_p;
-    i = item % n_p;
+  if (kItemOrder == 2) {
+    bh = item / (n_p + n_v);
+    i = item % (n_p + n_v);
+    return;
+  }
+  const int first = kItemOrder == 0 ? BH * n_p : BH * n_v;
+  const bool prefix = kItemOrder == 0 ? item < first : item >= first;
+  const int v = kItemOrder == 0 ? (prefix ? item : item - first) : (prefix ? item - first : item);
+  if (prefix) {
+    bh = v / n_p;
+    i = v % n_p;
   } else {
-    const int v = item - bh_np;
     bh = v / n_v;
     i = n_p + v % n_v;
   }
@@ -413,15 +473,15 @@ __device__ __forceinline__ int kept_tile(const AttnArgs& a, int64_t bh, int i, i
 
 // Producer loop shared by the K and the V warp: lane 0 issues one TMA tile per
 // kept key tile into an NS-stage ring; the K warp also loads Q per item and
-// prefetches K/V tiles kPrefetch ahead into L2.
+// (kPrefetch > 0) prefetches K/V tiles kPrefetch ahead into L2.
 template <int R, int D, int NS, bool kIsK>
 __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* tm_q,
                                          const CUtensorMap* tm_t, const CUtensorMap* tm_other,
                                          uint32_t sQ, uint32_t sT, uint32_t full, uint32_t empty,
                                          uint32_t q_full, uint32_t q_empty, int32_t* s_list,
-                                         volatile int* abort_flag, int lane, int bh_np, int n_v) {
+                                         volatile int* abort_flag, int lane, int BH, int n_v) {
   using C = Cfg<R, D>;
-  constexpr int kPrefetch = 4;
+  constexpr int kPrefetch = VSA_PREFETCH;
   VSA_TL_DECL;
   uint32_t g = 0, q_issued = 0;
   int t = 0;
@@ -429,7 +489,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
   for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
     int64_t bh;
     int i;
-    decode_item(item, bh_np, a.n_p, n_v, bh, i);
+    decode_item(item, BH, a.n_p, n_v, bh, i);
     const bool dense = i < a.n_p;
     const int nk = dense ? a.T : a.n_p + a.k;
     if (!dense)
@@ -445,7 +505,11 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
           mbar_expect_tx(q_full, C::QBYTES);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sQ + c * kBM * 128, tm_q, q_full, c * 64, int(row0 + int64_t(i) * R));
+            if (VSA_QHINT)
+              tma_load_2d_hint(sQ + c * kBM * 128, tm_q, q_full, c * 64, int(row0 + int64_t(i) * R),
+                               l2_evict_first_policy());
+            else
+              tma_load_2d(sQ + c * kBM * 128, tm_q, q_full, c * 64, int(row0 + int64_t(i) * R));
         }
       }
       for (int n = 0; n < nk && ok; ++n, ++g) {
@@ -461,8 +525,12 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
         mbar_expect_tx(full + 8 * s, C::TBYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sT + s * C::TBYTES + c * C::BN * 128, tm_t, full + 8 * s, c * 64, row);
-        if (kIsK && n + kPrefetch < nk) {
+          if (VSA_KVHINT)
+            tma_load_2d_hint(sT + s * C::TBYTES + c * C::BN * 128, tm_t, full + 8 * s, c * 64, row,
+                             l2_evict_last_policy());
+          else
+            tma_load_2d(sT + s * C::TBYTES + c * C::BN * 128, tm_t, full + 8 * s, c * 64, row);
+        if (kIsK && kPrefetch > 0 && n + kPrefetch < nk) {
           const int jp = (dense || n + kPrefetch < a.n_p) ? n + kPrefetch : s_list[n + kPrefetch - a.n_p];
           const int rp = int(row0 + int64_t(jp) * R);
 #pragma unroll
@@ -522,7 +590,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_v = a.T - a.n_p;
-  const int bh_np = a.n_items - (a.n_items / a.T) * n_v;   // = BH * n_p
+  const int BH = a.n_items / a.T;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -568,10 +636,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 
   if (warp == kWarpTmaK) {
     producer<R, D, NSK, true>(a, &tm_q, &tm_k, &tm_v, sQ, sK, k_full, k_empty, q_full, q_empty,
-                              s_klist, abort_flag, lane, bh_np, n_v);
+                              s_klist, abort_flag, lane, BH, n_v);
   } else if (warp == kWarpTmaV) {
     producer<R, D, NSV, false>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full, q_empty,
-                               s_vlist, abort_flag, lane, bh_np, n_v);
+                               s_vlist, abort_flag, lane, BH, n_v);
   } else if (warp == kWarpMmaS) {
     // ------------------------------------------------------------ S issuer
     // S_n = Q K_n^T into S_{n&1} (tile n of an item belongs to softmax
@@ -585,7 +653,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
         int64_t bh;
         int i;
-        decode_item(item, bh_np, a.n_p, n_v, bh, i);
+        decode_item(item, BH, a.n_p, n_v, bh, i);
         const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
         if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
         for (int n = 0; n < nk; ++n, ++g) {
@@ -638,7 +706,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
         int64_t bh;
         int i;
-        decode_item(item, bh_np, a.n_p, n_v, bh, i);
+        decode_item(item, BH, a.n_p, n_v, bh, i);
         const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
         for (int n = 0; n < nk; ++n, ++g) {
           const int w = n & 1;
@@ -688,7 +756,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
       int64_t bh;
       int i;
-      decode_item(item, bh_np, a.n_p, n_v, bh, i);
+      decode_item(item, BH, a.n_p, n_v, bh, i);
       const bool dense = i < a.n_p;
       const int nk = dense ? a.T : a.n_p + a.k;
       // Group barrier of the 256 softmax threads (it also keeps the next P
@@ -884,7 +952,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             }
             if (fused) {
               if (!live) continue;                  // pad rows have no natural token
-              const uint4 gv = __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
+              const uint4 gv = VSA_STREAM_IO ? __ldcs(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q))
+                                             : __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
               const float4 c0v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q));
               const float4 c1v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q + 4));
               const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
@@ -901,7 +970,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             u.y = pack_bf16(v[2], v[3]);
             u.z = pack_bf16(v[4], v[5]);
             u.w = pack_bf16(v[6], v[7]);
-            dst[q] = u;
+            if (VSA_STREAM_IO)
+              __stcs(dst + q, u);
+            else
+              dst[q] = u;
           }
         }
         if (a.lse != nullptr && wg == 0)
