@@ -45,9 +45,9 @@ METRIC = "ms/layer & kept-FLOP TFLOP/s (% bf16 peak) at 104k tokens, 90% tile sp
 UNIT = "ms/layer"
 
 # DRAM bytes (read + write) of one full-size sparse_attn launch, from the ncu
-# capture summarised in profiles/sparse_attn_veda_h8.md (8 heads, scaled by
-# 42/8), valid only for the kernel source it was taken on.
-ATTN_TRAFFIC = {"source_sha256_16": "0db0ee252c210a2a", "bytes": 23.42e9}
+# capture summarised in profiles/sparse_attn_veda_h8.md (8 heads: 2.270 GB,
+# scaled by 42/8), valid only for the kernel source it was taken on.
+ATTN_TRAFFIC = {"source_sha256_16": "54907c49e3ed86ab", "bytes": 11.92e9}
 
 
 # ----------------------------------------------------------------- accounting
