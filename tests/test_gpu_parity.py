@@ -60,10 +60,10 @@ def _keep(plan, w):
     return plan.keep_count(keep_ratio=w.keep_ratio, keep_tiles=w.keep_tiles)
 
 
-def _run(w: Workload):
+def _run(w: Workload, inp=None):
     """The unfused chain (every intermediate visible), plus the fused
     attention + combine entry point on the same inputs."""
-    inp = make_inputs(w)
+    inp = make_inputs(w) if inp is None else inp
     plan = vsa.Plan(w.prefix, w.grid, w.tile)
     k = _keep(plan, w)
     q, kk, v, g = (inp[x].cuda() for x in "qkvg")
@@ -82,7 +82,36 @@ def _run(w: Workload):
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_layer_parity(w):
-    inp, plan, k, layer, out, scores, lse, out_t = _run(w)
+    _check_layer(w, make_inputs(w))
+
+
+def _growing_logits(w: Workload):
+    """Inputs whose key rows grow with their key tile: K of tile j is scaled by
+    1 + 3j, so the row maximum of the scores jumps by more than 2^8 from tile
+    to tile and the attention kernel's running (reference) max moves, with the
+    O rescale that goes with it, on most tiles of every item.  The attention
+    is then nearly one-hot, so V is scaled by 1/4 to keep the outputs at the
+    unit scale the tolerance is stated for (the moving max does not depend
+    on V)."""
+    inp = make_inputs(w)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    tile_of_token = torch.from_numpy(p.untile // p.R)
+    c = (1.0 + 3.0 * tile_of_token.double()).view(1, 1, -1, 1)
+    inp["k"] = (inp["k"].double() * c).to(torch.bfloat16)
+    inp["v"] = (inp["v"].double() * 0.25).to(torch.bfloat16)
+    return inp
+
+
+@pytest.mark.parametrize("w", [
+    _w("growing_logits_r64", 1, 2, 128, (100, 28), (8, 8, 8), (4, 4, 4), keep_tiles=5),
+    _w("growing_logits_r128", 1, 2, 128, (256,), (8, 16, 8), (4, 8, 4), keep_tiles=3),
+], ids=lambda w: w.name)
+def test_layer_parity_moving_max(w):
+    _check_layer(w, _growing_logits(w))
+
+
+def _check_layer(w: Workload, inp):
+    inp, plan, k, layer, out, scores, lse, out_t = _run(w, inp)
     p = O.plan(w.prefix, w.grid, w.tile)
     gpu_idx = layer.topk_idx.cpu().numpy().astype(np.int64)
     ref = O.layer(*(inp[x] for x in "qkvg"), p, k, kept=gpu_idx)

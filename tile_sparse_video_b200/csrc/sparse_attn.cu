@@ -19,24 +19,29 @@
 //                    K_j per kept tile into a K ring.
 //   warp 9  (TMA V)  loads V_j into its own ring (V is needed later than K).
 //   warp 10 (MMA S)  one lane issues S_n = Q K_n^T (M=128, N=R, K=D) into the
-//                    TMEM S buffer of warpgroup n & 1 as soon as K_n is in and
-//                    the warpgroup has read its previous S.
-//   warp 11 (MMA PV) one lane issues O_w += P_n V_n (M=128, N=D, K=R) as soon
-//                    as P_n is written; the two issuers run independently.
+//                    TMEM S tile of softmax warpgroup n & 1 once that warpgroup
+//                    has read its previous S.
+//   warp 11 (MMA PV) one lane issues O += P_n V_n (M=128, N=D, K=R) with the A
+//                    operand P_n read from TMEM; the two issuers run
+//                    independently (S and PV touch disjoint TMEM columns).
 //   warps 0-7        two softmax warpgroups; warpgroup w takes the tiles
 //                    n = w (mod 2) of an item (a split of the key set inside the
-//                    CTA).  Thread = query row = TMEM lane: it loads its S row,
-//                    masks past block_len, keeps a running max (moved only when
-//                    a row grew by more than 2^8, exact), writes P = exp2(.) as
-//                    bf16 into the single 128-byte-swizzled shared P tile (the
-//                    A operand of the PV MMA; the two warpgroups take turns in
-//                    tile order) and rescales its O_w row in TMEM when the max
-//                    moved.  The epilogue merges the two partial (m, l, O)
-//                    states and stores bf16 rows (and the LSE).
-// TMEM columns: S_0 [0,R), S_1 [R,2R), O_0 [2R,2R+D), O_1 [2R+D,2R+2D).
-// P tiles live in shared memory: one per warpgroup when they fit (then a
-// warpgroup only waits for its own PV of tile n-2 before rewriting its P),
-// else one shared tile written in tile order.
+//                    CTA), and both add into one O.  Thread = query row = TMEM
+//                    lane: it loads its S row, masks past block_len, and scales
+//                    by a reference max m_ref shared by both warpgroups.  m_ref
+//                    after tile n is decided by the warp that runs tile n, from
+//                    m_ref after tile n-1 (published by the warp of the other
+//                    warpgroup on the same TMEM lanes through a shared-memory
+//                    mailbox) and its own row max; it moves only when a row grew
+//                    by more than 2^8 (exact: p <= 256), and then that warp
+//                    rescales its O rows once PV_{n-1} is complete.  P = exp2(.)
+//                    goes to TMEM as bf16 pairs.  The epilogue adds the two
+//                    warpgroups' row sums and stores bf16 rows (and the LSE), or
+//                    the gated combine in natural order.
+// TMEM columns: O [0,D), S_w [D + w*R, D + (w+1)*R), P_w [D + 2R + w*R/2,
+// D + 2R + (w+1)*R/2) (two bf16 per 32-bit column, key order, row = lane).
+// S_{n+2} depends only on S_n having been read, P_n only on PV_{n-2}, so MMA
+// latency stays off the softmax's path, and no P tile takes shared memory.
 // With R = 64 the MMA still runs with M = 128 (rows 64..127 of the Q box are
 // the next rows of the tensor, or zero past its end); their results are never
 // stored and the warps of those rows skip the softmax work.
@@ -59,11 +64,12 @@ constexpr int kThreadsAttn = 384;        // 8 softmax warps + TMA K + TMA V + MM
 constexpr int kWarpTmaK = 8, kWarpTmaV = 9, kWarpMmaS = 10, kWarpMmaPV = 11;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
-// K ring depth for 128-row tiles (a tuning knob: 2 stages leave room for one
-// P tile per softmax warpgroup, which measured faster on B200 than 3 stages
-// with one shared P tile: 27.4 vs 32.2 ms at the 104k-token Veda layer).
+// K and V ring depths for 128-row tiles (tuning knobs, bounded by shared memory).
 #ifndef VSA_NSK128
-#define VSA_NSK128 2
+#define VSA_NSK128 3
+#endif
+#ifndef VSA_NSV128
+#define VSA_NSV128 2
 #endif
 
 // Tuning knobs (compile-time).  L2 prefetch distance of the K producer in
@@ -210,9 +216,6 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100
 // descriptor version 1.  Addresses and offsets are in bytes.
@@ -239,6 +242,16 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t 
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Same with the A operand in TMEM (M rows = lanes, two bf16 per column along K).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
@@ -295,10 +308,6 @@ __device__ __forceinline__ float ex2(float x) {
 // relative error on that interval (max 2.2e-4, far below bf16's 2^-9); 2^j is
 // added to the exponent field.  x is clamped at -125 so the exponent stays
 // normal (the result is then ~2.4e-38, nothing for any sum it enters).
-#ifndef VSA_STAGGER
-#define VSA_STAGGER 1
-#endif
-constexpr bool kStagger = VSA_STAGGER != 0;
 
 #ifndef VSA_EXP2_FMA_SHARE
 #define VSA_EXP2_FMA_SHARE 0
@@ -307,6 +316,13 @@ constexpr bool kStagger = VSA_STAGGER != 0;
 // B200 every share measured slower (the softmax is issue-bound, not MUFU-bound:
 // 27.6 ms with none, 28.6 / 30.7 / 31.6 ms with 1 in 8 / 4 / 2), so it is off.
 constexpr int kExp2FmaShare = VSA_EXP2_FMA_SHARE;
+// The reference-max decision of a tile is published after this many of the
+// tile's 32-score exponential chunks (R/32 or more: after all of them), so
+// that the partner warp's exponentials start while ours finish.
+#ifndef VSA_PUB_CHUNK
+#define VSA_PUB_CHUNK 99
+#endif
+constexpr int kPubChunk = VSA_PUB_CHUNK;
 constexpr float kExp2C0 = 0.99996275f;
 constexpr float kExp2C1 = 0.69358679f;
 constexpr float kExp2C2 = 0.24215202f;
@@ -364,7 +380,6 @@ struct AttnArgs {
   const float* o_coarse;      // fp32 [BH, T, D]
   const int32_t* row_src;     // [N_pad] padded row -> token, -1 for a pad row
   int T, n_p, k, n_items;
-  int two_p;                  // 1: one P tile per softmax warpgroup, 0: one shared P tile
   int64_t n_pad, n_tok;
   float scale_log2;           // scale * log2(e)
 };
@@ -380,29 +395,34 @@ template <int R, int D>
 struct Cfg {
   static constexpr int BN = R;
   static constexpr int NSK = (R == 128) ? VSA_NSK128 : 4;   // K ring stages
-  static constexpr int NSV = (R == 128) ? 2 : 4;        // V ring stages
+  static constexpr int NSV = (R == 128) ? VSA_NSV128 : 4;   // V ring stages
   static constexpr int QBYTES = kBM * D * 2;
   static constexpr int TBYTES = BN * D * 2;              // one K (or V) tile
-  static constexpr int PBYTES = kBM * BN * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_V = OFF_K + NSK * TBYTES;
-  static constexpr int OFF_P = OFF_V + NSV * TBYTES;     // P_0, then P_1 when two_p
+  // reference-max mailbox fp32 [2 tile parities][128 rows], then the
+  // epilogue's (m, l) exchange fp32 [2 values][2 warpgroups][128 rows]
+  static constexpr int OFF_X = OFF_V + NSV * TBYTES;
+  static constexpr int OFF_BAR = OFF_X + (2 + 4) * 128 * 4;
   // barriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV],
-  //           s_full[2], s_empty[2], p_full[2], pv_done[2], o_full, o_empty, drain,
-  //           drain2
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 12;
+  //           s_full[2], s_empty[2], p_full[2], pv_done[2], dec[4], o_full, o_empty,
+  //           drain, drain2
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 4;
   static constexpr int TAIL = NBAR * 8 + 16;              // barriers + tmem slot + abort flag
-  static constexpr uint32_t TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256u : 512u;
-  static constexpr uint32_t COL_S = 0;                   // S_w at COL_S + w*BN
-  static constexpr uint32_t COL_O = 2 * BN;              // O_w at COL_O + w*D
+  // TMEM columns: O [0, D), S_w [D + w*BN, D + (w+1)*BN), P_w (bf16 pairs)
+  // [D + 2*BN + w*BN/2, D + 2*BN + (w+1)*BN/2)
+  static constexpr uint32_t COL_O = 0;
+  static constexpr uint32_t COL_S = D;
+  static constexpr uint32_t COL_P = D + 2 * BN;
+  static constexpr uint32_t TMEM_COLS = (D + 3 * BN) <= 256 ? 256u : 512u;
+  static_assert(D + 3 * BN <= 512, "TMEM columns");
   static constexpr uint32_t IDESC_QK = idesc_bf16(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, false, true);
-  // bytes after OFF_P: P tiles, barriers/misc, then the lists (blen uint8[T],
+  // bytes: tiles, exchanges, barriers/misc, then the lists (blen uint8[T],
   // two int32[k] kept-tile lists)
-  static size_t bytes(int two_p, int T, int k) {
-    return size_t(OFF_P) + size_t(two_p ? 2 : 1) * PBYTES + TAIL + size_t((T + 15) & ~15) +
-           size_t(8) * ((k + 3) & ~3);
+  static size_t bytes(int T, int k) {
+    return size_t(OFF_BAR) + TAIL + size_t((T + 15) & ~15) + size_t(8) * ((k + 3) & ~3);
   }
 };
 
@@ -412,13 +432,18 @@ __device__ __forceinline__ void record(unsigned int* status, unsigned int code, 
 
 // Bounded wait; false when the CTA is aborting (flag already set, or this wait
 // timed out, in which case it sets the flag and records the timeout).
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                      unsigned int* status, unsigned int where) {
+// Inline, so that a wait costs no call (at the softmax's call sites some 150
+// registers are live, and a call saved and restored them: measured ~450 SM
+// cycles per wait on B200 even when the phase had long completed).  The timer
+// and the abort flag are looked at every 16 polls; mbarrier.try_wait itself
+// suspends the thread for a while when the phase is not complete.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned int* status, unsigned int where) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
+    if ((it & 15u) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
@@ -564,27 +589,26 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V,
-                 sP = s_base + C::OFF_P;
-  const int n_ptiles = a.two_p ? 2 : 1;
-  const uint32_t off_bar = C::OFF_P + n_ptiles * C::PBYTES;
-  const uint32_t bar0 = s_base + off_bar;
+  const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V;
+  const uint32_t bar0 = s_base + C::OFF_BAR;
   const uint32_t q_full = bar0, q_empty = bar0 + 8;
   const uint32_t k_full = bar0 + 16, k_empty = k_full + 8 * NSK;
   const uint32_t v_full = k_empty + 8 * NSK, v_empty = v_full + 8 * NSV;
-  const uint32_t s_full = v_empty + 8 * NSV, s_empty = s_full + 16;
-  // p_full[w] / pv_done[w] complete once per tile of warpgroup w, o_full and
-  // o_empty once per item.  Every wait below targets a phase whose predecessor
-  // is already complete and whose successor cannot complete before the waiter
-  // has observed it, so the parity test never aliases.
-  const uint32_t p_full = s_empty + 16, pv_done = p_full + 16, o_full = pv_done + 16,
+  // s_full[w], s_empty[w], p_full[w] and pv_done[w] complete once per tile of
+  // warpgroup w, dec[q] once per tile (the reference-max decision for TMEM
+  // lane quadrant q), o_full and o_empty once per item.  Every wait targets a
+  // phase whose predecessor is already complete and whose successor cannot
+  // complete before the waiter has observed it, so the parity test never
+  // aliases.
+  const uint32_t s_full = v_empty + 8 * NSV, s_empty = s_full + 16, p_full = s_empty + 16,
+                 pv_done = p_full + 16, dec = pv_done + 16, o_full = dec + 32,
                  o_empty = o_full + 8, drain = o_empty + 8, drain2 = drain + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + C::NBAR * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + off_bar + C::NBAR * 8 + 4);
-  // merge exchange of (m, l) lives in P_0 (free once an item's PVs are done)
-  float* s_m = reinterpret_cast<float*>(smem + C::OFF_P);         // [2][128]
-  float* s_l = s_m + 2 * 128;                                      // [2][128]
-  uint8_t* s_blen = smem + off_bar + C::TAIL;                      // [T]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + C::NBAR * 8 + 4);
+  float* mbox = reinterpret_cast<float*>(smem + C::OFF_X);       // [2][128]
+  float* x_m = mbox + 2 * 128;                                    // [2][128]
+  float* x_l = x_m + 2 * 128;                                     // [2][128]
+  uint8_t* s_blen = smem + C::OFF_BAR + C::TAIL;                  // [T]
   int32_t* s_klist = reinterpret_cast<int32_t*>(s_blen + ((a.T + 15) & ~15));
   int32_t* s_vlist = s_klist + ((a.k + 3) & ~3);
 
@@ -609,6 +633,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       mbar_init(p_full + 8 * w, 128);
       mbar_init(pv_done + 8 * w, 1);
     }
+    for (int q = 0; q < 4; ++q) mbar_init(dec + 8 * q, 32);
     mbar_init(o_full, 1);
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
@@ -642,12 +667,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                s_vlist, abort_flag, lane, BH, n_v);
   } else if (warp == kWarpMmaS) {
     // ------------------------------------------------------------ S issuer
-    // S_n = Q K_n^T into S_{n&1} (tile n of an item belongs to softmax
-    // warpgroup n & 1); needs Q of the item, K_n, and the warpgroup done
-    // reading its previous S.  Runs ahead across items.
+    // S_n = Q K_n^T into S_w (w = n & 1) as soon as K_n is in and warpgroup w
+    // has read S_{n-2} out of it.  Runs ahead across items.
     if (lane == 0) {
       VSA_TL_DECL;
-      uint32_t g = 0, si[2] = {0, 0};
+      uint32_t gk = 0;                   // K tiles consumed (ring position)
+      uint32_t si[2] = {0, 0};           // S tiles issued per warpgroup
+      uint32_t g = 0;                    // tiles of earlier items (trace only)
       int t = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
@@ -656,25 +682,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         decode_item(item, BH, a.n_p, n_v, bh, i);
         const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
         if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
-        for (int n = 0; n < nk; ++n, ++g) {
+        for (int n = 0; n < nk; ++n) {
           const int w = n & 1;
-          const uint32_t s = g % NSK;
-          if (!wait_bar(k_full + 8 * s, (g / NSK) & 1, abort_flag, a.status, 6)) { ok = false; break; }
-          if (si[w] > 0 && !wait_bar(s_empty + 8 * w, (si[w] - 1) & 1, abort_flag, a.status, 7)) {
+          if (si[w] > 0 &&
+              !wait_bar(s_empty + 8 * w, (si[w] - 1) & 1, abort_flag, a.status, 7)) {
             ok = false;
             break;
           }
-          // Stagger the two softmax warpgroups by half a tile: warpgroup 1's
-          // first S of an item waits until warpgroup 0 has written its first P,
-          // so their exponential phases alternate on the MUFU unit instead of
-          // colliding.  (p_full[0] cannot move on meanwhile: warpgroup 0's next
-          // arrival needs an S that is not issued yet.)
-          if (kStagger && n == 1 &&
-              !wait_bar(p_full, (si[0] - 1) & 1, abort_flag, a.status, 13)) {
-            ok = false;
-            break;
-          }
-          VSA_TL(0, 'S', g);
+          const uint32_t s = gk % NSK;
+          if (!wait_bar(k_full + 8 * s, (gk / NSK) & 1, abort_flag, a.status, 6)) { ok = false; break; }
+          VSA_TL(0, 'S', g + n);
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
@@ -685,22 +702,28 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           }
           umma_commit(s_full + 8 * w);
           umma_commit(k_empty + 8 * s);
+          ++gk;
           ++si[w];
           if (n == nk - 1) umma_commit(q_empty);
         }
+        g += nk;
       }
       // Drain: wait until every MMA issued above has completed.
       umma_commit(drain);
       wait_bar_drain(drain, 0);
+      VSA_TR(11, 12, gk);
     }
     __syncwarp();
   } else if (warp == kWarpMmaPV) {
     // ------------------------------------------------------------ PV issuer
-    // O_{n&1} += P_n V_n; needs P_n written, V_n, and at an item's first tile
-    // the previous item's epilogue done reading O.
+    // O += P_n V_n (A operand P_n from TMEM tile P_w) as soon as P_n is
+    // written and V_n is in; an item's first PV also waits for the previous
+    // item's epilogue to have read O.  Both warpgroups add into the one O.
     if (lane == 0) {
       VSA_TL_DECL;
-      uint32_t g = 0, pc[2] = {0, 0};
+      uint32_t gv = 0;                   // V tiles consumed (ring position)
+      uint32_t pf[2] = {0, 0};           // p_full phases consumed per warpgroup
+      uint32_t g = 0;                    // tiles of earlier items (trace only)
       int t = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
@@ -708,37 +731,47 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         int i;
         decode_item(item, BH, a.n_p, n_v, bh, i);
         const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
-        for (int n = 0; n < nk; ++n, ++g) {
+        for (int n = 0; n < nk; ++n) {
           const int w = n & 1;
-          const uint32_t sv = g % NSV;
           if (n == 0 && t > 0 && !wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) {
             ok = false;
             break;
           }
-          if (!wait_bar(p_full + 8 * w, pc[w] & 1, abort_flag, a.status, 4)) { ok = false; break; }
-          if (!wait_bar(v_full + 8 * sv, (g / NSV) & 1, abort_flag, a.status, 12)) { ok = false; break; }
-          VSA_TL(5, 'P', g);
+          if (!wait_bar(p_full + 8 * w, pf[w] & 1, abort_flag, a.status, 4)) { ok = false; break; }
+          ++pf[w];
+          const uint32_t sv = gv % NSV;
+          if (!wait_bar(v_full + 8 * sv, (gv / NSV) & 1, abort_flag, a.status, 12)) {
+            ok = false;
+            break;
+          }
+          VSA_TL(5, 'P', g + n);
           tc_fence_after();
-          const uint32_t sp = sP + (a.two_p ? w * C::PBYTES : 0);
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t ad = sdesc_sw128(sp + (ks / 4) * kBM * 128 + (ks % 4) * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(sV + sv * C::TBYTES + ks * 16 * 128, BN * 128, 1024);
-            umma_bf16(tmem + C::COL_O + w * D, ad, bd, C::IDESC_PV, (n >= 2 || ks > 0) ? 1u : 0u);
+            umma_bf16_ts(tmem + C::COL_O, tmem + C::COL_P + w * (BN / 2) + ks * 8, bd, C::IDESC_PV,
+                         (n > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(pv_done + 8 * w);
           umma_commit(v_empty + 8 * sv);
           if (n == nk - 1) umma_commit(o_full);
-          ++pc[w];
+          ++gv;
         }
+        g += nk;
       }
       umma_commit(drain2);
       wait_bar_drain(drain2, 0);
-      VSA_TR(11, 12, g);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warpgroups
+    // Warpgroup wg takes the tiles n = wg (mod 2) of an item; both add into
+    // one O, scaled by one reference max m_ref per row.  m_ref after tile n is
+    // decided by the warp that runs tile n from m_ref after tile n-1 (read
+    // from the mailbox its partner warp on the same TMEM lanes wrote) and its
+    // own row max, and published in turn; it moves only when a row grew by
+    // more than 2^8 (exact: p <= 256), and then that warp rescales its O rows
+    // once PV_{n-1} is complete.
     VSA_TL_DECL;
     const int wg = warp >> 2;                            // 0 or 1
     const int quad = warp & 3;
@@ -746,11 +779,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const int row = quad * 32 + lane;                    // = TMEM lane
     const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
     const uint32_t col_s = C::COL_S + wg * BN;
-    const uint32_t col_o = C::COL_O + wg * D;
-    const uint32_t my_p = sP + (a.two_p ? wg * C::PBYTES : 0);
-    uint32_t g = 0;              // global tile counter (trace only)
+    const uint32_t col_p = C::COL_P + wg * (BN / 2);
+    const uint32_t dbar = dec + 8 * quad;
+    uint32_t G = 0;              // global index of the item's first tile
     uint32_t cnt[2] = {0, 0};    // tiles of each warpgroup in earlier items
-    uint32_t cw = 0;             // tiles processed by this warpgroup (s_full phases)
+    uint32_t cw = 0;             // tiles processed by this warpgroup
     int t = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
@@ -759,10 +792,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       decode_item(item, BH, a.n_p, n_v, bh, i);
       const bool dense = i < a.n_p;
       const int nk = dense ? a.T : a.n_p + a.k;
-      // Group barrier of the 256 softmax threads (it also keeps the next P
-      // write behind the previous item's (m, l) exchange in P_0).  A warp that
-      // sees the abort flag leaves instead: the others then also see it before
-      // they could block here (they wait on the same mbarrier phases first).
+      // Group barrier of the 256 softmax threads around the per-item list.  A
+      // warp that sees the abort flag leaves instead: the others then also see
+      // it before they could block here (they wait on the same mbarrier phases
+      // first).
       if (*abort_flag) { ok = false; break; }
       asm volatile("bar.sync 1, 256;" ::: "memory");
       for (int x = threadIdx.x; x < nk; x += 256) {
@@ -773,15 +806,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       asm volatile("bar.sync 1, 256;" ::: "memory");
       const int q_live = __ldg(a.block_len + i);
 
-      float m = -INFINITY, l = 0.f;
+      float m_mine = -INFINITY, l = 0.f;   // l: this warpgroup's row sum, relative to m_mine
       for (int n = wg; n < nk; n += 2, ++cw) {
-        const uint32_t gn = g + n;
-        (void)gn;
-        if (lane == 0) VSA_TR(quad + 4 * wg, 13, gn);
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'a', gn);
+        const uint32_t Gn = G + n;
+        if (lane == 0) VSA_TR(quad + 4 * wg, 13, Gn);
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'a', Gn);
         ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * wg, cw & 1, abort_flag, a.status, 8));
         if (!ok) break;
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 's', gn);
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 's', Gn);
         tc_fence_after();
         uint32_t r[BN / 32][32];
         if (rows_active) {
@@ -792,14 +824,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         tc_fence_before();
         mbar_arrive(s_empty + 8 * wg);
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'l', gn);
-
-        bool rescale = false;
-        float alpha = 1.f;
-        uint32_t pw[BN / 2];                               // P as packed bf16 pairs
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'l', Gn);
+        // row max over raw scores (scale > 0 commutes with max), four chains
+        float mx = -INFINITY;
         if (rows_active) {
-          // Row max over raw scores (scale > 0 commutes with max), four
-          // independent chains so the warp is not latency-bound.
           const int bl = int(s_blen[n]) + 1;
           if (bl < BN) {
 #pragma unroll
@@ -817,92 +845,116 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             for (int e = 0; e < 32; e += 2)
               mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(r[c][e]),
                                         __uint_as_float(r[c][e + 1]));
-          const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
-          // Lazy rescale: the reference max moves only when some row of the
-          // warp grew by more than 2^8 (exact math: p <= 256 stays well inside
-          // bf16/fp32 range).  The decision is warp-uniform because the O
-          // rescale below uses warp-collective TMEM loads and stores.
-          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'm', gn);
-          const float m_cand = fmaxf(m, mx * a.scale_log2);
-          rescale = __any_sync(0xFFFFFFFFu, m_cand > m + 8.0f);
-          const float m_new = rescale ? m_cand : m;
-          alpha = ex2(m - m_new);
-          const float neg_m = -m_new;
-          // exponentials on pairs: packed scale-and-subtract, two exp2, packed
-          // row sums, and P packed to bf16 right away (one in kExp2FmaShare on
-          // the FMA pipe)
-          const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(neg_m, neg_m);
-          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float x0, x1;
-              f2unpack(ffma2(f2pack(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), sc2, nm2),
-                       x0, x1);
-              const bool fma0 = kExp2FmaShare > 0 && e % kExp2FmaShare == kExp2FmaShare - 1;
-              const bool fma1 = kExp2FmaShare > 0 && (e + 1) % kExp2FmaShare == kExp2FmaShare - 1;
-              const float p0 = fma0 ? exp2_fma(x0) : ex2(x0);
-              const float p1 = fma1 ? exp2_fma(x1) : ex2(x1);
-              acc2[(e >> 1) & 3] = fadd2(acc2[(e >> 1) & 3], f2pack(p0, p1));
-              pw[16 * c + (e >> 1)] = pack_bf16(p0, p1);
-            }
-          float s0, s1, s2, s3;
-          f2unpack(fadd2(acc2[0], acc2[1]), s0, s1);
-          f2unpack(fadd2(acc2[2], acc2[3]), s2, s3);
-          l = l * alpha + ((s0 + s1) + (s2 + s3));
-          m = m_new;
+          mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
         }
-        // Before P_n is written (and O_w possibly rescaled): with one P tile per
-        // warpgroup, this warpgroup's own PV of tile n-2 must be done; with one
-        // shared P tile, the other warpgroup's PV of tile n-1 (which orders our
-        // own n-2 before it).  At an item's first tiles the previous item's
-        // epilogue already waited for every PV.  The exponentials above overlap
-        // that PV.
-        if (lane == 0) VSA_TR(quad + 4 * wg, 15, gn);
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'w', gn);
-        if (a.two_p ? n >= 2 : n >= 1) {
-          const int ow = a.two_p ? wg : 1 - wg;
-          const uint32_t idx = cnt[ow] + uint32_t(a.two_p ? (n - 2) >> 1 : (n - 1) >> 1);
+        // m_ref after tile n-1 (the previous global tile's decision; an item's
+        // first tile starts from -inf), then this tile's decision
+        float m_prev = -INFINITY;
+        if (Gn > 0) {
+          ok = __all_sync(0xFFFFFFFFu, wait_bar(dbar, (Gn - 1) & 1, abort_flag, a.status, 14));
+          if (!ok) break;
+          if (n > 0) m_prev = mbox[((Gn - 1) & 1) * 128 + row];
+        }
+        const float m_cand = fmaxf(m_prev, mx * a.scale_log2);
+        // warp-uniform (the O rescale below uses warp-collective TMEM access)
+        const bool rescale = __any_sync(0xFFFFFFFFu, m_cand > m_prev + 8.0f);
+        const float m_new = rescale ? m_cand : m_prev;
+        bool published = false;            // warp-uniform
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'm', Gn);
+        if (rows_active) {
+          // this warpgroup's row sum follows the reference max
+          l *= ex2(m_mine - m_new);
+          m_mine = m_new;
+        }
+        // P_w is free once this warpgroup's previous PV is complete
+        if (cw > 0) {
           ok = __all_sync(0xFFFFFFFFu,
-                          wait_bar(pv_done + 8 * ow, idx & 1, abort_flag, a.status, 9));
+                          wait_bar(pv_done + 8 * wg, (cw - 1) & 1, abort_flag, a.status, 9));
           if (!ok) break;
         }
         tc_fence_after();
         if (rows_active) {
+          // exponentials on pairs: packed scale-and-subtract, two exp2, packed
+          // row sums, P packed to bf16 and stored to P_w every 64 scores.  One
+          // exponential in kExp2FmaShare runs on the FMA pipe.
+          const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(-m_new, -m_new);
+          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int c8 = 0; c8 < BN / 8; ++c8) {
-            const uint32_t addr =
-                my_p + (c8 / 8) * kBM * 128 + row * 128 + ((uint32_t(c8 % 8) ^ uint32_t(row & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pw[4 * c8]),
-                         "r"(pw[4 * c8 + 1]), "r"(pw[4 * c8 + 2]), "r"(pw[4 * c8 + 3])
-                         : "memory");
+          for (int c2 = 0; c2 < BN / 64; ++c2) {
+            uint32_t pw[32];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int c = 2 * c2 + h;
+              if (kPubChunk > 0 && kPubChunk < BN / 32 && c == kPubChunk) {
+                mbox[(Gn & 1) * 128 + row] = m_new;
+                mbar_arrive(dbar);
+                published = true;
+              }
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float x0, x1;
+                f2unpack(ffma2(f2pack(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), sc2,
+                               nm2),
+                         x0, x1);
+                const bool fma0 = kExp2FmaShare > 0 && e % kExp2FmaShare == kExp2FmaShare - 1;
+                const bool fma1 = kExp2FmaShare > 0 && (e + 1) % kExp2FmaShare == kExp2FmaShare - 1;
+                const float p0 = fma0 ? exp2_fma(x0) : ex2(x0);
+                const float p1 = fma1 ? exp2_fma(x1) : ex2(x1);
+                acc2[(e >> 1) & 3] = fadd2(acc2[(e >> 1) & 3], f2pack(p0, p1));
+                pw[16 * h + (e >> 1)] = pack_bf16(p0, p1);
+              }
+            }
+            tmem_st32(t_lane + col_p + 32 * c2, pw);
           }
-          // O_w rescale after the S registers are dead (PV(n) is not issued
-          // before the p_full arrival below).
-          if (n >= 2 && rescale) {
+          float s0, s1, s2, s3;
+          f2unpack(fadd2(acc2[0], acc2[1]), s0, s1);
+          f2unpack(fadd2(acc2[2], acc2[3]), s2, s3);
+          l += (s0 + s1) + (s2 + s3);
+        }
+        // Publish the decision only now: the partner warp, which shares this
+        // warp's SM sub-partition and its MUFU unit, cannot start its own
+        // exponentials before ours are done, so the two warps take turns on
+        // the MUFU and each does its loads, max and stores during the
+        // other's exponentials.
+        if (!published) {
+          mbox[(Gn & 1) * 128 + row] = m_new;
+          mbar_arrive(dbar);
+        }
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'w', Gn);
+        // O rescale when the reference max moved: O holds PV_0..PV_{n-1}
+        // relative to m_prev; PV_{n-1} (the partner's tile) must be complete,
+        // and PV_n is not issued before the p_full arrival below.
+        if (rescale && n > 0) {
+          const uint32_t idx = cnt[1 - wg] + uint32_t((n - 1) >> 1);
+          ok = __all_sync(0xFFFFFFFFu,
+                          wait_bar(pv_done + 8 * (1 - wg), idx & 1, abort_flag, a.status, 15));
+          if (!ok) break;
+          tc_fence_after();
+          if (rows_active) {
+            const float alpha = ex2(m_prev - m_new);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
-              tmem_ld32(t_lane + col_o + 32 * c, o);
+              tmem_ld32(t_lane + C::COL_O + 32 * c, o);
               tmem_wait_ld(o);
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(t_lane + col_o + 32 * c, o);
+              tmem_st32(t_lane + C::COL_O + 32 * c, o);
             }
-            tmem_wait_st();
           }
         }
-        fence_proxy_async_smem();
+        if (rows_active) tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + 8 * wg);
-        if (lane == 0) VSA_TR(quad + 4 * wg, 16, gn);
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'W', gn);
+        if (lane == 0) VSA_TR(quad + 4 * wg, 16, Gn);
+        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'W', Gn);
       }
       if (!ok) break;
-      // ---- epilogue: merge the two warpgroups' partial softmax states once
-      // every PV of the item is complete (o_full).
-      const uint32_t g_last = g + nk - 1;
+      // ---- epilogue: once every PV of the item is complete (o_full), add the
+      // two row sums (each relative to its warpgroup's last reference max; O
+      // is relative to the larger) and store O / l (warpgroup wg: columns
+      // [wg*D/2, (wg+1)*D/2)), fused with the gated combine when a gate is given.
+      const uint32_t g_last = G + nk - 1;
       (void)g_last;
       if (lane == 0) VSA_TR(quad + 4 * wg, 17, g_last);
       ok = __all_sync(0xFFFFFFFFu, wait_bar(o_full, t & 1, abort_flag, a.status, 10));
@@ -910,22 +962,17 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       cnt[0] += uint32_t((nk + 1) / 2);
       cnt[1] += uint32_t(nk / 2);
       tc_fence_after();
-      s_m[wg * 128 + row] = m;
-      s_l[wg * 128 + row] = l;
+      x_m[wg * 128 + row] = m_mine;
+      x_l[wg * 128 + row] = l;
       if (*abort_flag) { ok = false; break; }
       asm volatile("bar.sync 1, 256;" ::: "memory");
       if (rows_active) {
-        const float m0 = s_m[row], m1 = s_m[128 + row];
-        const float l0 = s_l[row], l1 = s_l[128 + row];
+        const float m0 = x_m[row], m1 = x_m[128 + row];
+        const float l0 = x_l[row], l1 = x_l[128 + row];
         const float mm = fmaxf(m0, m1);
-        const float a0 = l0 > 0.f ? ex2(m0 - mm) : 0.f;
-        const float a1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
-        const float lt = a0 * l0 + a1 * l1;
+        const float lt = (l0 > 0.f ? l0 * ex2(m0 - mm) : 0.f) + (l1 > 0.f ? l1 * ex2(m1 - mm) : 0.f);
         const bool live = row < q_live;
         const float inv = live ? 1.0f / lt : 0.f;
-        const float f0 = a0 * inv, f1 = a1 * inv;
-        // warpgroup wg stores columns [wg*D/2, (wg+1)*D/2) of the row; fused:
-        // the gated combine, written to the row's natural token position
         const bool fused = a.gate != nullptr;
         const int64_t tok = (fused && live) ? int64_t(__ldg(a.row_src + int64_t(i) * R + row)) : 0;
         uint16_t* orow = fused ? a.out + (bh * a.n_tok + tok) * D + wg * (D / 2)
@@ -934,26 +981,20 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         const float* ocrow = fused ? a.o_coarse + (bh * a.T + i) * D + wg * (D / 2) : nullptr;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          uint32_t o0[32], o1[32];
-          tmem_ld32(t_lane + C::COL_O + wg * (D / 2) + 32 * c, o0);
-          tmem_ld32(t_lane + C::COL_O + D + wg * (D / 2) + 32 * c, o1);
-          tmem_wait_ld(o0);
-          tmem_wait_ld(o1);
+          uint32_t o[32];
+          tmem_ld32(t_lane + C::COL_O + wg * (D / 2) + 32 * c, o);
+          tmem_wait_ld(o);
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float v[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              // a warpgroup that saw no tile left its O columns unwritten
-              const float x0 = l0 > 0.f ? __uint_as_float(o0[8 * q + e]) * f0 : 0.f;
-              const float x1 = l1 > 0.f ? __uint_as_float(o1[8 * q + e]) * f1 : 0.f;
-              v[e] = x0 + x1;
-            }
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[8 * q + e]) * inv;
             if (fused) {
               if (!live) continue;                  // pad rows have no natural token
-              const uint4 gv = VSA_STREAM_IO ? __ldcs(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q))
-                                             : __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
+              const uint4 gv =
+                  VSA_STREAM_IO ? __ldcs(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q))
+                                : __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
               const float4 c0v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q));
               const float4 c1v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q + 4));
               const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
@@ -983,7 +1024,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       tc_fence_before();
       mbar_arrive(o_empty);
       if (lane == 0) VSA_TR(quad + 4 * wg, 18, g_last);
-      g += nk;
+      G += nk;
     }
   }
 
@@ -1035,17 +1076,13 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int D, int box_rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Dynamic shared memory of one CTA.  At least 120 KB, so that two CTAs never
-// share an SM (each allocates its TMEM columns for its whole lifetime).
 // Dynamic shared memory of one CTA (+1 KB so the kernel can align its base to
 // 1024 bytes), at least 120 KB so that two CTAs never share an SM (each holds
-// its TMEM columns for its whole lifetime).  Two P tiles when they fit.
+// its TMEM columns for its whole lifetime).
 constexpr size_t kMaxSmem = 227 * 1024;
 template <int R, int D>
-size_t attn_smem_bytes(int T, int k, int* two_p) {
-  using C = Cfg<R, D>;
-  *two_p = (C::bytes(1, T, k) + 1024 <= kMaxSmem) ? 1 : 0;
-  const size_t need = C::bytes(*two_p, T, k) + 1024;
+size_t attn_smem_bytes(int T, int k) {
+  const size_t need = Cfg<R, D>::bytes(T, k) + 1024;
   return need < size_t(120 * 1024) ? size_t(120 * 1024) : need;
 }
 
@@ -1053,8 +1090,7 @@ template <int R, int D>
 vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, const void* v_t,
                      const int32_t* topk_idx, int64_t bh, int k, float scale, void* out,
                      float* lse_t, const void* gate, const float* o_coarse, cudaStream_t stream) {
-  int two_p = 0;
-  const size_t smem = attn_smem_bytes<R, D>(p->n_tiles, k, &two_p);
+  const size_t smem = attn_smem_bytes<R, D>(p->n_tiles, k);
   if (smem > kMaxSmem)
     return fail(VSA_ERR_UNSUPPORTED, "too many tiles for the sparse attention kernel's lists");
   const int64_t rows = bh * p->n_padded;
@@ -1079,7 +1115,6 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   a.n_p = p->n_prefix_tiles;
   a.k = k;
   a.n_pad = p->n_padded;
-  a.two_p = two_p;
   a.scale_log2 = scale * 1.4426950408889634f;
   const int64_t items = bh * p->n_tiles;
   if (items >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "too many work items");
