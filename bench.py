@@ -44,10 +44,11 @@ from tile_sparse_video_b200.inputs import VEDA_104K, WORKLOADS, Workload, make_i
 METRIC = "ms/layer & kept-FLOP TFLOP/s (% bf16 peak) at 104k tokens, 90% tile sparsity"
 UNIT = "ms/layer"
 
-# DRAM bytes (read + write) of one full-size sparse_attn launch, from the ncu
-# capture summarised in profiles/sparse_attn_veda_h8.md (8 heads: 2.270 GB,
-# scaled by 42/8), valid only for the kernel source it was taken on.
-ATTN_TRAFFIC = {"source_sha256_16": "54907c49e3ed86ab", "bytes": 11.92e9}
+# DRAM bytes (read + write) of one full-size sparse_attn launch, from the
+# one-pass ncu capture at the benchmark size summarised in
+# profiles/sparse_attn_veda_h8.md, valid only for the kernel source it was
+# taken on.
+ATTN_TRAFFIC = {"source_sha256_16": "22dc35d71a58beb3", "bytes": 21.20e9}
 
 
 # ----------------------------------------------------------------- accounting

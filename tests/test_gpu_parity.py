@@ -50,6 +50,8 @@ CASES = [
     _w("keep_none", 1, 2, 128, (40, 70), (4, 8, 8), (4, 4, 4), keep_tiles=0),
     _w("one_video_tile", 1, 1, 128, (64,), (4, 4, 4), (4, 4, 4), keep_tiles=1),
     _w("prefix_only", 1, 2, 128, (100, 28), (0, 0, 0), (4, 4, 4), keep_tiles=0),
+    # 128-row tiles with long kept-tile lists (250 of 300 video tiles)
+    _w("wide_k_r128", 1, 1, 128, (256,), (24, 40, 40), (4, 8, 4), keep_tiles=250),
 ]
 # sweep shapes that the oracle finishes quickly (shortest clips, both families)
 CASES += [w for w in sweep_workloads() if w.grid[0] == 16 and ("s90" in w.name or "k24" in w.name)
