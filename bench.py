@@ -3,9 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one whole layer (permute Q/K/V, pool + coarse attention + top-k,
-block-sparse attention with the gated combine fused into its epilogue, writing
-natural order) on the 104,704-token
+One step = one whole layer (permute Q/K/V with the tile means taken in the
+same pass, coarse attention + top-k, block-sparse attention with the gated
+combine fused into its epilogue, writing natural order) on the 104,704-token
 Veda workload: 42 heads x 128, 128-token key tiles (4x8x4), 2 prefix tiles and
 816 video tiles, 90 % sparsity (82 kept video tiles per query tile).
 
@@ -65,10 +65,9 @@ def geometry_counts(w: Workload, n_p: int, T: int, k: int) -> dict:
         kept_flop=4.0 * D * R * R * pairs * BH,            # QK^T and PV over kept tile pairs
         dense_flop=4.0 * N * N * D * BH,
         # bytes: read N real rows, write N_pad padded rows; Q, K and V (the gate
-        # is read in natural order by the fused attention + combine)
+        # is read in natural order by the fused attention + combine); the tile
+        # means are taken in the same pass
         permute_bytes=3.0 * BH * (N + N_pad) * D * 2,
-        # pool reads the live rows of Q, K, V
-        pool_bytes=3.0 * BH * N * D * 2,
         # attention + combine: Q, K, V read once, the gate read and the output
         # written once (natural order)
         attn_bytes=3.0 * BH * N_pad * D * 2 + 2.0 * BH * N * D * 2,
@@ -242,18 +241,19 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     q, kk, v, g = (inp[n].to(dev) for n in "qkvg")
     layer = vsa.Layer(plan, w.B, w.H, w.D, k)
     stream = torch.cuda.current_stream()
-    launches_per_step = 6          # 3 permutes, pool, coarse+top-k, attention with fused combine
+    launches_per_step = 5          # 3 permute+pool, coarse+top-k, attention with fused combine
+    slots = vsa.pooled_slots(plan, layer.ws, w.B, w.H, w.D)
 
     def step(ev=None):
         p = plan
         if ev is not None:
             ev[0].record(stream)
-        for src, dst in ((q, layer.q_t), (kk, layer.k_t), (v, layer.v_t)):
-            vsa.vsa_permute(p, src, dst)
+        for src, dst, pooled in zip((q, kk, v), (layer.q_t, layer.k_t, layer.v_t), slots):
+            vsa.vsa_permute_pool(p, src, dst, pooled)
         if ev is not None:
             ev[1].record(stream)
-        vsa.vsa_coarse_topk(p, layer.q_t, layer.k_t, layer.v_t, k, layer.scale, ws=layer.ws,
-                            o_coarse=layer.o_coarse, topk_idx=layer.topk_idx)
+        vsa.vsa_coarse_topk_pooled(p, w.B, w.H, w.D, k, layer.ws, layer.scale,
+                                   o_coarse=layer.o_coarse, topk_idx=layer.topk_idx)
         if ev is not None:
             ev[2].record(stream)
         vsa.vsa_sparse_attn_combine(p, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k, g,
@@ -334,10 +334,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "kept_tflops": round(acct["kept_flop"] * layers / (elapsed * 1e-3) / 1e12, 2),
         "dense_equiv_tflops": round(acct["dense_flop"] * layers / (elapsed * 1e-3) / 1e12, 2),
         "pct_bf16_peak_layer": round(100 * acct["kept_flop"] * layers / (elapsed * 1e-3) / 1e12 / peaks["bf16"], 2),
-        "kernels_ms": {"permute_q_k_v": round(float(part_ms[0]), 4),
-                       "pool_coarse_topk": round(float(part_ms[1]), 4),
+        "kernels_ms": {"permute_pool_q_k_v": round(float(part_ms[0]), 4),
+                       "coarse_topk": round(float(part_ms[1]), 4),
                        "sparse_attn_combine": round(attn_ms, 4)},
-        "kernels_hbm_gbs": {"permute_q_k_v": round(acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9, 1)},
+        "kernels_hbm_gbs": {"permute_pool_q_k_v": round(acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9, 1)},
         "roofline": {"kernel": "sparse_attn_combine", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
                      "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),

@@ -138,6 +138,25 @@ vsa_status vsa_coarse_topk(vsa_plan plan, const void* q_t, const void* k_t, cons
                            float* o_coarse, int32_t* topk_idx, float* topk_score,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Steps 1 and 2 fused for one of Q, K, V: the permute of vsa_permute, and in
+ * the same pass the fp32 mean over each tile's live rows, written to
+ * pooled[b,h,t,:] (fp32 [B,H,T,D]; 16-byte aligned).  Same permuted output as
+ * vsa_permute; the pooled means equal those vsa_coarse_topk computes up to
+ * fp32 summation order.  For a layer, point `pooled` at the workspace slot of
+ * the tensor (qbar, kbar or vbar, see vsa_workspace_size) and finish with
+ * vsa_coarse_topk_pooled.  Sources: SnackOnAI snippet two (the permute) and
+ * this library's reading of "coarse tile selection" (mean pooling). */
+vsa_status vsa_permute_pool(vsa_plan plan, const void* x, void* x_t, int B, int H, int D,
+                            float* pooled, void* stream);
+
+/* Steps 2 (coarse part) and 3 of vsa_coarse_topk from pooled means already in
+ * `ws` (qbar, kbar, vbar in the layout of vsa_workspace_size, as written by
+ * vsa_permute_pool): no pooling pass and no q_t/k_t/v_t arguments.  Same
+ * outputs, validation and errors as vsa_coarse_topk. */
+vsa_status vsa_coarse_topk_pooled(vsa_plan plan, int B, int H, int D, float scale, int k,
+                                  float* o_coarse, int32_t* topk_idx, float* topk_score,
+                                  void* ws, size_t ws_bytes, void* stream);
+
 /* Allocation-free variant of vsa_coarse_topk (the pages have no counterpart:
  * this is a library convenience).  For callers that cannot call cudaMalloc --
  * a host application that owns all device memory and gives plugins no

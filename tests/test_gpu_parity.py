@@ -76,9 +76,17 @@ def _run(w: Workload, inp=None):
     out_t = vsa.vsa_gate_combine(plan, layer.o_fine_t, layer.g_t, layer.o_coarse, natural=False)
     fused, lse_f = vsa.vsa_sparse_attn_combine(plan, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k,
                                                g, layer.o_coarse, want_lse=True)
+    # the fused permute + pool pass, and coarse + top-k from its pooled means
+    ws2 = torch.empty_like(layer.ws)
+    slots = vsa.pooled_slots(plan, ws2, w.B, w.H, w.D)
+    for x, x_t, pooled in zip((q, kk, v), (layer.q_t, layer.k_t, layer.v_t), slots):
+        x_t2, _ = vsa.vsa_permute_pool(plan, x, pooled=pooled)
+        assert torch.equal(x_t2, x_t)
+    oc2, idx2, _ = vsa.vsa_coarse_topk_pooled(plan, w.B, w.H, w.D, k, ws2)
     vsa.vsa_sync_status(plan)
     assert torch.equal(lse_f, lse)
     layer.fused_out = fused
+    layer.pp = (slots, oc2, idx2)
     return inp, plan, k, layer, out, scores, lse, out_t
 
 
@@ -127,9 +135,15 @@ def _check_layer(w: Workload, inp):
     for i, name in enumerate(("qbar", "kbar", "vbar")):
         np.testing.assert_allclose(f64(pooled[i]), ref[name], rtol=1e-5, atol=1e-6, err_msg=name)
     np.testing.assert_allclose(f64(layer.o_coarse), ref["o_coarse"], rtol=1e-4, atol=1e-5)
+    slots, oc2, idx2 = layer.pp
+    for i, name in enumerate(("qbar", "kbar", "vbar")):
+        np.testing.assert_allclose(f64(slots[i]), ref[name], rtol=1e-5, atol=1e-6, err_msg=name + " (fused)")
+    np.testing.assert_allclose(f64(oc2), ref["o_coarse"], rtol=1e-4, atol=1e-5)
     # step 3: selection, bit-exact up to legal near-tie swaps
     near = check_topk(gpu_idx, ref["scores"], p, k)
     assert near <= max(1, int(np.prod(gpu_idx.shape[:-1])) // 50)
+    near2 = check_topk(idx2.cpu().numpy().astype(np.int64), ref["scores"], p, k)
+    assert near2 <= max(1, int(np.prod(gpu_idx.shape[:-1])) // 50)
     if k > 0:
         gs = f64(scores)
         want = np.take_along_axis(ref["scores"][..., p.n_prefix_tiles:, :], gpu_idx, axis=-1)

@@ -234,6 +234,51 @@ vsa_status vsa_coarse_topk(vsa_plan p, const void* q_t, const void* k_t, const v
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "coarse_topk launch");
 }
 
+vsa_status vsa_permute_pool(vsa_plan p, const void* x, void* x_t, int B, int H, int D,
+                            float* pooled, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(x, "x"));
+  VSA_TRY(check_ptr(x_t, "x_t"));
+  VSA_TRY(check_ptr(pooled, "pooled"));
+  cudaError_t e = launch_permute_pool(static_cast<const uint16_t*>(x), static_cast<uint16_t*>(x_t),
+                                      p->d_row_src, p->d_block_len, pooled, int64_t(B) * H,
+                                      p->n_tiles, p->R, p->n_tokens, p->n_padded, D, p->num_sms,
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "vsa_permute_pool launch");
+}
+
+vsa_status vsa_coarse_topk_pooled(vsa_plan p, int B, int H, int D, float scale, int k,
+                                  float* o_coarse, int32_t* topk_idx, float* topk_score, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  VSA_TRY(check_k(p, k));
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(o_coarse, "o_coarse"));
+  const int n_v = p->n_tiles - p->n_prefix_tiles;
+  if (k > 0 && n_v > 0) VSA_TRY(check_ptr(topk_idx, "topk_idx"));
+  if (topk_score != nullptr && !aligned16(topk_score))
+    return fail(VSA_ERR_INVALID_ARG, "topk_score is not 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(VSA_ERR_INVALID_ARG, "scale is not finite");
+  if (p->n_tiles > 4096)
+    return fail(VSA_ERR_UNSUPPORTED, "coarse attention supports at most 4096 tiles");
+  size_t need = 0;
+  vsa_workspace_size(p, B, H, D, k, &need);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(VSA_ERR_WORKSPACE, "workspace missing or too small (see vsa_workspace_size)");
+  if (!aligned16(ws)) return fail(VSA_ERR_INVALID_ARG, "ws is not 16-byte aligned");
+  const int64_t bh = int64_t(B) * H;
+  const float* qbar = static_cast<const float*>(ws);
+  const float* kbar = qbar + bh * p->n_tiles * D;
+  const float* vbar = kbar + bh * p->n_tiles * D;
+  cudaError_t e = launch_coarse_topk(qbar, kbar, vbar, bh, p->n_tiles, p->n_prefix_tiles, D, scale,
+                                     k, o_coarse, topk_idx, topk_score,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "coarse_topk launch");
+}
+
 vsa_status vsa_sparse_attn(vsa_plan p, const void* q_t, const void* k_t, const void* v_t,
                            const int32_t* topk_idx, int B, int H, int D, int k, float scale,
                            void* o_fine_t, float* lse_t, void* ws, size_t ws_bytes,

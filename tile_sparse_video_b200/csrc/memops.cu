@@ -1,5 +1,5 @@
 // HBM-bound passes of the layer: row gather (permute / unpermute), per-tile
-// mean pooling, and the gated combine.
+// mean pooling, the two fused (permute + pool), and the gated combine.
 //
 // All three move whole rows of D bf16 values (128 or 256 bytes) as 16-byte
 // vectors.  A thread owns one 16-byte chunk of a row per step and keeps
@@ -107,6 +107,66 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const uint4* __restrict_
     if (lane < kCpr) {
       const float inv = 1.0f / float(n);
       float4* o = reinterpret_cast<float4*>(out + (bh * T + t) * int64_t(kCpr * 8) + lane * 8);
+      o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+    }
+  }
+}
+
+// Permute and pool in one pass (the permute's gather, with the tile mean
+// taken on the way): one warp per (bh, tile).  Lane l owns 16-byte chunk
+// l % kCpr of rows l / kCpr, l / kCpr + 32 / kCpr, ...; it gathers the tile's
+// live rows from their natural positions (row_src), writes the tile's R rows
+// contiguously to the permuted layout (zeros past block_len) and adds the
+// live rows into 8 fp32 column sums, kU loads in flight.  The lanes that
+// share a chunk are then summed with shuffles and the mean written fp32.
+// Same HBM bytes as the permute alone; the pooled means cost no extra pass.
+template <int kCpr>
+__global__ void __launch_bounds__(kThreads) permute_pool_kernel(
+    const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ row_src,
+    const int32_t* __restrict__ block_len, float* __restrict__ pooled, int64_t n_items, int T,
+    int R, int64_t src_rows, int64_t dst_rows) {
+  constexpr int kRowsPerPass = 32 / kCpr;
+  constexpr int kU = 8;
+  const int lane = threadIdx.x & 31;
+  const int cc = lane % kCpr;
+  const int64_t warps = int64_t(gridDim.x) * (kThreads / 32);
+  for (int64_t item = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); item < n_items;
+       item += warps) {
+    const int64_t bh = item / T;
+    const int t = int(item % T);
+    const int n = __ldg(block_len + t);
+    const uint4* s = src + bh * src_rows * kCpr + cc;
+    uint4* d = dst + (bh * dst_rows + int64_t(t) * R) * kCpr + cc;
+    const int32_t* rs = row_src + int64_t(t) * R;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r = lane / kCpr; r < R; r += kRowsPerPass * kU) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int rr = r + u * kRowsPerPass;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (rr < n) {
+          const int32_t m = __ldg(rs + rr);
+          if (m >= 0) v[u] = ldg_nc(s + int64_t(m) * kCpr);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int rr = r + u * kRowsPerPass;
+        if (rr < R) {
+          d[int64_t(rr) * kCpr] = v[u];
+          if (rr < n) add_bf16x8(acc, v[u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int off = kCpr; off < 32; off <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], off);
+    if (lane < kCpr) {
+      const float inv = 1.0f / float(n);
+      float4* o = reinterpret_cast<float4*>(pooled + item * int64_t(kCpr * 8) + lane * 8);
       o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
       o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
     }
@@ -230,6 +290,25 @@ cudaError_t launch_pool(const uint16_t* q_t, const uint16_t* k_t, const uint16_t
     pool_kernel<8><<<grid, kThreads, 0, stream>>>(
         reinterpret_cast<const uint4*>(q_t), reinterpret_cast<const uint4*>(k_t),
         reinterpret_cast<const uint4*>(v_t), block_len, qbar, kbar, vbar, n_items, T, R);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_pool(const uint16_t* src, uint16_t* dst, const int32_t* row_src,
+                                const int32_t* block_len, float* pooled, int64_t bh, int T, int R,
+                                int64_t src_rows, int64_t dst_rows, int D, int num_sms,
+                                cudaStream_t stream) {
+  const int64_t n_items = bh * T;
+  const int64_t want = int64_t(num_sms > 0 ? num_sms : 148) * 8;
+  int64_t blocks = (n_items + 7) / 8;
+  if (blocks > want) blocks = want;
+  if (D == 128)
+    permute_pool_kernel<16><<<unsigned(blocks), kThreads, 0, stream>>>(
+        reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), row_src, block_len,
+        pooled, n_items, T, R, src_rows, dst_rows);
+  else
+    permute_pool_kernel<8><<<unsigned(blocks), kThreads, 0, stream>>>(
+        reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), row_src, block_len,
+        pooled, n_items, T, R, src_rows, dst_rows);
   return cudaGetLastError();
 }
 

@@ -44,6 +44,10 @@ cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, const int32_t
 cudaError_t launch_pool(const uint16_t* q_t, const uint16_t* k_t, const uint16_t* v_t,
                         const int32_t* block_len, float* qbar, float* kbar, float* vbar,
                         int64_t bh, int T, int R, int D, int num_sms, cudaStream_t stream);
+cudaError_t launch_permute_pool(const uint16_t* src, uint16_t* dst, const int32_t* row_src,
+                                const int32_t* block_len, float* pooled, int64_t bh, int T, int R,
+                                int64_t src_rows, int64_t dst_rows, int D, int num_sms,
+                                cudaStream_t stream);
 cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float* vbar,
                                int64_t bh, int T, int n_p, int D, float scale, int k,
                                float* o_coarse, int32_t* topk_idx, float* topk_score,

@@ -26,8 +26,9 @@ STATUS_NAMES = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED",
 # exported C symbols (kept in step with include/vsa.h)
 EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_count",
            "vsa_plan_destroy", "vsa_workspace_size", "vsa_permute", "vsa_unpermute",
-           "vsa_coarse_topk", "vsa_coarse_topk_noalloc", "vsa_sparse_attn",
-           "vsa_sparse_attn_combine", "vsa_gate_combine", "vsa_sync_status", "vsa_last_error")
+           "vsa_permute_pool", "vsa_coarse_topk", "vsa_coarse_topk_pooled",
+           "vsa_coarse_topk_noalloc", "vsa_sparse_attn", "vsa_sparse_attn_combine",
+           "vsa_gate_combine", "vsa_sync_status", "vsa_last_error")
 
 
 class VsaError(RuntimeError):
@@ -62,6 +63,8 @@ def lib():
             "vsa_workspace_size": [P, I, I, I, I, ctypes.POINTER(Z)],
             "vsa_permute": [P, V, V, I, I, I, V],
             "vsa_unpermute": [P, V, V, I, I, I, V],
+            "vsa_permute_pool": [P, V, V, I, I, I, V, V],
+            "vsa_coarse_topk_pooled": [P, I, I, I, F, I, V, V, V, V, Z, V],
             "vsa_coarse_topk": [P, V, V, V, I, I, I, F, I, V, V, V, V, Z, V],
             "vsa_coarse_topk_noalloc": [P, V, V, V, I, I, I, F, I, V, V, V, V],
             "vsa_sparse_attn": [P, V, V, V, V, I, I, I, I, F, V, V, V, Z, V],
@@ -214,6 +217,50 @@ def vsa_coarse_topk(plan: Plan, q_t, k_t, v_t, k: int, scale: Optional[float] = 
     return o_coarse, topk_idx, scores, ws
 
 
+def vsa_permute_pool(plan: Plan, x: torch.Tensor, x_t: Optional[torch.Tensor] = None,
+                     pooled: Optional[torch.Tensor] = None, stream=None):
+    """Permute x into x_t and write the fp32 per-tile means of its live rows to
+    pooled [B,H,T,D] in the same pass.  Returns (x_t, pooled)."""
+    B, H, N, D = x.shape
+    _need(x, "x", torch.bfloat16, (B, H, plan.n_tokens, D))
+    if x_t is None:
+        x_t = torch.empty(B, H, plan.n_padded, D, dtype=torch.bfloat16, device=x.device)
+    _need(x_t, "x_t", torch.bfloat16, (B, H, plan.n_padded, D))
+    if pooled is None:
+        pooled = torch.empty(B, H, plan.n_tiles, D, dtype=torch.float32, device=x.device)
+    _need(pooled, "pooled", torch.float32, (B, H, plan.n_tiles, D))
+    _check(lib().vsa_permute_pool(plan.handle, _ptr(x), _ptr(x_t), B, H, D, _ptr(pooled),
+                                  _stream(stream)))
+    return x_t, pooled
+
+
+def pooled_slots(plan: Plan, ws: torch.Tensor, B: int, H: int, D: int):
+    """Views of the workspace's qbar, kbar, vbar slots (fp32 [B,H,T,D] each)."""
+    n = B * H * plan.n_tiles * D
+    f = ws[: 3 * n * 4].view(torch.float32)
+    return tuple(f[i * n:(i + 1) * n].view(B, H, plan.n_tiles, D) for i in range(3))
+
+
+def vsa_coarse_topk_pooled(plan: Plan, B: int, H: int, D: int, k: int, ws, scale: Optional[float] = None,
+                           o_coarse=None, topk_idx=None, want_scores: bool = False, stream=None):
+    """vsa_coarse_topk from pooled means already in ``ws`` (written by
+    vsa_permute_pool into pooled_slots(ws)).  Returns (o_coarse, topk_idx,
+    scores or None)."""
+    dev = ws.device
+    scale = D ** -0.5 if scale is None else float(scale)
+    T, n_v = plan.n_tiles, plan.n_video_tiles
+    if o_coarse is None:
+        o_coarse = torch.empty(B, H, T, D, dtype=torch.float32, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty(B, H, n_v, max(k, 0), dtype=torch.int32, device=dev)
+    scores = torch.empty(B, H, n_v, max(k, 0), dtype=torch.float32, device=dev) if want_scores else None
+    _check(lib().vsa_coarse_topk_pooled(plan.handle, B, H, D, scale, k, _ptr(o_coarse),
+                                        _ptr(topk_idx) if topk_idx.numel() else None,
+                                        _ptr(scores) if scores is not None and scores.numel() else None,
+                                        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return o_coarse, topk_idx, scores
+
+
 def vsa_coarse_topk_noalloc(plan: Plan, q_t, k_t, v_t, k: int, scale: Optional[float] = None,
                             o_coarse=None, topk_idx=None, want_scores: bool = False, stream=None):
     """Like vsa_coarse_topk, but the library keeps the scratch in its own fixed
@@ -298,10 +345,11 @@ def vsa_sync_status(plan: Plan, stream=None):
 
 class Layer:
     """The five steps in sequence on caller-visible buffers, all launches on
-    one stream.  ``fused=True`` (default): permute Q, K, V; coarse + top-k;
-    attention with the gated combine fused into its epilogue, writing natural
-    order (the gate is read in natural order).  ``fused=False``: the unfused
-    chain (permute Q, K, V, G; coarse + top-k; attention; combine).  Buffers
+    one stream.  ``fused=True`` (default): permute Q, K, V with the tile means
+    taken in the same pass; coarse + top-k from those means; attention with
+    the gated combine fused into its epilogue, writing natural order (the gate
+    is read in natural order): 5 launches.  ``fused=False``: the unfused chain
+    (permute Q, K, V, G; pool + coarse + top-k; attention; combine).  Buffers
     are allocated once and reused by every call."""
 
     def __init__(self, plan: Plan, B: int, H: int, D: int, k: int, scale: Optional[float] = None,
@@ -321,15 +369,21 @@ class Layer:
 
     def __call__(self, q, k, v, g, stream=None):
         p = self.plan
+        if self.fused:
+            qbar, kbar, vbar = pooled_slots(p, self.ws, self.B, self.H, self.D)
+            vsa_permute_pool(p, q, self.q_t, qbar, stream)
+            vsa_permute_pool(p, k, self.k_t, kbar, stream)
+            vsa_permute_pool(p, v, self.v_t, vbar, stream)
+            vsa_coarse_topk_pooled(p, self.B, self.H, self.D, self.k, self.ws, self.scale,
+                                   o_coarse=self.o_coarse, topk_idx=self.topk_idx, stream=stream)
+            vsa_sparse_attn_combine(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, g,
+                                    self.o_coarse, self.scale, out=self.out, stream=stream)
+            return self.out
         vsa_permute(p, q, self.q_t, stream)
         vsa_permute(p, k, self.k_t, stream)
         vsa_permute(p, v, self.v_t, stream)
         vsa_coarse_topk(p, self.q_t, self.k_t, self.v_t, self.k, self.scale, ws=self.ws,
                         o_coarse=self.o_coarse, topk_idx=self.topk_idx, stream=stream)
-        if self.fused:
-            vsa_sparse_attn_combine(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, g,
-                                    self.o_coarse, self.scale, out=self.out, stream=stream)
-            return self.out
         vsa_permute(p, g, self.g_t, stream)
         vsa_sparse_attn(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, self.scale,
                         out=self.o_fine_t, stream=stream)
