@@ -227,6 +227,42 @@ def job_ms_per_layer(elapsed_max_ms: float, steps: int, world: int) -> float:
     return elapsed_max_ms / (steps * world)
 
 
+def projection_timing(w: Workload, plan, dev, stream, steps: int) -> dict:
+    """The gate projection of the layer (y = x W^T split into heads, the
+    tcgen05 GEMM behind vsa_project) at this workload's shape, inputs resident
+    (seeded on the device), timed with CUDA events; torch.matmul (cuBLAS) on
+    the same bf16 operands is timed beside it as a library reference."""
+    from tile_sparse_video_b200 import vsa
+    N, C, HD = plan.n_tokens, w.gate_width, w.H * w.D
+    g = torch.Generator(device=dev).manual_seed(w.seed_base + 7777)
+    x = torch.randn(1, N, C, device=dev, generator=g).to(torch.bfloat16)
+    wt = (torch.randn(HD, C, device=dev, generator=g) * w.gate_std).to(torch.bfloat16)
+    y = torch.empty(1, w.H, N, w.D, dtype=torch.bfloat16, device=dev)
+    x2 = x.view(N, C)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    ms = timed(lambda: vsa.vsa_project(plan, x, wt, w.H, w.D, y=y))
+    vsa.vsa_sync_status(plan)
+    ref_ms = timed(lambda: torch.matmul(x2, wt.t()))
+    flop = 2.0 * N * C * HD
+    peaks = load_peaks()
+    return {"shape": f"x[{N}x{C}] W[{HD}x{C}] -> [{w.H},{N},{w.D}]", "ms": round(ms, 4),
+            "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+            "frac": round(flop / (ms * 1e-3) / 1e12 / peaks["bf16"], 4),
+            "cublas_ms": round(ref_ms, 4), "gpu_launches_per_call": 1}
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     from tile_sparse_video_b200 import vsa
     import torch.distributed as dist
@@ -350,6 +386,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if not args.no_projection:
+        res["projection"] = projection_timing(w, plan, dev, stream, max(3, min(args.steps, 10)))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = oracle_sample(w, inp)
     if rank == 0:
@@ -390,6 +428,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
+    ap.add_argument("--no-projection", action="store_true", help="skip the gate projection timing")
     ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
                     help="profiling runs only: another named workload")
     ap.add_argument("--heads", type=int, default=0, help="profiling runs only: fewer heads")

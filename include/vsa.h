@@ -157,6 +157,18 @@ vsa_status vsa_coarse_topk_pooled(vsa_plan plan, int B, int H, int D, float scal
                                   float* o_coarse, int32_t* topk_idx, float* topk_score,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/* Head projection, the gate's bias-free linear (SnackOnAI, "The Code,
+ * Annotated", snippet three: gate = x W_gate^T viewed as [.., heads,
+ * head_dim]; with act = 0 any projection of that shape):
+ *   y[b,h,n,d] = act( sum_c x[b,n,c] * w[h*D+d, c] ),  act 0: identity, 1: sigmoid.
+ * x: bf16 [B,N,C] (N = the plan's real tokens, natural order), w: bf16 [H*D,C]
+ * (nn.Linear weight layout), y: bf16 [B,H,N,D] natural order, the layout
+ * vsa_sparse_attn_combine reads the gate in.  fp32 accumulation, bf16 round to
+ * nearest even.  All pointers 16-byte aligned, C a multiple of 8 (TMA row
+ * stride).  A tcgen05 GEMM on the device of the plan; asynchronous on `stream`. */
+vsa_status vsa_project(vsa_plan plan, const void* x, const void* w, int B, int H, int D, int C,
+                       int act, void* y, void* stream);
+
 /* Allocation-free variant of vsa_coarse_topk (the pages have no counterpart:
  * this is a library convenience).  For callers that cannot call cudaMalloc --
  * a host application that owns all device memory and gives plugins no

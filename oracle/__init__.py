@@ -5,4 +5,4 @@ benchmark's CPU-baseline leg, never by the product package.
 """
 from .vsa_oracle import (Plan, plan, keep_count, permute, unpermute, pool,  # noqa: F401
                          coarse_attention, select_topk, key_tiles, fine_tile, fine,
-                         sigmoid, gate_combine, layer)
+                         sigmoid, gate_combine, project, layer)

@@ -302,6 +302,24 @@ def gate_combine(o_fine, g_t, o_coarse, p: Plan):
     return out
 
 
+def project(x, w, n_heads: int, head_dim: int, act=None):
+    """Bias-free linear of the layer input, split into heads:
+    y[b, h, n, d] = act( sum_c x[b, n, c] * w[h*head_dim + d, c] ).
+
+    The gate is such a projection: [SNACK] snippet two computes ``gate_t`` as
+    ``to_gate_compress(x_t)`` viewed as [1, S, heads, head_dim], and snippet
+    three installs ``to_gate_compress`` as an ``nn.Linear`` without bias (weight
+    layout [out = heads*head_dim, in = width]).  ``act`` is None or "sigmoid".
+    x: [B, N, C], w: [H*D, C], any float dtype (converted exactly to fp64);
+    returns fp64 [B, H, N, D].
+    """
+    xf, wf = as_f64(x), as_f64(w)
+    y = xf @ wf.T                                        # [B, N, H*D]
+    B, N = y.shape[0], y.shape[1]
+    y = y.reshape(B, N, n_heads, head_dim).transpose(0, 2, 1, 3)
+    return sigmoid(y) if act == "sigmoid" else y
+
+
 # ---------------------------------------------------------------------------
 # The whole layer.
 # ---------------------------------------------------------------------------

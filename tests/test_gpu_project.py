@@ -1,0 +1,85 @@
+"""GPU parity of the head projection (vsa_project, a tcgen05 GEMM) against the
+fp64 oracle on the same bf16 inputs.
+
+Every output is one bf16 rounding (relative 2^-9) of an fp32 sum of C
+products; the bound checked is 2^-8 relative to the largest |y| of the
+output row plus 1e-6 absolute (fp32 accumulation over C <= 5376 terms
+contributes ~1e-6 relative).  Shapes cover a partial last M tile, H*D not a
+multiple of the 256-column N tile, C not a multiple of the 64-wide K block,
+D = 64 and 128, both activations, and B = 2 (rows of two batch elements in
+one M tile)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tile_sparse_video_b200 import vsa
+from tile_sparse_video_b200.inputs import SMALL, TINY, VEDA_104K, Workload, make_projection_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda(libvsa):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.synchronize()
+
+
+def _check(got, want):
+    got = got.to(torch.float64).cpu().numpy()
+    assert np.all(np.isfinite(got))
+    scale = np.abs(want).max(axis=-1, keepdims=True)
+    err = np.abs(got - want)
+    bound = 2.0 ** -8 * scale + 1e-6
+    assert np.all(err <= bound), float((err / (scale + 1e-30)).max())
+
+
+def _case(name, prefix, grid, tile, B, H, D, C, seed):
+    return Workload(name, B=B, H=H, D=D, prefix=prefix, grid=grid, tile=tile, keep_tiles=1,
+                    gate_width=C, gate_std=0.05, seed_base=seed)
+
+
+CASES = [
+    (_case("tiny_gate", TINY.prefix, TINY.grid, TINY.tile, 1, 2, 128, 64, 11), False),
+    (_case("d64_hd192_c200_b2", (40, 70), (4, 8, 8), (4, 4, 4), 2, 3, 64, 200, 12), True),
+    (_case("hd384_c520", (100,), (8, 16, 8), (4, 8, 4), 1, 3, 128, 520, 13), False),
+    (SMALL, True),
+]
+
+
+@pytest.mark.parametrize("w,sig", CASES, ids=lambda c: getattr(c, "name", str(c)))
+def test_projection_parity(w, sig):
+    inp = make_projection_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    y = vsa.vsa_project(plan, inp["x"].cuda(), inp["w"].cuda(), w.H, w.D, sigmoid=sig)
+    vsa.vsa_sync_status(plan)
+    want = O.project(inp["x"], inp["w"], w.H, w.D, act="sigmoid" if sig else None)
+    _check(y, want)
+
+
+def test_projection_full_size_sampled():
+    """The gate projection at the 104,704-token Veda size (C = 5,376 ->
+    42 x 128): every output of 96 sampled rows against fp64."""
+    w = VEDA_104K
+    inp = make_projection_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    y = vsa.vsa_project(plan, inp["x"].cuda(), inp["w"].cuda(), w.H, w.D)
+    vsa.vsa_sync_status(plan)
+    rows = np.sort(np.random.default_rng(3).choice(plan.n_tokens, 96, replace=False))
+    rows = np.unique(np.concatenate([rows, [0, plan.n_tokens - 1]]))
+    want = O.project(inp["x"][:, rows], inp["w"], w.H, w.D)
+    _check(y[:, :, rows], want)
+
+
+def test_projection_rejects_bad_arguments():
+    w = TINY
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    x = torch.zeros(1, plan.n_tokens, 60, dtype=torch.bfloat16, device="cuda")
+    wt = torch.zeros(256, 60, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(vsa.VsaError) as e:           # C not a multiple of 8
+        vsa.vsa_project(plan, x, wt, 2, 128)
+    assert e.value.status == 1
+    vsa.vsa_sync_status(plan)

@@ -301,6 +301,28 @@ def test_combine_limits():
     np.testing.assert_allclose(out[..., live, :], (of + 0.75 * oc[..., tile_of_row, :])[..., live, :], rtol=1e-14)
 
 
+def test_projection_closed_forms():
+    """The head projection against values fixed without its formula: a hand
+    computed 2x2 case, identity weights (y is x's columns split into heads),
+    a one-hot permutation of the output features (catches a transposed
+    operand or a head/dim mix-up), and sigmoid(0) = 1/2."""
+    y = O.project(np.array([[[1.0, 2.0]]]), np.array([[3.0, 4.0], [5.0, 6.0]]), 1, 2)
+    np.testing.assert_array_equal(y, [[[[11.0, 17.0]]]])          # [B=1, H=1, N=1, D=2]
+    rng = np.random.default_rng(8)
+    H, D, B, N = 3, 4, 2, 5
+    x = rng.standard_normal((B, N, H * D))
+    y = O.project(x, np.eye(H * D), H, D)
+    for h in range(H):
+        np.testing.assert_array_equal(y[:, h], x[:, :, h * D:(h + 1) * D])
+    perm = rng.permutation(H * D)
+    y = O.project(x, np.eye(H * D)[perm], H, D)                     # row f of W picks column perm[f]
+    for h in range(H):
+        for d in range(D):
+            np.testing.assert_array_equal(y[:, h, :, d], x[:, :, perm[h * D + d]])
+    y = O.project(x, np.zeros((H * D, H * D)), H, D, act="sigmoid")
+    assert np.all(y == 0.5)
+
+
 # --------------------------------------------------------------------------
 # Planted mistakes: each must make one of the pins above fail.
 # --------------------------------------------------------------------------
@@ -357,6 +379,23 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(V, "fine_tile", no_mask)
     assert _fails(lambda: test_fine_at_full_keep_is_dense_attention((40, 70), (4, 8, 8), (4, 4, 4)))
     monkeypatch.undo()
+
+    # 6. projection with the weight not transposed (x @ w instead of x @ w^T)
+    orig_project = V.project
+    def untransposed(x, w, n_heads, head_dim, act=None):
+        y = V.as_f64(x) @ V.as_f64(w)
+        B, N = y.shape[0], y.shape[1]
+        return y.reshape(B, N, n_heads, head_dim).transpose(0, 2, 1, 3)
+    monkeypatch.setattr(O, "project", untransposed)
+    assert _fails(test_projection_closed_forms)
+    # 7. heads and dims swapped in the split
+    def swapped(x, w, n_heads, head_dim, act=None):
+        y = V.as_f64(x) @ V.as_f64(w).T
+        B, N = y.shape[0], y.shape[1]
+        return y.reshape(B, N, head_dim, n_heads).transpose(0, 3, 1, 2)
+    monkeypatch.setattr(O, "project", swapped)
+    assert _fails(test_projection_closed_forms)
+    monkeypatch.setattr(O, "project", orig_project)
 
 
 def _high_tie_select(s, p, k):

@@ -279,6 +279,19 @@ vsa_status vsa_coarse_topk_pooled(vsa_plan p, int B, int H, int D, float scale, 
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "coarse_topk launch");
 }
 
+vsa_status vsa_project(vsa_plan p, const void* x, const void* w, int B, int H, int D, int C,
+                       int act, void* y, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  if (C <= 0 || C % 8 != 0) return fail(VSA_ERR_INVALID_ARG, "C must be a positive multiple of 8");
+  if (act != 0 && act != 1) return fail(VSA_ERR_INVALID_ARG, "act must be 0 (identity) or 1 (sigmoid)");
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(x, "x"));
+  VSA_TRY(check_ptr(w, "w"));
+  VSA_TRY(check_ptr(y, "y"));
+  return launch_project(p, x, w, B, H, D, C, act, y, static_cast<cudaStream_t>(stream));
+}
+
 vsa_status vsa_sparse_attn(vsa_plan p, const void* q_t, const void* k_t, const void* v_t,
                            const int32_t* topk_idx, int B, int H, int D, int k, float scale,
                            void* o_fine_t, float* lse_t, void* ws, size_t ws_bytes,

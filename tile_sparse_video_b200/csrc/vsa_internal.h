@@ -64,6 +64,9 @@ vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* 
                               int k, float scale, void* out, float* lse_t, const void* gate,
                               const float* o_coarse, cudaStream_t stream);
 
+vsa_status launch_project(const vsa_plan_s* p, const void* x, const void* w, int B, int H, int D,
+                          int C, int act, void* y, cudaStream_t stream);
+
 // Device status codes written by kernels into vsa_plan_s::d_status.
 enum : unsigned int { kStatusOk = 0, kStatusTimeout = 1, kStatusBadIndex = 2 };
 

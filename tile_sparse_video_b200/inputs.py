@@ -198,3 +198,19 @@ def make_inputs(w: Workload, batch: Optional[Sequence[int]] = None,
                 if h in hsel:
                     out["g"][bi, hsel.index(h)] = _bf16(x)
     return out
+
+
+def make_projection_inputs(w: Workload, batch: Optional[Sequence[int]] = None) -> dict:
+    """Draw the inputs of a head projection for workload ``w``: the layer input
+    x ~ N(0, 1) [B, N, C] and a bias-free weight W ~ N(0, gate_std^2)
+    [H*D, C], C = gate_width, both rounded to bf16 (the gate projection's
+    shapes; its own seed stream, separate from Q/K/V/G)."""
+    bsel = list(range(w.B)) if batch is None else list(batch)
+    N, C, HD = w.n_tokens, w.gate_width, w.H * w.D
+    gen = torch.Generator().manual_seed(w.seed_base + 7777)
+    weight = _bf16(torch.randn(HD, C, generator=gen) * w.gate_std)
+    x = torch.empty(len(bsel), N, C, dtype=torch.bfloat16)
+    for bi, b in enumerate(bsel):
+        g = torch.Generator().manual_seed(w.seed_base + 7777 + 17 * (b + 1))
+        x[bi] = _bf16(torch.randn(N, C, generator=g))
+    return {"x": x, "w": weight}

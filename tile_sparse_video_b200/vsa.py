@@ -28,7 +28,7 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_coun
            "vsa_plan_destroy", "vsa_workspace_size", "vsa_permute", "vsa_unpermute",
            "vsa_permute_pool", "vsa_coarse_topk", "vsa_coarse_topk_pooled",
            "vsa_coarse_topk_noalloc", "vsa_sparse_attn", "vsa_sparse_attn_combine",
-           "vsa_gate_combine", "vsa_sync_status", "vsa_last_error")
+           "vsa_gate_combine", "vsa_project", "vsa_sync_status", "vsa_last_error")
 
 
 class VsaError(RuntimeError):
@@ -70,6 +70,7 @@ def lib():
             "vsa_sparse_attn": [P, V, V, V, V, I, I, I, I, F, V, V, V, Z, V],
             "vsa_sparse_attn_combine": [P, V, V, V, V, I, I, I, I, F, V, V, V, V, V],
             "vsa_gate_combine": [P, V, V, V, V, I, I, I, I, V],
+            "vsa_project": [P, V, V, I, I, I, I, I, V, V],
             "vsa_sync_status": [P, V],
         }
         for name, args in sig.items():
@@ -337,6 +338,21 @@ def vsa_gate_combine(plan: Plan, o_fine_t, gate_t, o_coarse, natural: bool = Tru
     _check(lib().vsa_gate_combine(plan.handle, _ptr(o_fine_t), _ptr(gate_t), _ptr(o_coarse), _ptr(out),
                                   1 if natural else 0, B, H, D, _stream(stream)))
     return out
+
+
+def vsa_project(plan: Plan, x: torch.Tensor, w: torch.Tensor, H: int, D: int, sigmoid: bool = False,
+                y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y[b,h,n,d] = act(sum_c x[b,n,c] w[h*D+d,c]) (tcgen05 GEMM; act = sigmoid or
+    identity).  x bf16 [B,N,C], w bf16 [H*D,C]; returns y bf16 [B,H,N,D]."""
+    B, N, C = x.shape
+    _need(x, "x", torch.bfloat16, (B, plan.n_tokens, C))
+    _need(w, "w", torch.bfloat16, (H * D, C))
+    if y is None:
+        y = torch.empty(B, H, plan.n_tokens, D, dtype=torch.bfloat16, device=x.device)
+    _need(y, "y", torch.bfloat16, (B, H, plan.n_tokens, D))
+    _check(lib().vsa_project(plan.handle, _ptr(x), _ptr(w), B, H, D, C, 1 if sigmoid else 0, _ptr(y),
+                             _stream(stream)))
+    return y
 
 
 def vsa_sync_status(plan: Plan, stream=None):
