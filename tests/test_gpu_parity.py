@@ -264,3 +264,24 @@ def test_empty_batch_is_a_no_op():
     x = torch.empty(0, 2, plan.n_tokens, 64, dtype=torch.bfloat16, device="cuda")
     assert vsa.vsa_permute(plan, x).shape == (0, 2, plan.n_padded, 64)
     vsa.vsa_sync_status(plan)
+
+
+def test_layer_pipeline_matches_layer():
+    """vsa.LayerPipeline (copy-in, compute and copy-out of consecutive layers
+    overlapped on three streams, two buffer sets) gives bit-identical outputs
+    to calling the Layer once per input set, for more layers than buffers."""
+    from dataclasses import replace
+    w = SMALL
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    sets = [make_inputs(replace(w, seed_base=w.seed_base + 31 * i)) for i in range(5)]
+    host = [{n: s[n].pin_memory() for n in "qkvg"} for s in sets]
+    outs = [torch.empty(w.B, w.H, plan.n_tokens, w.D, dtype=torch.bfloat16).pin_memory() for _ in sets]
+    pipe = vsa.LayerPipeline(plan, w.B, w.H, w.D, k)
+    pipe.run(host, outs)
+    torch.cuda.synchronize()
+    layer = vsa.Layer(plan, w.B, w.H, w.D, k)
+    for s, got in zip(sets, outs):
+        want = layer(*(s[n].cuda() for n in "qkvg")).cpu()
+        assert torch.equal(got, want)
+    vsa.vsa_sync_status(plan)

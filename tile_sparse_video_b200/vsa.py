@@ -406,3 +406,67 @@ class Layer:
         vsa_gate_combine(p, self.o_fine_t, self.g_t, self.o_coarse, natural=True, out=self.out,
                          stream=stream)
         return self.out
+
+
+class LayerPipeline:
+    """Layers over host-resident inputs with the transfers overlapped: while
+    layer i computes, the inputs of layer i+1 are copied in and the output of
+    layer i-1 is copied out (three CUDA streams, ``depth`` sets of device
+    buffers, one Layer per set).  Host tensors must be pinned for the copies
+    to run asynchronously.  Each layer is the fused Layer above; results are
+    the same as calling it once per input set."""
+
+    def __init__(self, plan: Plan, B: int, H: int, D: int, k: int, scale: Optional[float] = None,
+                 device=None, depth: int = 2):
+        if depth < 1:
+            raise ValueError("depth must be >= 1")
+        dev = torch.device("cuda", plan.device) if device is None else torch.device(device)
+        self.plan, self.depth, self.dev = plan, depth, dev
+        self.layers = [Layer(plan, B, H, D, k, scale, dev) for _ in range(depth)]
+        shape = (B, H, plan.n_tokens, D)
+        self.inputs = [{n: torch.empty(shape, dtype=torch.bfloat16, device=dev) for n in "qkvg"}
+                       for _ in range(depth)]
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_comp = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+
+    def run(self, host_inputs: Sequence[dict], host_outputs: Sequence[torch.Tensor],
+            start_event=None, end_event=None):
+        """Layer i reads host_inputs[i] (dict of pinned "q", "k", "v", "g"
+        [B,H,N,D] bf16) and writes host_outputs[i] (pinned [B,H,N,D] bf16).
+        Asynchronous: returns the event recorded after the last copy-out.
+        ``start_event`` / ``end_event`` (CUDA timing events) are recorded
+        before the first copy-in and after the last copy-out."""
+        n = len(host_inputs)
+        if len(host_outputs) != n:
+            raise ValueError("one output per input set")
+        mk = lambda: torch.cuda.Event()
+        ev_in, ev_comp, ev_out = [mk() for _ in range(n)], [mk() for _ in range(n)], [mk() for _ in range(n)]
+        # the new streams start after everything already queued on the current one
+        here = torch.cuda.current_stream(self.dev)
+        for st in (self.s_in, self.s_comp, self.s_out):
+            st.wait_stream(here)
+        if start_event is not None:
+            start_event.record(self.s_in)
+        for i in range(n):
+            b = i % self.depth
+            buf, layer = self.inputs[b], self.layers[b]
+            if i >= self.depth:
+                self.s_in.wait_event(ev_comp[i - self.depth])      # buffer set b read by layer i-depth
+            with torch.cuda.stream(self.s_in):
+                for name in "qkvg":
+                    buf[name].copy_(host_inputs[i][name], non_blocking=True)
+            ev_in[i].record(self.s_in)
+            self.s_comp.wait_event(ev_in[i])
+            if i >= self.depth:
+                self.s_comp.wait_event(ev_out[i - self.depth])     # layer b's output copied out
+            layer(buf["q"], buf["k"], buf["v"], buf["g"], stream=self.s_comp)
+            ev_comp[i].record(self.s_comp)
+            self.s_out.wait_event(ev_comp[i])
+            with torch.cuda.stream(self.s_out):
+                host_outputs[i].copy_(layer.out, non_blocking=True)
+            ev_out[i].record(self.s_out)
+        if end_event is not None:
+            end_event.record(self.s_out)
+        here.wait_event(ev_out[n - 1])
+        return ev_out[n - 1]
