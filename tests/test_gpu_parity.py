@@ -9,6 +9,8 @@ the fp64 oracle on the same seeded bf16 inputs.
 * the full-size workloads in the benchmark's launch configuration, on sampled
   heads and query tiles the oracle computes one by one.
 """
+from dataclasses import replace
+
 import numpy as np
 import pytest
 import torch
@@ -215,8 +217,9 @@ def _sampled(w: Workload, heads, n_video_samples, seed):
     assert n_near <= max(2, w.B * len(heads) * p.n_video_tiles // 50)
 
 
-@pytest.mark.parametrize("w,heads,n", [(REF2VA, (0, 17, 41), 24), (VEDA_104K, (0, 23, 41), 16)],
-                         ids=["ref2va_full", "veda_104k_full"])
+@pytest.mark.parametrize("w,heads,n", [(REF2VA, (0, 17, 41), 24), (VEDA_104K, (0, 23, 41), 16),
+                                       (replace(VEDA_104K, name="veda_h56", H=56), (0, 55), 8)],
+                         ids=["ref2va_full", "veda_104k_full", "veda_h56_full"])
 def test_full_size_sampled(w, heads, n):
     _sampled(w, heads, n, seed=11)
 

@@ -60,10 +60,13 @@ def test_projection_parity(w, sig):
     _check(y, want)
 
 
-def test_projection_full_size_sampled():
+@pytest.mark.parametrize("H", [42, 56], ids=["h42", "h56"])
+def test_projection_full_size_sampled(H):
     """The gate projection at the 104,704-token Veda size (C = 5,376 ->
-    42 x 128): every output of 96 sampled rows against fp64."""
-    w = VEDA_104K
+    42 x 128, and the 56-head layout with inner width 7,168): every output of
+    98 sampled rows against fp64."""
+    from dataclasses import replace
+    w = VEDA_104K if H == VEDA_104K.H else replace(VEDA_104K, name=f"veda_h{H}", H=H)
     inp = make_projection_inputs(w)
     plan = vsa.Plan(w.prefix, w.grid, w.tile)
     y = vsa.vsa_project(plan, inp["x"].cuda(), inp["w"].cuda(), w.H, w.D)

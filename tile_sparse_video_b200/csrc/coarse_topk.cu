@@ -22,13 +22,21 @@
 namespace vsa {
 namespace {
 
-constexpr int kKC = 64;                // key / value tiles per staged chunk
+#ifndef VSA_COARSE_KC
+#define VSA_COARSE_KC 64
+#endif
+constexpr int kKC = VSA_COARSE_KC;     // key / value tiles per staged chunk
 // Warps per CTA for T <= 960 (32 query tiles per CTA, 32 / NW per warp).
+static_assert(kKC % 32 == 0, "staged chunk: a multiple of 32 tiles");
 // Fewer warps with more rows each reuse more registers but hide less
 // latency: at the 104k-token Veda layer 16 warps take 1.39 ms, 8 warps
-// 1.69 ms, 4 warps 2.93 ms on B200.
+// 1.69 ms, 4 warps 2.93 ms on B200.  Two CTAs per SM (32-tile chunks, 8
+// warps x 2 rows) measured 1.32 ms, within the run-to-run spread of the layer.
 #ifndef VSA_COARSE_NW
 #define VSA_COARSE_NW 16
+#endif
+#ifndef VSA_COARSE_RW
+#define VSA_COARSE_RW (32 / VSA_COARSE_NW)
 #endif
 constexpr int kMaxTiles = 4096;        // bound on T (shared-memory budget)
 
@@ -167,33 +175,40 @@ __global__ void __launch_bounds__(NW * 32) coarse_topk_kernel(
       cp_async_wait<0>();
     }
     __syncthreads();
-    float acc[RW][2];
+    constexpr int KPL = kKC / 32;                  // keys per lane: lane, lane + 32, ...
+    float acc[RW][KPL];
 #pragma unroll
-    for (int r = 0; r < RW; ++r) acc[r][0] = acc[r][1] = 0.f;
-    const float4* k0 = reinterpret_cast<const float4*>(stage + lane * kStride);
-    const float4* k1 = reinterpret_cast<const float4*>(stage + (lane + 32) * kStride);
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int u = 0; u < KPL; ++u) acc[r][u] = 0.f;
     const float* qw = qT + warp * RW;
 #pragma unroll 4
     for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 a0 = k0[d4], a1 = k1[d4];
-      const float a0v[4] = {a0.x, a0.y, a0.z, a0.w};
-      const float a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+      float av[KPL][4];
+#pragma unroll
+      for (int u = 0; u < KPL; ++u) {
+        const float4 a = reinterpret_cast<const float4*>(stage + (lane + 32 * u) * kStride)[d4];
+        av[u][0] = a.x;
+        av[u][1] = a.y;
+        av[u][2] = a.z;
+        av[u][3] = a.w;
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float q[RW];
         QVec<RW>::load(qw + (4 * d4 + e) * QB, q);
 #pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          acc[r][0] = fmaf(q[r], a0v[e], acc[r][0]);
-          acc[r][1] = fmaf(q[r], a1v[e], acc[r][1]);
-        }
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+          for (int u = 0; u < KPL; ++u) acc[r][u] = fmaf(q[r], av[u][e], acc[r][u]);
       }
     }
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
       float* row = sc + (warp * RW + r) * Tpad + j0;
-      if (lane < nj) row[lane] = scale * acc[r][0];
-      if (lane + 32 < nj) row[lane + 32] = scale * acc[r][1];
+#pragma unroll
+      for (int u = 0; u < KPL; ++u)
+        if (lane + 32 * u < nj) row[lane + 32 * u] = scale * acc[r][u];
     }
     __syncthreads();     // stage (c & 1) is refilled two chunks later
   }
@@ -370,7 +385,7 @@ cudaError_t launch_coarse_d(const float* qbar, const float* kbar, const float* v
   // 16 warps per CTA (one CTA fills an SM's shared memory), and as many query
   // tiles per CTA as the score rows leave room for
   if (T <= 960)
-    return launch_coarse_cfg<D, VSA_COARSE_NW, 32 / VSA_COARSE_NW>(
+    return launch_coarse_cfg<D, VSA_COARSE_NW, VSA_COARSE_RW>(
         qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx, topk_score, stream);
   if (T <= 1920)
     return launch_coarse_cfg<D, 16, 1>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
