@@ -151,6 +151,19 @@ def keep_count(n_video_tiles: int, n_prefix_tiles: int, keep_ratio=None,
     return k
 
 
+def keep_count_ref(n_prefix_tiles: int, keep_ratio=None, keep_tiles=None) -> int:
+    """Number of reference (prefix) key tiles each video query tile keeps when
+    the reference tiles are thinned too ([VEDA] input table: reference_sparsity
+    applies "the same setting" to the reference tokens; 0 % is full attention).
+    Reading: the keep rule of ``keep_count`` applied to the n_p reference tiles
+    (ratio mode ceil(clamp(keep_ratio, 0, 1) * n_p - 1e-9); integer mode
+    min(keep_tiles, n_p)), so keep_ratio = 1 keeps every reference tile."""
+    if keep_tiles is not None and keep_tiles >= 0:
+        return min(int(keep_tiles), n_prefix_tiles)
+    r = min(1.0, max(0.0, float(keep_ratio)))
+    return min(n_prefix_tiles, int(math.ceil(r * n_prefix_tiles - 1e-9)))
+
+
 # ---------------------------------------------------------------------------
 # Step 1 (data movement): permute into / out of the padded tile layout.
 # ---------------------------------------------------------------------------
@@ -228,13 +241,33 @@ def select_topk(s: np.ndarray, p: Plan, k: int) -> np.ndarray:
     return out
 
 
-def key_tiles(p: Plan, i: int, kept_row) -> np.ndarray:
+def select_topk_ref(s: np.ndarray, p: Plan, k_ref: int) -> np.ndarray:
+    """For each video query tile i and head: the k_ref reference (prefix) key
+    tiles with the highest coarse score s[i, j], j < n_p, ties towards the
+    lower index, in ascending order.  Reading of [VEDA] reference_sparsity:
+    the reference key tiles are thinned by the same per-head top-k as the
+    generated-video ones, with their own keep count (``keep_count_ref``);
+    reference query tiles stay dense.  Result: int64 [.., n_v, k_ref]."""
+    n_p, T = p.n_prefix_tiles, p.n_tiles
+    lead = s.shape[:-2]
+    out = np.zeros(lead + (T - n_p, k_ref), dtype=np.int64)
+    cand = np.arange(n_p)
+    for idx in np.ndindex(*lead):
+        for i in range(n_p, T):
+            order = np.lexsort((cand, -s[idx + (i,)][:n_p]))
+            out[idx + (i - n_p,)] = np.sort(cand[order[:k_ref]])
+    return out
+
+
+def key_tiles(p: Plan, i: int, kept_row, kept_ref_row=None) -> np.ndarray:
     """Key tile set of query tile i: all tiles for a prefix query tile (prefix
-    queries attend densely, [SNACK] snippet two ``sink_q``); the prefix sinks
-    plus the kept video tiles for a video query tile (``sink_blocks``)."""
+    queries attend densely, [SNACK] snippet two ``sink_q``); for a video query
+    tile the prefix sinks (or, with reference thinning, its kept reference
+    tiles ``kept_ref_row``) plus its kept video tiles (``sink_blocks``)."""
     if i < p.n_prefix_tiles:
         return np.arange(p.n_tiles)
-    return np.concatenate([np.arange(p.n_prefix_tiles), np.asarray(kept_row, dtype=np.int64)])
+    ref = np.arange(p.n_prefix_tiles) if kept_ref_row is None else np.asarray(kept_ref_row, dtype=np.int64)
+    return np.concatenate([ref, np.asarray(kept_row, dtype=np.int64)])
 
 
 # ---------------------------------------------------------------------------
@@ -258,9 +291,10 @@ def fine_tile(q_t, k_t, v_t, p: Plan, i: int, tiles, scale):
     return (e @ vv) / l, (m + np.log(l))[:, 0]
 
 
-def fine(q_t, k_t, v_t, p: Plan, kept, scale):
+def fine(q_t, k_t, v_t, p: Plan, kept, scale, kept_ref=None):
     """o_fine for every live row of every tile (pad rows zero), and its
-    log-sum-exp.  q_t, k_t, v_t: [B, H, N_pad, D]; kept: [B, H, n_v, k]."""
+    log-sum-exp.  q_t, k_t, v_t: [B, H, N_pad, D]; kept: [B, H, n_v, k];
+    kept_ref (optional): [B, H, n_v, k_ref] kept reference tiles."""
     B, H = q_t.shape[:2]
     o = np.zeros(q_t.shape, dtype=np.float64)
     lse = np.zeros(q_t.shape[:-1], dtype=np.float64)
@@ -268,8 +302,10 @@ def fine(q_t, k_t, v_t, p: Plan, kept, scale):
         for h in range(H):
             for i in range(p.n_tiles):
                 row = kept[b, h, i - p.n_prefix_tiles] if i >= p.n_prefix_tiles else None
+                ref = (kept_ref[b, h, i - p.n_prefix_tiles]
+                       if kept_ref is not None and i >= p.n_prefix_tiles else None)
                 oi, li = fine_tile(q_t[b, h], k_t[b, h], v_t[b, h], p, i,
-                                   key_tiles(p, i, row), scale)
+                                   key_tiles(p, i, row, ref), scale)
                 n = p.block_len[i]
                 o[b, h, i * p.R: i * p.R + n] = oi
                 lse[b, h, i * p.R: i * p.R + n] = li
@@ -333,19 +369,27 @@ def as_f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def layer(q, k, v, g, p: Plan, kk: int, scale=None, kept=None):
+def layer(q, k, v, g, p: Plan, kk: int, scale=None, kept=None, k_ref=None, kept_ref=None):
     """Steps 1-5 on natural-order inputs [B, H, N, D] (any float dtype,
     converted exactly to fp64).  ``kept`` overrides the top-k selection (used
-    to evaluate the oracle under another legal tie-break).  Returns a dict of
-    every intermediate, all fp64 except the integer selection."""
+    to evaluate the oracle under another legal tie-break).  ``k_ref`` (None:
+    every reference tile is a sink) thins the reference key tiles of video
+    query tiles to their top k_ref; ``kept_ref`` overrides that selection.
+    Returns a dict of every intermediate, all fp64 except the integer
+    selections."""
     D = q.shape[-1]
     scale = D ** -0.5 if scale is None else scale
     q_t, k_t, v_t, g_t = (permute(as_f64(x), p) for x in (q, k, v, g))
     qbar, kbar, vbar = pool(q_t, p), pool(k_t, p), pool(v_t, p)
     s, o_coarse = coarse_attention(qbar, kbar, vbar, scale)
     sel = select_topk(s, p, kk) if kept is None else np.asarray(kept, dtype=np.int64)
-    o_fine, lse = fine(q_t, k_t, v_t, p, sel, scale)
+    sel_ref = None
+    if kept_ref is not None:
+        sel_ref = np.asarray(kept_ref, dtype=np.int64)
+    elif k_ref is not None:
+        sel_ref = select_topk_ref(s, p, k_ref)
+    o_fine, lse = fine(q_t, k_t, v_t, p, sel, scale, sel_ref)
     out_t = gate_combine(o_fine, g_t, o_coarse, p)
     return dict(q_t=q_t, k_t=k_t, v_t=v_t, g_t=g_t, qbar=qbar, kbar=kbar, vbar=vbar,
-                scores=s, o_coarse=o_coarse, topk=sel, o_fine=o_fine, lse=lse,
+                scores=s, o_coarse=o_coarse, topk=sel, topk_ref=sel_ref, o_fine=o_fine, lse=lse,
                 out_t=out_t, out=unpermute(out_t, p))

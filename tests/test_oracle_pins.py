@@ -214,6 +214,53 @@ def test_topk_matches_brute_force_with_ties(seed):
                 assert np.array_equal(sel[h, i - n_p], want)
 
 
+@pytest.mark.parametrize("seed", [0, 1])
+def test_reference_topk_matches_brute_force_with_ties(seed):
+    rng = np.random.default_rng(100 + seed)
+    p = O.plan((64, 64, 64, 64, 30), (4, 8, 8), (4, 4, 4))   # n_p = 5 reference tiles
+    T, n_p = p.n_tiles, p.n_prefix_tiles
+    s = rng.integers(0, 3, size=(2, T, T)).astype(np.float64)   # many exact ties
+    for k_ref in (0, 1, 2, 4, n_p):
+        sel = O.select_topk_ref(s, p, k_ref)
+        for h in range(2):
+            for i in range(n_p, T):
+                assert np.array_equal(sel[h, i - n_p], brute_topk(s[h, i, :n_p], k_ref))
+
+
+def test_reference_keep_count():
+    # 26 reference tiles (the pages' H3 prefix) at 90 % -> 3; at 0 % -> all (full attention)
+    assert O.keep_count_ref(26, keep_ratio=0.10) == 3
+    assert O.keep_count_ref(26, keep_ratio=1.0) == 26
+    assert O.keep_count_ref(2, keep_ratio=0.10) == 1
+    assert O.keep_count_ref(26, keep_tiles=24) == 24 and O.keep_count_ref(5, keep_tiles=24) == 5
+
+
+def test_reference_thinning_reduces_and_restricts():
+    """k_ref = n_p keeps every reference tile: the layer is the unthinned one.
+    With k_ref < n_p a video query row attends exactly to the tokens of its
+    kept reference tiles and kept video tiles (library attention over them)."""
+    prefix, grid, tile = (40, 70, 30), (8, 8, 8), (4, 4, 4)
+    p = O.plan(prefix, grid, tile)
+    _, tiles, _, _ = coord_rows(prefix, grid, tile)
+    rng = np.random.default_rng(9)
+    q, k, v, g = (rng.standard_normal((1, 2, p.n_tokens, 16)) for _ in range(4))
+    base = O.layer(q, k, v, g, p, 3, scale=0.25)
+    full = O.layer(q, k, v, g, p, 3, scale=0.25, k_ref=p.n_prefix_tiles)
+    np.testing.assert_array_equal(full["out"], base["out"])
+    res = O.layer(q, k, v, g, p, 3, scale=0.25, k_ref=1)
+    of = O.unpermute(res["o_fine"], p)
+    n_prefix_tok = sum(prefix)
+    np.testing.assert_array_equal(of[:, :, :n_prefix_tok], O.unpermute(base["o_fine"], p)[:, :, :n_prefix_tok])
+    for h in range(2):
+        for n in range(n_prefix_tok, p.n_tokens, 11):
+            i = tiles[n]
+            allowed = (set(res["topk_ref"][0, h, i - p.n_prefix_tiles].tolist())
+                       | set(res["topk"][0, h, i - p.n_prefix_tiles].tolist()))
+            keys = np.array([m for m in range(p.n_tokens) if tiles[m] in allowed])
+            want = sdpa64(q[0, h, n:n + 1], k[0, h, keys], v[0, h, keys], 0.25)
+            np.testing.assert_allclose(of[0, h, n:n + 1], want, rtol=1e-11, atol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # Fine attention
 # --------------------------------------------------------------------------
@@ -379,6 +426,21 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(V, "fine_tile", no_mask)
     assert _fails(lambda: test_fine_at_full_keep_is_dense_attention((40, 70), (4, 8, 8), (4, 4, 4)))
     monkeypatch.undo()
+
+    # 6'. reference ties broken towards the higher index
+    orig_ref = V.select_topk_ref
+    def high_tie_ref(s, p, k_ref):
+        n_p, T = p.n_prefix_tiles, p.n_tiles
+        out = np.zeros(s.shape[:-2] + (T - n_p, k_ref), dtype=np.int64)
+        cand = np.arange(n_p)
+        for idx in np.ndindex(*s.shape[:-2]):
+            for i in range(n_p, T):
+                order = np.lexsort((-cand, -s[idx + (i,)][:n_p]))
+                out[idx + (i - n_p,)] = np.sort(cand[order[:k_ref]])
+        return out
+    monkeypatch.setattr(O, "select_topk_ref", high_tie_ref)
+    assert _fails(lambda: test_reference_topk_matches_brute_force_with_ties(0))
+    monkeypatch.setattr(O, "select_topk_ref", orig_ref)
 
     # 6. projection with the weight not transposed (x @ w instead of x @ w^T)
     orig_project = V.project
