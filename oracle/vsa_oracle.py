@@ -393,3 +393,129 @@ def layer(q, k, v, g, p: Plan, kk: int, scale=None, kept=None, k_ref=None, kept_
     return dict(q_t=q_t, k_t=k_t, v_t=v_t, g_t=g_t, qbar=qbar, kbar=kbar, vbar=vbar,
                 scores=s, o_coarse=o_coarse, topk=sel, topk_ref=sel_ref, o_fine=o_fine, lse=lse,
                 out_t=out_t, out=unpermute(out_t, p))
+
+
+# ---------------------------------------------------------------------------
+# The backward pass: gradients of a scalar loss through steps 5 .. 1.
+#
+# The method is trained end to end ([SNACK] "The Architecture, Unpacked":
+# the coarse stage and the gate are learned; the VSA paper it builds on
+# trains the sparse kernel).  Reading: the top-k selection is an index choice
+# and passes no gradient (it is piecewise constant in the scores); gradients
+# flow through the coarse branch (pooling, coarse attention), the fine
+# attention over the selected tiles and the gate.  Every function takes the
+# upstream gradient of its output and returns the gradients of its inputs,
+# written from the definitions of the forward steps above.
+# ---------------------------------------------------------------------------
+
+def gate_combine_backward(d_out_t, o_fine, g_t, o_coarse, p: Plan):
+    """Backward of out = o_fine + sigmoid(g) * o_coarse[tile(row)] (live rows).
+
+    Returns (d_o_fine [.., N_pad, D], d_g_t [.., N_pad, D],
+    d_o_coarse [.., T, D]); pad rows carry no gradient.
+    """
+    tile_of_row = np.repeat(np.arange(p.n_tiles), p.R)
+    live = p.row_src >= 0
+    d = np.array(d_out_t, dtype=np.float64)
+    d[..., ~live, :] = 0.0
+    sg = sigmoid(g_t.astype(np.float64))
+    d_o_fine = d.copy()
+    d_g_t = d * o_coarse[..., tile_of_row, :] * sg * (1.0 - sg)
+    d_o_coarse = np.zeros(o_coarse.shape, dtype=np.float64)
+    for t in range(p.n_tiles):
+        rows = slice(t * p.R, t * p.R + p.block_len[t])
+        d_o_coarse[..., t, :] = (d[..., rows, :] * sg[..., rows, :]).sum(axis=-2)
+    return d_o_fine, d_g_t, d_o_coarse
+
+
+def softmax_backward(prob, d_prob):
+    """Row-wise softmax Jacobian applied to an upstream gradient:
+    d_s = prob * (d_prob - sum_j prob_j d_prob_j)."""
+    return prob * (d_prob - (prob * d_prob).sum(axis=-1, keepdims=True))
+
+
+def fine_tile_backward(q_t, k_t, v_t, p: Plan, i: int, tiles, scale, d_o):
+    """Backward of ``fine_tile`` for one head: given d_o [block_len[i], D],
+    the gradients of the query rows of tile i and of the key / value rows
+    of ``tiles`` (as (rows, dq, dk, dv): the key rows in ``tiles`` order)."""
+    rows = np.concatenate([j * p.R + np.arange(p.block_len[j]) for j in tiles])
+    q = q_t[i * p.R: i * p.R + p.block_len[i]].astype(np.float64)
+    kk = k_t[rows].astype(np.float64)
+    vv = v_t[rows].astype(np.float64)
+    s = scale * (q @ kk.T)
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    prob = e / e.sum(axis=1, keepdims=True)
+    dv = prob.T @ d_o
+    d_s = softmax_backward(prob, d_o @ vv.T)
+    dq = scale * (d_s @ kk)
+    dk = scale * (d_s.T @ q)
+    return rows, dq, dk, dv
+
+
+def fine_backward(q_t, k_t, v_t, p: Plan, kept, scale, d_o_fine, kept_ref=None):
+    """Backward of ``fine``: gradients of q_t, k_t, v_t [B, H, N_pad, D]
+    (pad rows zero) for the upstream d_o_fine, under the fixed selection."""
+    B, H = q_t.shape[:2]
+    dq = np.zeros(q_t.shape, dtype=np.float64)
+    dk = np.zeros(k_t.shape, dtype=np.float64)
+    dv = np.zeros(v_t.shape, dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for i in range(p.n_tiles):
+                row = kept[b, h, i - p.n_prefix_tiles] if i >= p.n_prefix_tiles else None
+                ref = (kept_ref[b, h, i - p.n_prefix_tiles]
+                       if kept_ref is not None and i >= p.n_prefix_tiles else None)
+                qrows = slice(i * p.R, i * p.R + p.block_len[i])
+                rows, dqi, dki, dvi = fine_tile_backward(
+                    q_t[b, h], k_t[b, h], v_t[b, h], p, i, key_tiles(p, i, row, ref), scale,
+                    np.asarray(d_o_fine[b, h, qrows], dtype=np.float64))
+                dq[b, h, qrows] += dqi
+                np.add.at(dk[b, h], rows, dki)
+                np.add.at(dv[b, h], rows, dvi)
+    return dq, dk, dv
+
+
+def coarse_attention_backward(qbar, kbar, vbar, scale, d_o_coarse):
+    """Backward of ``coarse_attention``: (d_qbar, d_kbar, d_vbar), fp64."""
+    s = scale * (qbar @ np.swapaxes(kbar, -1, -2))
+    e = np.exp(s - s.max(axis=-1, keepdims=True))
+    prob = e / e.sum(axis=-1, keepdims=True)
+    d_vbar = np.swapaxes(prob, -1, -2) @ d_o_coarse
+    d_s = softmax_backward(prob, d_o_coarse @ np.swapaxes(vbar, -1, -2))
+    d_qbar = scale * (d_s @ kbar)
+    d_kbar = scale * (np.swapaxes(d_s, -1, -2) @ qbar)
+    return d_qbar, d_kbar, d_vbar
+
+
+def pool_backward(d_bar, p: Plan):
+    """Backward of ``pool``: each live row of tile t receives d_bar[t] /
+    block_len[t]; pad rows receive nothing.  Returns [.., N_pad, D]."""
+    out = np.zeros(d_bar.shape[:-2] + (p.n_padded, d_bar.shape[-1]), dtype=np.float64)
+    for t in range(p.n_tiles):
+        n = p.block_len[t]
+        out[..., t * p.R: t * p.R + n, :] = d_bar[..., t: t + 1, :] / n
+    return out
+
+
+def layer_backward(d_out, fwd: dict, p: Plan, scale=None):
+    """Gradients of the loss sum(d_out * out) with respect to the natural-order
+    inputs q, k, v, g [B, H, N, D] of ``layer`` (``fwd`` is its result), under
+    the forward's selection.  Returns a dict with dq, dk, dv, dg (natural
+    order) and the tiled intermediates, all fp64."""
+    D = fwd["q_t"].shape[-1]
+    scale = D ** -0.5 if scale is None else scale
+    d_out_t = permute(as_f64(d_out), p)
+    d_o_fine, d_g_t, d_o_coarse = gate_combine_backward(d_out_t, fwd["o_fine"], fwd["g_t"],
+                                                        fwd["o_coarse"], p)
+    dq_f, dk_f, dv_f = fine_backward(fwd["q_t"], fwd["k_t"], fwd["v_t"], p, fwd["topk"], scale,
+                                     d_o_fine, fwd["topk_ref"])
+    d_qbar, d_kbar, d_vbar = coarse_attention_backward(fwd["qbar"], fwd["kbar"], fwd["vbar"],
+                                                       scale, d_o_coarse)
+    dq_t = dq_f + pool_backward(d_qbar, p)
+    dk_t = dk_f + pool_backward(d_kbar, p)
+    dv_t = dv_f + pool_backward(d_vbar, p)
+    return dict(d_out_t=d_out_t, d_o_fine=d_o_fine, d_o_coarse=d_o_coarse,
+                d_qbar=d_qbar, d_kbar=d_kbar, d_vbar=d_vbar,
+                dq_t=dq_t, dk_t=dk_t, dv_t=dv_t, dg_t=d_g_t,
+                dq=unpermute(dq_t, p), dk=unpermute(dk_t, p), dv=unpermute(dv_t, p),
+                dg=unpermute(d_g_t, p))
