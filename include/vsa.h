@@ -157,6 +157,40 @@ vsa_status vsa_coarse_topk_pooled(vsa_plan plan, int B, int H, int D, float scal
                                   float* o_coarse, int32_t* topk_idx, float* topk_score,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/* Reference-tile thinning (the Veda node's reference_sparsity, "Veda Sparse
+ * Attention" input table: the generated-video keep setting applied to the
+ * reference tokens, 0 % = full attention).  Reading taken: each generated-
+ * video query tile keeps only its top k_ref reference (prefix) key tiles by
+ * coarse score instead of all n_p of them; reference query tiles stay dense.
+ *
+ * vsa_keep_count_ref: k_ref for n_p reference tiles, the keep rule of
+ * vsa_keep_count: keep_tiles >= 0 -> min(keep_tiles, n_p), else
+ * min(n_p, ceil(clamp(keep_ratio,0,1) * n_p - 1e-9)). */
+vsa_status vsa_keep_count_ref(vsa_plan plan, double keep_ratio, int32_t keep_tiles, int32_t* k_ref);
+
+/* For every video query tile i (n_p <= i < T) and (b,h): the k_ref reference
+ * tiles j < n_p with the largest s[i,j] = scale * <qbar_i, kbar_j> (fp32, the
+ * same scores vsa_coarse_topk ranks), ties to the lower j, ascending, into
+ * topk_ref_idx (int32 [B,H,n_v,k_ref]).  Reads the pooled means qbar, kbar
+ * from `ws` (the layout of vsa_workspace_size, as left by vsa_coarse_topk or
+ * vsa_permute_pool).  n_p <= 256 (else VSA_ERR_UNSUPPORTED); k_ref in
+ * [0, n_p]. */
+vsa_status vsa_select_reference(vsa_plan plan, int B, int H, int D, float scale, int k_ref,
+                                int32_t* topk_ref_idx, const void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* Sparse attention with thinned reference tiles: a video query tile attends to
+ * its k_ref kept reference tiles (topk_ref_idx [B,H,n_v,k_ref]) and its k kept
+ * video tiles; prefix query tiles stay dense.  gate == NULL: o_fine in the
+ * padded layout (as vsa_sparse_attn); gate and o_coarse given: the fused
+ * gated combine writing natural order (as vsa_sparse_attn_combine).  k_ref =
+ * n_p with topk_ref_idx = NULL is the unthinned layer.  k + k_ref >= 1.
+ * lse_t nullable. */
+vsa_status vsa_sparse_attn_ref(vsa_plan plan, const void* q_t, const void* k_t, const void* v_t,
+                               const int32_t* topk_idx, int k, const int32_t* topk_ref_idx,
+                               int k_ref, int B, int H, int D, float scale, const void* gate,
+                               const float* o_coarse, void* out, float* lse_t, void* stream);
+
 /* Head projection, the gate's bias-free linear (SnackOnAI, "The Code,
  * Annotated", snippet three: gate = x W_gate^T viewed as [.., heads,
  * head_dim]; with act = 0 any projection of that shape):
@@ -230,6 +264,67 @@ vsa_status vsa_sparse_attn_combine(vsa_plan plan, const void* q_t, const void* k
 vsa_status vsa_gate_combine(vsa_plan plan, const void* o_fine_t, const void* gate_t,
                             const float* o_coarse, void* out, int out_natural,
                             int B, int H, int D, void* stream);
+
+/* ---------------------------------------------------------------- backward
+ * Gradients of a loss through steps 5 .. 1, for training (SnackOnAI, "The
+ * Architecture, Unpacked": the coarse stage and the gate are learned; the VSA
+ * paper it builds on trains its sparse kernel).  The top-k selection passes no
+ * gradient: the backward runs under the forward's topk_idx (and topk_ref_idx).
+ * A training step calls, in this order: vsa_permute of d_out (natural -> tiled),
+ * vsa_combine_backward, vsa_coarse_backward, vsa_sparse_attn_backward, and
+ * vsa_unpermute of dq_t, dk_t, dv_t and d_gate_t.  All launches asynchronous on
+ * `stream`; the caller owns every buffer. */
+
+/* Bytes of the workspace that vsa_coarse_backward and vsa_sparse_attn_backward
+ * need (the larger of the two: they may share one buffer, called in turn). */
+vsa_status vsa_backward_workspace_size(vsa_plan plan, int B, int H, int D, size_t* bytes);
+
+/* Backward of step 5 for out = o_fine + sigmoid(g) * o_coarse[tile]:
+ *   d_gate_t = d_out * o_coarse[tile] * s (1 - s),  s = sigmoid(g)
+ *   d_o_coarse[t] = sum over the live rows of tile t of d_out * s
+ *   delta[r] = sum_d d_out[r] o_fine[r]  (the row statistic of the fine
+ *              softmax backward)
+ * d_out_t, o_fine_t, gate_t: bf16 [B,H,N_pad,D] tiled (d_out_t with pad rows 0,
+ * as vsa_permute writes it; o_fine_t as vsa_sparse_attn writes it).  o_coarse:
+ * fp32 [B,H,T,D].  Writes delta fp32 [B,H,N_pad] and d_gate_t bf16
+ * [B,H,N_pad,D] (0 on pad rows), d_o_coarse fp32 [B,H,T,D]. */
+vsa_status vsa_combine_backward(vsa_plan plan, const void* d_out_t, const void* o_fine_t,
+                                const void* gate_t, const float* o_coarse, int B, int H, int D,
+                                float* delta, void* d_gate_t, float* d_o_coarse, void* stream);
+
+/* Backward of the coarse attention of step 2 (o_coarse = softmax(scale qbar
+ * kbar^T) vbar over all T tiles): d_qbar, d_kbar, d_vbar fp32 [B,H,T,D] from
+ * the pooled means qbar, kbar, vbar fp32 [B,H,T,D] (as vsa_permute_pool writes
+ * them) and d_o_coarse.  fp32 arithmetic.  ws: at least
+ * vsa_backward_workspace_size bytes, 16-byte aligned. */
+vsa_status vsa_coarse_backward(vsa_plan plan, const float* qbar, const float* kbar,
+                               const float* vbar, const float* d_o_coarse, int B, int H, int D,
+                               float scale, float* d_qbar, float* d_kbar, float* d_vbar, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Backward of step 4 (and of the pooling of step 2): for every query tile i
+ * and key tile j of its key set (as in vsa_sparse_attn / vsa_sparse_attn_ref),
+ * P = exp(scale Q_i K_j^T - lse_i) on live rows and columns, dP = dO_i V_j^T,
+ * dS = P (dP - delta_i), and
+ *   dq_t = scale sum_j dS K_j + d_qbar[tile] / block_len[tile]
+ *   dk_t = scale sum_i dS^T Q_i + d_kbar[tile] / block_len[tile]
+ *   dv_t = sum_i P^T dO_i + d_vbar[tile] / block_len[tile]
+ * on live rows (pad rows written 0).  q_t, k_t, v_t, d_out_t: bf16
+ * [B,H,N_pad,D]; lse_t: fp32 [B,H,N_pad] from the forward; delta from
+ * vsa_combine_backward; d_qbar, d_kbar, d_vbar: fp32 [B,H,T,D] from
+ * vsa_coarse_backward, or all three NULL (no pooling term).  topk_ref_idx and
+ * k_ref as for vsa_sparse_attn_ref (NULL with k_ref = n_p: every reference
+ * tile).  Outputs bf16 [B,H,N_pad,D].  fp32 accumulation in tensor memory; P and
+ * dS are rounded to bf16 before their products.  An index outside its range is
+ * skipped and recorded (VSA_ERR_DEVICE_INDEX).  ws: at least
+ * vsa_backward_workspace_size bytes. */
+vsa_status vsa_sparse_attn_backward(vsa_plan plan, const void* q_t, const void* k_t,
+                                    const void* v_t, const void* d_out_t, const int32_t* topk_idx,
+                                    int k, const int32_t* topk_ref_idx, int k_ref,
+                                    const float* lse_t, const float* delta, const float* d_qbar,
+                                    const float* d_kbar, const float* d_vbar, int B, int H, int D,
+                                    float scale, void* dq_t, void* dk_t, void* dv_t, void* ws,
+                                    size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read and clear the plan's device status word.
  * Returns VSA_OK, VSA_ERR_DEVICE_TIMEOUT, VSA_ERR_DEVICE_INDEX or VSA_ERR_CUDA. */

@@ -288,3 +288,59 @@ def test_layer_pipeline_matches_layer():
         want = layer(*(s[n].cuda() for n in "qkvg")).cpu()
         assert torch.equal(got, want)
     vsa.vsa_sync_status(plan)
+
+
+REF_CASES = [
+    (SMALL, 3),                                                    # 25 reference tiles -> 3
+    (SMALL, 0),                                                    # no reference tile kept
+    (_w("ref_r128", 1, 2, 128, (256, 200, 60), (8, 16, 8), (4, 8, 4), keep_tiles=3), 1),
+    (_w("ref_d64_b2", 2, 2, 64, (64, 64, 64, 30), (4, 8, 8), (4, 4, 4), sparsity=0.75), 2),
+]
+
+
+@pytest.mark.parametrize("w,k_ref", REF_CASES, ids=lambda c: getattr(c, "name", str(c)))
+def test_reference_thinning_parity(w, k_ref):
+    """Reference tiles thinned to each video query tile's top k_ref (the Veda
+    reference_sparsity reading): the reference selection against the oracle's
+    fp64 ranking (bit-exact up to legal near-ties), and o_fine, the unfused and
+    the fused outputs against the oracle under the GPU's selections."""
+    inp = make_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    q, kk, v, g = (inp[x].cuda() for x in "qkvg")
+    layer = vsa.Layer(plan, w.B, w.H, w.D, k, fused=False, k_ref=k_ref)
+    out = layer(q, kk, v, g)
+    fused = vsa.Layer(plan, w.B, w.H, w.D, k, k_ref=k_ref)
+    out_f = fused(q, kk, v, g)
+    vsa.vsa_sync_status(plan)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    gpu_idx = layer.topk_idx.cpu().numpy().astype(np.int64)
+    gpu_ref = layer.topk_ref.cpu().numpy().astype(np.int64)
+    assert torch.equal(layer.topk_ref, fused.topk_ref)
+    ref = O.layer(*(inp[x] for x in "qkvg"), p, k, kept=gpu_idx, kept_ref=gpu_ref)
+    n_near = 0
+    for idx in np.ndindex(*gpu_ref.shape[:-2]):
+        for r in range(gpu_ref.shape[-2]):
+            row = ref["scores"][idx + (p.n_prefix_tiles + r,)][:p.n_prefix_tiles]
+            n_near += check_topk_row(gpu_ref[idx + (r,)], row, 0, k_ref)
+    assert n_near <= max(1, int(np.prod(gpu_ref.shape[:-1])) // 50)
+    assert_close(f64(layer.o_fine_t), ref["o_fine"], what="o_fine")
+    assert_close(f64(out), ref["out"], what="out")
+    assert_close(f64(out_f), ref["out"], what="fused out")
+
+
+def test_reference_thinning_keep_all_is_unthinned():
+    """k_ref = n_p through the thinned path (selection list of every reference
+    tile in order) gives the unthinned layer's output bit for bit."""
+    w = SMALL
+    inp = make_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    q, kk, v, g = (inp[x].cuda() for x in "qkvg")
+    thin = vsa.Layer(plan, w.B, w.H, w.D, k, k_ref=plan.n_prefix_tiles)
+    base = vsa.Layer(plan, w.B, w.H, w.D, k)
+    assert torch.equal(thin(q, kk, v, g), base(q, kk, v, g))
+    want = torch.arange(plan.n_prefix_tiles, dtype=torch.int32, device="cuda")
+    assert torch.equal(thin.topk_ref, want.expand_as(thin.topk_ref))
+    assert vsa.vsa_keep_count_ref(plan, keep_ratio=0.1) == 3
+    vsa.vsa_sync_status(plan)

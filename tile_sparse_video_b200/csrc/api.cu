@@ -1,4 +1,5 @@
 // libvsa C ABI: argument checks, plan lifetime and dispatch to the kernels.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <new>
@@ -313,7 +314,7 @@ vsa_status vsa_sparse_attn(vsa_plan p, const void* q_t, const void* k_t, const v
   if (!(scale > 0.0f) || !std::isfinite(scale))
     return fail(VSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   return launch_sparse_attn(p, q_t, k_t, v_t, topk_idx, int64_t(B) * H, D, k, scale, o_fine_t,
-                            lse_t, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+                            lse_t, nullptr, nullptr, nullptr, -1, static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_sparse_attn_combine(vsa_plan p, const void* q_t, const void* k_t, const void* v_t,
@@ -337,7 +338,82 @@ vsa_status vsa_sparse_attn_combine(vsa_plan p, const void* q_t, const void* k_t,
   if (!(scale > 0.0f) || !std::isfinite(scale))
     return fail(VSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   return launch_sparse_attn(p, q_t, k_t, v_t, topk_idx, int64_t(B) * H, D, k, scale, out, lse_t,
-                            gate, o_coarse, static_cast<cudaStream_t>(stream));
+                            gate, o_coarse, nullptr, -1, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_keep_count_ref(vsa_plan p, double keep_ratio, int32_t keep_tiles, int32_t* k_ref) {
+  if (p == nullptr || k_ref == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan or k_ref is NULL");
+  const int n_p = p->n_prefix_tiles;
+  int64_t kk = 0;
+  if (keep_tiles >= 0) {
+    kk = std::min<int64_t>(keep_tiles, n_p);
+  } else {
+    if (!(keep_ratio == keep_ratio)) return fail(VSA_ERR_INVALID_ARG, "keep_ratio is NaN");
+    const double r = std::min(1.0, std::max(0.0, keep_ratio));
+    kk = std::min<int64_t>(n_p, int64_t(std::ceil(r * n_p - 1e-9)));
+  }
+  *k_ref = int32_t(kk);
+  return VSA_OK;
+}
+
+vsa_status vsa_select_reference(vsa_plan p, int B, int H, int D, float scale, int k_ref,
+                                int32_t* topk_ref_idx, const void* ws, size_t ws_bytes,
+                                void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  if (k_ref < 0 || k_ref > p->n_prefix_tiles)
+    return fail(VSA_ERR_INVALID_ARG, "k_ref must be in [0, n_prefix_tiles]");
+  if (p->n_prefix_tiles > 256)
+    return fail(VSA_ERR_UNSUPPORTED, "reference selection supports at most 256 prefix tiles");
+  if (empty || k_ref == 0 || p->n_tiles == p->n_prefix_tiles) return VSA_OK;
+  VSA_TRY(check_ptr(topk_ref_idx, "topk_ref_idx"));
+  if (!std::isfinite(scale)) return fail(VSA_ERR_INVALID_ARG, "scale is not finite");
+  size_t need = 0;
+  vsa_workspace_size(p, B, H, D, 0, &need);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(VSA_ERR_WORKSPACE, "workspace missing or too small (see vsa_workspace_size)");
+  if (!aligned16(ws)) return fail(VSA_ERR_INVALID_ARG, "ws is not 16-byte aligned");
+  const int64_t bh = int64_t(B) * H;
+  const float* qbar = static_cast<const float*>(ws);
+  const float* kbar = qbar + bh * p->n_tiles * D;
+  cudaError_t e = launch_select_ref(qbar, kbar, bh, p->n_tiles, p->n_prefix_tiles, D, scale, k_ref,
+                                    topk_ref_idx, p->num_sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "select_ref launch");
+}
+
+vsa_status vsa_sparse_attn_ref(vsa_plan p, const void* q_t, const void* k_t, const void* v_t,
+                               const int32_t* topk_idx, int k, const int32_t* topk_ref_idx,
+                               int k_ref, int B, int H, int D, float scale, const void* gate,
+                               const float* o_coarse, void* out, float* lse_t, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  const int n_p = p->n_prefix_tiles, n_v = p->n_tiles - p->n_prefix_tiles;
+  if (k < 0 || k > n_v) return fail(VSA_ERR_INVALID_ARG, "k must be in [0, n_video_tiles]");
+  if (k_ref < 0 || k_ref > n_p) return fail(VSA_ERR_INVALID_ARG, "k_ref must be in [0, n_prefix_tiles]");
+  if (n_v > 0 && k + k_ref == 0)
+    return fail(VSA_ERR_INVALID_ARG, "k + k_ref must be >= 1 (a video query tile needs a key)");
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(q_t, "q_t"));
+  VSA_TRY(check_ptr(k_t, "k_t"));
+  VSA_TRY(check_ptr(v_t, "v_t"));
+  VSA_TRY(check_ptr(out, "out"));
+  if (k > 0 && n_v > 0) VSA_TRY(check_ptr(topk_idx, "topk_idx"));
+  // k_ref = n_p with no list: every reference tile, the unthinned layer
+  const bool all_refs = k_ref == n_p && topk_ref_idx == nullptr;
+  if (k_ref > 0 && n_v > 0 && !all_refs) VSA_TRY(check_ptr(topk_ref_idx, "topk_ref_idx"));
+  if ((gate == nullptr) != (o_coarse == nullptr))
+    return fail(VSA_ERR_INVALID_ARG, "gate and o_coarse are given together or not at all");
+  if (gate != nullptr) {
+    VSA_TRY(check_ptr(gate, "gate"));
+    VSA_TRY(check_ptr(o_coarse, "o_coarse"));
+  }
+  if (lse_t != nullptr && !aligned16(lse_t))
+    return fail(VSA_ERR_INVALID_ARG, "lse_t is not 16-byte aligned");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  return launch_sparse_attn(p, q_t, k_t, v_t, topk_idx, int64_t(B) * H, D, k, scale, out, lse_t,
+                            gate, o_coarse, all_refs ? nullptr : topk_ref_idx, all_refs ? -1 : k_ref,
+                            static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_gate_combine(vsa_plan p, const void* o_fine_t, const void* gate_t,
@@ -357,6 +433,104 @@ vsa_status vsa_gate_combine(vsa_plan p, const void* o_fine_t, const void* gate_t
       static_cast<uint16_t*>(out), out_natural, p->d_row_src, p->d_untile, int64_t(B) * H,
       p->n_tokens, p->n_padded, p->R, p->n_tiles, D, p->num_sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "gate_combine launch");
+}
+
+vsa_status vsa_backward_workspace_size(vsa_plan p, int B, int H, int D, size_t* bytes) {
+  if (p == nullptr || bytes == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan or bytes is NULL");
+  if (B < 0 || H < 0) return fail(VSA_ERR_INVALID_ARG, "B and H must be >= 0");
+  if (D != 64 && D != 128) return fail(VSA_ERR_UNSUPPORTED, "head dim D must be 64 or 128");
+  const int64_t bh = int64_t(B) * H;
+  *bytes = std::max(colmask_bytes(p, bh), coarse_bwd_bytes(p, bh));
+  return VSA_OK;
+}
+
+vsa_status vsa_combine_backward(vsa_plan p, const void* d_out_t, const void* o_fine_t,
+                                const void* gate_t, const float* o_coarse, int B, int H, int D,
+                                float* delta, void* d_gate_t, float* d_o_coarse, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(d_out_t, "d_out_t"));
+  VSA_TRY(check_ptr(o_fine_t, "o_fine_t"));
+  VSA_TRY(check_ptr(gate_t, "gate_t"));
+  VSA_TRY(check_ptr(o_coarse, "o_coarse"));
+  VSA_TRY(check_ptr(delta, "delta"));
+  VSA_TRY(check_ptr(d_gate_t, "d_gate_t"));
+  VSA_TRY(check_ptr(d_o_coarse, "d_o_coarse"));
+  cudaError_t e = launch_combine_backward(p, d_out_t, o_fine_t, gate_t, o_coarse, int64_t(B) * H, D,
+                                          delta, d_gate_t, d_o_coarse,
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "combine backward launch");
+}
+
+vsa_status vsa_coarse_backward(vsa_plan p, const float* qbar, const float* kbar, const float* vbar,
+                               const float* d_o_coarse, int B, int H, int D, float scale,
+                               float* d_qbar, float* d_kbar, float* d_vbar, void* ws,
+                               size_t ws_bytes, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(qbar, "qbar"));
+  VSA_TRY(check_ptr(kbar, "kbar"));
+  VSA_TRY(check_ptr(vbar, "vbar"));
+  VSA_TRY(check_ptr(d_o_coarse, "d_o_coarse"));
+  VSA_TRY(check_ptr(d_qbar, "d_qbar"));
+  VSA_TRY(check_ptr(d_kbar, "d_kbar"));
+  VSA_TRY(check_ptr(d_vbar, "d_vbar"));
+  VSA_TRY(check_ptr(ws, "ws"));
+  if (ws_bytes < coarse_bwd_bytes(p, int64_t(B) * H))
+    return fail(VSA_ERR_WORKSPACE, "workspace smaller than vsa_backward_workspace_size");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  cudaError_t e = launch_coarse_backward(p, qbar, kbar, vbar, d_o_coarse, int64_t(B) * H, D, scale,
+                                         d_qbar, d_kbar, d_vbar, ws, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "coarse backward launch");
+}
+
+vsa_status vsa_sparse_attn_backward(vsa_plan p, const void* q_t, const void* k_t, const void* v_t,
+                                    const void* d_out_t, const int32_t* topk_idx, int k,
+                                    const int32_t* topk_ref_idx, int k_ref, const float* lse_t,
+                                    const float* delta, const float* d_qbar, const float* d_kbar,
+                                    const float* d_vbar, int B, int H, int D, float scale,
+                                    void* dq_t, void* dk_t, void* dv_t, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  const int n_p = p->n_prefix_tiles, n_v = p->n_tiles - p->n_prefix_tiles;
+  if (k < 0 || k > n_v) return fail(VSA_ERR_INVALID_ARG, "k must be in [0, n_video_tiles]");
+  if (k_ref < 0 || k_ref > n_p) return fail(VSA_ERR_INVALID_ARG, "k_ref must be in [0, n_prefix_tiles]");
+  if (n_v > 0 && k + k_ref == 0)
+    return fail(VSA_ERR_INVALID_ARG, "k + k_ref must be >= 1 (a video query tile needs a key)");
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(q_t, "q_t"));
+  VSA_TRY(check_ptr(k_t, "k_t"));
+  VSA_TRY(check_ptr(v_t, "v_t"));
+  VSA_TRY(check_ptr(d_out_t, "d_out_t"));
+  VSA_TRY(check_ptr(lse_t, "lse_t"));
+  VSA_TRY(check_ptr(delta, "delta"));
+  VSA_TRY(check_ptr(dq_t, "dq_t"));
+  VSA_TRY(check_ptr(dk_t, "dk_t"));
+  VSA_TRY(check_ptr(dv_t, "dv_t"));
+  VSA_TRY(check_ptr(ws, "ws"));
+  if (k > 0 && n_v > 0) VSA_TRY(check_ptr(topk_idx, "topk_idx"));
+  const bool all_refs = k_ref == n_p && topk_ref_idx == nullptr;
+  if (k_ref > 0 && n_v > 0 && !all_refs) VSA_TRY(check_ptr(topk_ref_idx, "topk_ref_idx"));
+  const int given = (d_qbar != nullptr) + (d_kbar != nullptr) + (d_vbar != nullptr);
+  if (given != 0 && given != 3)
+    return fail(VSA_ERR_INVALID_ARG, "d_qbar, d_kbar and d_vbar are given together or not at all");
+  if (given == 3) {
+    VSA_TRY(check_ptr(d_qbar, "d_qbar"));
+    VSA_TRY(check_ptr(d_kbar, "d_kbar"));
+    VSA_TRY(check_ptr(d_vbar, "d_vbar"));
+  }
+  if (ws_bytes < colmask_bytes(p, int64_t(B) * H))
+    return fail(VSA_ERR_WORKSPACE, "workspace smaller than vsa_backward_workspace_size");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  return launch_sparse_attn_backward(p, q_t, k_t, v_t, d_out_t, topk_idx, k,
+                                     all_refs ? nullptr : topk_ref_idx, all_refs ? -1 : k_ref,
+                                     lse_t, delta, d_qbar, d_kbar, d_vbar, int64_t(B) * H, D, scale,
+                                     dq_t, dk_t, dv_t, ws, static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_sync_status(vsa_plan p, void* stream) {

@@ -394,7 +394,87 @@ cudaError_t launch_coarse_d(const float* qbar, const float* kbar, const float* v
                                     topk_score, stream);
 }
 
+// Reference-tile selection (the Veda node's reference_sparsity): for every
+// video query tile i (n_p <= i < T) of every (b, h), the k_ref reference key
+// tiles j < n_p with the largest s[i,j] = scale * <qbar_i, kbar_j>, ties to
+// the lower j, written ascending to out[bh, i - n_p, :].  One warp per row:
+// lane-strided fp32 dot products (d ascending, the order the coarse kernel
+// uses, so the scores are the same bits) into a shared row of n_p scores;
+// then every candidate's rank by counting the keys that beat it (a larger
+// score, or an equal one at a lower index), and a ballot prefix count of the
+// kept ones for the ascending output.
+constexpr int kRefMaxTiles = 256;
+constexpr int kRefWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kRefWarps * 32) select_ref_kernel(
+    const float* __restrict__ qbar, const float* __restrict__ kbar, int64_t n_rows, int T, int n_p,
+    float scale, int k_ref, int32_t* __restrict__ out) {
+  __shared__ float sc[kRefWarps][kRefMaxTiles];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_v = T - n_p;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int64_t r = int64_t(blockIdx.x) * kRefWarps + warp; r < n_rows;
+       r += int64_t(gridDim.x) * kRefWarps) {
+    const int64_t bh = r / n_v;
+    const int i = n_p + int(r % n_v);
+    const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * T + i) * D);
+    for (int j = lane; j < n_p; j += 32) {
+      const float4* k4 = reinterpret_cast<const float4*>(kbar + (bh * T + j) * D);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int d4 = 0; d4 < D / 4; ++d4) {
+        const float4 a = __ldg(q4 + d4), b = __ldg(k4 + d4);
+        acc = fmaf(a.x, b.x, acc);
+        acc = fmaf(a.y, b.y, acc);
+        acc = fmaf(a.z, b.z, acc);
+        acc = fmaf(a.w, b.w, acc);
+      }
+      sc[warp][j] = scale * acc;
+    }
+    __syncwarp();
+    int32_t* o = out + r * k_ref;
+    int base = 0;
+    for (int j0 = 0; j0 < n_p; j0 += 32) {
+      const int j = j0 + lane;
+      bool keep = false;
+      if (j < n_p) {
+        const float sj = sc[warp][j];
+        int rank = 0;
+        for (int m = 0; m < n_p; ++m) {
+          const float sm = sc[warp][m];
+          rank += (sm > sj || (sm == sj && m < j)) ? 1 : 0;
+        }
+        keep = rank < k_ref;
+      }
+      const uint32_t b = __ballot_sync(0xFFFFFFFFu, keep);
+      const int pos = base + __popc(b & lt_mask);
+      if (keep && pos < k_ref) o[pos] = j;      // exactly k_ref keep for finite scores
+      base += __popc(b);
+    }
+    __syncwarp();
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_select_ref(const float* qbar, const float* kbar, int64_t bh, int T, int n_p, int D,
+                              float scale, int k_ref, int32_t* topk_ref, int num_sms,
+                              cudaStream_t stream) {
+  if (n_p > kRefMaxTiles) return cudaErrorInvalidValue;
+  const int64_t n_rows = bh * (T - n_p);
+  if (n_rows == 0 || k_ref == 0) return cudaSuccess;
+  int64_t blocks = (n_rows + kRefWarps - 1) / kRefWarps;
+  const int64_t cap = int64_t(num_sms > 0 ? num_sms : 148) * 8;
+  if (blocks > cap) blocks = cap;
+  if (D == 128)
+    select_ref_kernel<128><<<unsigned(blocks), kRefWarps * 32, 0, stream>>>(qbar, kbar, n_rows, T, n_p,
+                                                                             scale, k_ref, topk_ref);
+  else
+    select_ref_kernel<64><<<unsigned(blocks), kRefWarps * 32, 0, stream>>>(qbar, kbar, n_rows, T, n_p,
+                                                                            scale, k_ref, topk_ref);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float* vbar, int64_t bh,
                                int T, int n_p, int D, float scale, int k, float* o_coarse,

@@ -224,6 +224,11 @@ struct AttnArgs {
   int T, n_p, k, n_items;
   int64_t n_pad, n_tok;
   float scale_log2;           // scale * log2(e)
+  // reference thinning: the kept reference tiles of each video query tile
+  // [BH, n_v, k_ref], or null (every reference tile is a sink)
+  int k_ref;
+  int n_sink;                 // reference tiles of a video item: k_ref, or n_p
+  const int32_t* topk_ref;
 };
 
 // sigmoid(g) = (1 + tanh(g/2)) / 2 with the hardware tanh.
@@ -302,10 +307,51 @@ __device__ __forceinline__ int kept_tile(const AttnArgs& a, int64_t bh, int i, i
   return j;
 }
 
+// Reference key tile x (< n_sink) of video item (bh, i): tile x when every
+// reference tile is kept, else the item's x-th kept reference tile, clamped
+// into [0, n_p) (recording a fault).
+__device__ __forceinline__ int sink_tile(const AttnArgs& a, int64_t bh, int i, int x) {
+  if (a.topk_ref == nullptr) return x;
+  const int n_v = a.T - a.n_p;
+  int j = __ldg(a.topk_ref + (bh * n_v + (i - a.n_p)) * int64_t(a.k_ref) + x);
+  if (j < 0 || j >= a.n_p) {
+    record(a.status, kStatusBadIndex, unsigned(j));
+    j = 0;
+  }
+  return j;
+}
+
+// Reference tiles a video item attends to: all n_p, or the k_ref listed ones
+// when the kernel is built for reference thinning (kRef).  A template flag,
+// so that the unthinned kernel carries none of the list's arithmetic.
+template <bool kRef>
+__device__ __forceinline__ int n_sink(const AttnArgs& a) {
+  return kRef ? a.n_sink : a.n_p;
+}
+
+// Key tile of step x of item (bh, i): every tile in order for a dense
+// (prefix) item; else the reference tiles, then the kept video tiles, read
+// from the item's shared-memory list (step_tile) or from the kept-tile array
+// (step_tile_global).
+template <bool kRef>
+__device__ __forceinline__ int step_tile(const AttnArgs& a, int64_t bh, int i, bool dense, int x,
+                                         const int32_t* list) {
+  const int ns = n_sink<kRef>(a);
+  if (dense || x < ns) return (kRef && !dense) ? sink_tile(a, bh, i, x) : x;
+  return list[x - ns];
+}
+template <bool kRef>
+__device__ __forceinline__ int step_tile_global(const AttnArgs& a, int64_t bh, int i, bool dense,
+                                                int x) {
+  const int ns = n_sink<kRef>(a);
+  if (dense || x < ns) return (kRef && !dense) ? sink_tile(a, bh, i, x) : x;
+  return kept_tile(a, bh, i, x - ns);
+}
+
 // Producer loop shared by the K and the V warp: lane 0 issues one TMA tile per
 // kept key tile into an NS-stage ring; the K warp also loads Q per item and
 // (kPrefetch > 0) prefetches K/V tiles kPrefetch ahead into L2.
-template <int R, int D, int NS, bool kIsK>
+template <int R, int D, int NS, bool kIsK, bool kRef>
 __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* tm_q,
                                          const CUtensorMap* tm_t, const CUtensorMap* tm_other,
                                          uint32_t sQ, uint32_t sT, uint32_t full, uint32_t empty,
@@ -322,7 +368,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
     int i;
     decode_item(item, BH, a.n_p, n_v, bh, i);
     const bool dense = i < a.n_p;
-    const int nk = dense ? a.T : a.n_p + a.k;
+    const int nk = dense ? a.T : n_sink<kRef>(a) + a.k;
     if (!dense)
       for (int x = lane; x < a.k; x += 32) s_list[x] = kept_tile(a, bh, i, x);
     __syncwarp();
@@ -351,7 +397,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
           if (!ok) break;
         }
         VSA_TL(kIsK ? 3 : 4, kIsK ? 'K' : 'V', g);
-        const int j = (dense || n < a.n_p) ? n : s_list[n - a.n_p];
+        const int j = step_tile<kRef>(a, bh, i, dense, n, s_list);
         const int row = int(row0 + int64_t(j) * R);
         mbar_expect_tx(full + 8 * s, C::TBYTES);
 #pragma unroll
@@ -362,7 +408,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
           else
             tma_load_2d(sT + s * C::TBYTES + c * C::BN * 128, tm_t, full + 8 * s, c * 64, row);
         if (kIsK && kPrefetch > 0 && n + kPrefetch < nk) {
-          const int jp = (dense || n + kPrefetch < a.n_p) ? n + kPrefetch : s_list[n + kPrefetch - a.n_p];
+          const int jp = step_tile<kRef>(a, bh, i, dense, n + kPrefetch, s_list);
           const int rp = int(row0 + int64_t(jp) * R);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
@@ -384,7 +430,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
   }
 }
 
-template <int R, int D>
+template <int R, int D, bool kRef>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -466,10 +512,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   if (threadIdx.x == 0) VSA_TR(10, 21, tmem);
 
   if (warp == kWarpTmaK) {
-    producer<R, D, NSK, true>(a, &tm_q, &tm_k, &tm_v, sQ, sK, k_full, k_empty, q_full, q_empty,
+    producer<R, D, NSK, true, kRef>(a, &tm_q, &tm_k, &tm_v, sQ, sK, k_full, k_empty, q_full, q_empty,
                               s_klist, abort_flag, lane, BH, n_v);
   } else if (warp == kWarpTmaV) {
-    producer<R, D, NSV, false>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full, q_empty,
+    producer<R, D, NSV, false, kRef>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full, q_empty,
                                s_vlist, abort_flag, lane, BH, n_v);
   } else if (warp == kWarpMmaS) {
     // ------------------------------------------------------------ S issuer
@@ -486,7 +532,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         int64_t bh;
         int i;
         decode_item(item, BH, a.n_p, n_v, bh, i);
-        const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
+        const int nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
         if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
         for (int n = 0; n < nk; ++n) {
           const int w = n & 1;
@@ -536,7 +582,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         int64_t bh;
         int i;
         decode_item(item, BH, a.n_p, n_v, bh, i);
-        const int nk = (i < a.n_p) ? a.T : a.n_p + a.k;
+        const int nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
         for (int n = 0; n < nk; ++n) {
           const int w = n & 1;
           if (n == 0 && t > 0 && !wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) {
@@ -597,7 +643,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       int i;
       decode_item(item, BH, a.n_p, n_v, bh, i);
       const bool dense = i < a.n_p;
-      const int nk = dense ? a.T : a.n_p + a.k;
+      const int nk = dense ? a.T : n_sink<kRef>(a) + a.k;
       // Group barrier of the 256 softmax threads around the per-item list.  A
       // warp that sees the abort flag leaves instead: the others then also see
       // it before they could block here (they wait on the same mbarrier phases
@@ -605,7 +651,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       if (*abort_flag) { ok = false; break; }
       asm volatile("bar.sync 1, 256;" ::: "memory");
       for (int x = threadIdx.x; x < nk; x += 256) {
-        const int j = (dense || x < a.n_p) ? x : kept_tile(a, bh, i, x - a.n_p);
+        const int j = step_tile_global<kRef>(a, bh, i, dense, x);
         s_blen[x] = uint8_t(__ldg(a.block_len + j) - 1);
       }
       if (*abort_flag) { ok = false; break; }
@@ -863,7 +909,8 @@ size_t attn_smem_bytes(int T, int k) {
 template <int R, int D>
 vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, const void* v_t,
                      const int32_t* topk_idx, int64_t bh, int k, float scale, void* out,
-                     float* lse_t, const void* gate, const float* o_coarse, cudaStream_t stream) {
+                     float* lse_t, const void* gate, const float* o_coarse, const int32_t* topk_ref,
+                     int k_ref, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes<R, D>(p->n_tiles, k);
   if (smem > kMaxSmem)
     return fail(VSA_ERR_UNSUPPORTED, "too many tiles for the sparse attention kernel's lists");
@@ -872,8 +919,10 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   if (!make_map(&mq, q_t, rows, D, kBM) || !make_map(&mk, k_t, rows, D, R) ||
       !make_map(&mv, v_t, rows, D, R))
     return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<R, D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  const bool thin = k_ref >= 0;
+  auto kernel = thin ? sparse_attn_kernel<R, D, true> : sparse_attn_kernel<R, D, false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return fail(VSA_ERR_CUDA, cudaGetErrorString(e));
   AttnArgs a;
   a.topk = topk_idx;
@@ -888,13 +937,17 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   a.T = p->n_tiles;
   a.n_p = p->n_prefix_tiles;
   a.k = k;
+  // k_ref < 0: every reference tile is a sink; else the k_ref listed ones
+  a.topk_ref = thin ? topk_ref : nullptr;
+  a.k_ref = thin ? k_ref : 0;
+  a.n_sink = thin ? k_ref : p->n_prefix_tiles;
   a.n_pad = p->n_padded;
   a.scale_log2 = scale * 1.4426950408889634f;
   const int64_t items = bh * p->n_tiles;
   if (items >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "too many work items");
   a.n_items = int(items);
   const int grid = int(std::min<int64_t>(items, p->num_sms > 0 ? p->num_sms : 148));
-  sparse_attn_kernel<R, D><<<grid, kThreadsAttn, smem, stream>>>(mq, mk, mv, a);
+  kernel<<<grid, kThreadsAttn, smem, stream>>>(mq, mk, mv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(VSA_ERR_CUDA, std::string("sparse_attn launch: ") + cudaGetErrorString(e));
   return VSA_OK;
@@ -905,21 +958,22 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
 vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* k_t,
                               const void* v_t, const int32_t* topk_idx, int64_t bh, int D, int k,
                               float scale, void* out, float* lse_t, const void* gate,
-                              const float* o_coarse, cudaStream_t stream) {
+                              const float* o_coarse, const int32_t* topk_ref, int k_ref,
+                              cudaStream_t stream) {
   if (p->n_padded * bh >= (int64_t(1) << 31))
     return fail(VSA_ERR_UNSUPPORTED, "B*H*N_pad rows exceed the 32-bit TMA coordinate range");
   if (p->R == 128) {
     if (D == 128)
       return launch_rd<128, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate,
-                                 o_coarse, stream);
+                                 o_coarse, topk_ref, k_ref, stream);
     return launch_rd<128, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate, o_coarse,
-                              stream);
+                              topk_ref, k_ref, stream);
   }
   if (D == 128)
     return launch_rd<64, 128>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate, o_coarse,
-                              stream);
+                              topk_ref, k_ref, stream);
   return launch_rd<64, 64>(p, q_t, k_t, v_t, topk_idx, bh, k, scale, out, lse_t, gate, o_coarse,
-                           stream);
+                           topk_ref, k_ref, stream);
 }
 
 }  // namespace vsa

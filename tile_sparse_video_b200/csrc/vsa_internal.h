@@ -52,6 +52,10 @@ cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float
                                int64_t bh, int T, int n_p, int D, float scale, int k,
                                float* o_coarse, int32_t* topk_idx, float* topk_score,
                                cudaStream_t stream);
+// Top k_ref reference tiles per video query tile (n_p <= 256), ascending.
+cudaError_t launch_select_ref(const float* qbar, const float* kbar, int64_t bh, int T, int n_p, int D,
+                              float scale, int k_ref, int32_t* topk_ref, int num_sms,
+                              cudaStream_t stream);
 cudaError_t launch_gate_combine(const uint16_t* o_fine_t, const uint16_t* gate_t,
                                 const float* o_coarse, uint16_t* out, int out_natural,
                                 const int32_t* row_src, const int32_t* untile,
@@ -59,13 +63,36 @@ cudaError_t launch_gate_combine(const uint16_t* o_fine_t, const uint16_t* gate_t
                                 int D, int num_sms, cudaStream_t stream);
 // gate == nullptr: o_fine in the padded layout; otherwise the fused gated
 // combine writing natural order (gate natural [BH,N,D], o_coarse [BH,T,D]).
+// k_ref < 0: every reference tile is a key of every video query tile;
+// otherwise only its k_ref kept reference tiles, topk_ref [BH,n_v,k_ref].
 vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* k_t,
                               const void* v_t, const int32_t* topk_idx, int64_t bh, int D,
                               int k, float scale, void* out, float* lse_t, const void* gate,
-                              const float* o_coarse, cudaStream_t stream);
+                              const float* o_coarse, const int32_t* topk_ref, int k_ref,
+                              cudaStream_t stream);
 
 vsa_status launch_project(const vsa_plan_s* p, const void* x, const void* w, int B, int H, int D,
                           int C, int act, void* y, cudaStream_t stream);
+
+// Backward (backward.cu).
+size_t colmask_bytes(const vsa_plan_s* p, int64_t bh);
+size_t coarse_bwd_bytes(const vsa_plan_s* p, int64_t bh);
+cudaError_t launch_combine_backward(const vsa_plan_s* p, const void* d_out_t, const void* o_fine_t,
+                                    const void* gate_t, const float* o_coarse, int64_t bh, int D,
+                                    float* delta, void* d_gate_t, float* d_oc, cudaStream_t stream);
+cudaError_t launch_coarse_backward(const vsa_plan_s* p, const float* qbar, const float* kbar,
+                                   const float* vbar, const float* d_oc, int64_t bh, int D,
+                                   float scale, float* d_qbar, float* d_kbar, float* d_vbar,
+                                   void* ws, cudaStream_t stream);
+// k_ref < 0: every reference tile (topk_ref ignored).
+vsa_status launch_sparse_attn_backward(const vsa_plan_s* p, const void* q_t, const void* k_t,
+                                       const void* v_t, const void* d_out_t,
+                                       const int32_t* topk_idx, int k, const int32_t* topk_ref,
+                                       int k_ref, const float* lse_t, const float* delta,
+                                       const float* d_qbar, const float* d_kbar,
+                                       const float* d_vbar, int64_t bh, int D, float scale,
+                                       void* dq_t, void* dk_t, void* dv_t, void* ws,
+                                       cudaStream_t stream);
 
 // Device status codes written by kernels into vsa_plan_s::d_status.
 enum : unsigned int { kStatusOk = 0, kStatusTimeout = 1, kStatusBadIndex = 2 };

@@ -214,3 +214,20 @@ def make_projection_inputs(w: Workload, batch: Optional[Sequence[int]] = None) -
         g = torch.Generator().manual_seed(w.seed_base + 7777 + 17 * (b + 1))
         x[bi] = _bf16(torch.randn(N, C, generator=g))
     return {"x": x, "w": weight}
+
+
+def make_grad_output(w: Workload, batch: Optional[Sequence[int]] = None,
+                     heads: Optional[Sequence[int]] = None) -> torch.Tensor:
+    """Upstream gradient d_out of the layer output for the backward pass:
+    bf16 [B,H,N,D] natural order, N(0, 1), from its own generator per batch
+    element (seed ``seed_base + 17*b + 5``), drawn head by head."""
+    bsel = list(range(w.B)) if batch is None else list(batch)
+    hsel = list(range(w.H)) if heads is None else list(heads)
+    out = torch.empty(len(bsel), len(hsel), w.n_tokens, w.D, dtype=torch.bfloat16)
+    for bi, b in enumerate(bsel):
+        gen = torch.Generator().manual_seed(w.seed_base + 17 * b + 5)
+        for h in range(w.H):
+            x = torch.randn(w.n_tokens, w.D, generator=gen)
+            if h in hsel:
+                out[bi, hsel.index(h)] = _bf16(x)
+    return out

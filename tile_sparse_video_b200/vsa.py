@@ -28,7 +28,9 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_coun
            "vsa_plan_destroy", "vsa_workspace_size", "vsa_permute", "vsa_unpermute",
            "vsa_permute_pool", "vsa_coarse_topk", "vsa_coarse_topk_pooled",
            "vsa_coarse_topk_noalloc", "vsa_sparse_attn", "vsa_sparse_attn_combine",
-           "vsa_gate_combine", "vsa_project", "vsa_sync_status", "vsa_last_error")
+           "vsa_gate_combine", "vsa_project", "vsa_keep_count_ref", "vsa_select_reference",
+           "vsa_sparse_attn_ref", "vsa_backward_workspace_size", "vsa_combine_backward",
+           "vsa_coarse_backward", "vsa_sparse_attn_backward", "vsa_sync_status", "vsa_last_error")
 
 
 class VsaError(RuntimeError):
@@ -71,6 +73,14 @@ def lib():
             "vsa_sparse_attn_combine": [P, V, V, V, V, I, I, I, I, F, V, V, V, V, V],
             "vsa_gate_combine": [P, V, V, V, V, I, I, I, I, V],
             "vsa_project": [P, V, V, I, I, I, I, I, V, V],
+            "vsa_keep_count_ref": [P, D, I32, ctypes.POINTER(I32)],
+            "vsa_select_reference": [P, I, I, I, F, I, V, V, Z, V],
+            "vsa_sparse_attn_ref": [P, V, V, V, V, I, V, I, I, I, I, F, V, V, V, V, V],
+            "vsa_backward_workspace_size": [P, I, I, I, ctypes.POINTER(Z)],
+            "vsa_combine_backward": [P, V, V, V, V, I, I, I, V, V, V, V],
+            "vsa_coarse_backward": [P, V, V, V, V, I, I, I, F, V, V, V, V, Z, V],
+            "vsa_sparse_attn_backward": [P, V, V, V, V, V, I, V, I, V, V, V, V, V, I, I, I, F,
+                                         V, V, V, V, Z, V],
             "vsa_sync_status": [P, V],
         }
         for name, args in sig.items():
@@ -355,8 +365,126 @@ def vsa_project(plan: Plan, x: torch.Tensor, w: torch.Tensor, H: int, D: int, si
     return y
 
 
+def vsa_keep_count_ref(plan: Plan, keep_ratio: Optional[float] = None,
+                       keep_tiles: Optional[int] = None) -> int:
+    """Reference tiles each video query tile keeps (reference_sparsity)."""
+    out = ctypes.c_int32()
+    _check(lib().vsa_keep_count_ref(plan.handle, 0.0 if keep_ratio is None else float(keep_ratio),
+                                    -1 if keep_tiles is None else int(keep_tiles), ctypes.byref(out)))
+    return out.value
+
+
+def vsa_select_reference(plan: Plan, B: int, H: int, D: int, k_ref: int, ws,
+                         scale: Optional[float] = None, out=None, stream=None):
+    """Top k_ref reference tiles of every video query tile from the pooled
+    means in ``ws``; returns int32 [B,H,n_v,k_ref]."""
+    scale = D ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty(B, H, plan.n_video_tiles, max(k_ref, 0), dtype=torch.int32, device=ws.device)
+    _check(lib().vsa_select_reference(plan.handle, B, H, D, scale, k_ref,
+                                      _ptr(out) if out.numel() else None, _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def vsa_sparse_attn_ref(plan: Plan, q_t, k_t, v_t, topk_idx, k: int, topk_ref, k_ref: int,
+                        scale: Optional[float] = None, gate=None, o_coarse=None, out=None,
+                        want_lse: bool = False, stream=None):
+    """Sparse attention with the video query tiles' reference tiles thinned to
+    ``topk_ref``.  gate/o_coarse given: fused combine, natural-order output;
+    else o_fine in the padded layout.  Returns (out, lse or None)."""
+    B, H, _, D = q_t.shape
+    scale = D ** -0.5 if scale is None else float(scale)
+    dev = q_t.device
+    fused = gate is not None
+    if out is None:
+        rows = plan.n_tokens if fused else plan.n_padded
+        out = torch.empty(B, H, rows, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, plan.n_padded, dtype=torch.float32, device=dev) if want_lse else None
+    _check(lib().vsa_sparse_attn_ref(plan.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t),
+                                     _ptr(topk_idx) if topk_idx is not None and topk_idx.numel() else None, k,
+                                     _ptr(topk_ref) if topk_ref is not None and topk_ref.numel() else None, k_ref,
+                                     B, H, D, scale, _ptr(gate) if fused else None,
+                                     _ptr(o_coarse) if fused else None, _ptr(out), _ptr(lse),
+                                     _stream(stream)))
+    return out, lse
+
+
 def vsa_sync_status(plan: Plan, stream=None):
     _check(lib().vsa_sync_status(plan.handle, _stream(stream)))
+
+
+# ---------------------------------------------------------------- backward
+
+def vsa_backward_workspace_size(plan: Plan, B: int, H: int, D: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().vsa_backward_workspace_size(plan.handle, B, H, D, ctypes.byref(n)))
+    return int(n.value)
+
+
+def vsa_combine_backward(plan: Plan, d_out_t, o_fine_t, gate_t, o_coarse, delta=None, d_gate_t=None,
+                         d_o_coarse=None, stream=None):
+    """Backward of the gated combine.  Returns (delta fp32 [B,H,N_pad],
+    d_gate_t bf16 [B,H,N_pad,D], d_o_coarse fp32 [B,H,T,D])."""
+    B, H, _, D = d_out_t.shape
+    tiled = (B, H, plan.n_padded, D)
+    for name, t in (("d_out_t", d_out_t), ("o_fine_t", o_fine_t), ("gate_t", gate_t)):
+        _need(t, name, torch.bfloat16, tiled)
+    _need(o_coarse, "o_coarse", torch.float32, (B, H, plan.n_tiles, D))
+    dev = d_out_t.device
+    if delta is None:
+        delta = torch.empty(B, H, plan.n_padded, dtype=torch.float32, device=dev)
+    if d_gate_t is None:
+        d_gate_t = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+    if d_o_coarse is None:
+        d_o_coarse = torch.empty(B, H, plan.n_tiles, D, dtype=torch.float32, device=dev)
+    _check(lib().vsa_combine_backward(plan.handle, _ptr(d_out_t), _ptr(o_fine_t), _ptr(gate_t),
+                                      _ptr(o_coarse), B, H, D, _ptr(delta), _ptr(d_gate_t),
+                                      _ptr(d_o_coarse), _stream(stream)))
+    return delta, d_gate_t, d_o_coarse
+
+
+def vsa_coarse_backward(plan: Plan, qbar, kbar, vbar, d_o_coarse, ws, scale: Optional[float] = None,
+                        out=None, stream=None):
+    """Backward of the coarse attention: (d_qbar, d_kbar, d_vbar), fp32 [B,H,T,D]."""
+    B, H, T, D = qbar.shape
+    for name, t in (("qbar", qbar), ("kbar", kbar), ("vbar", vbar), ("d_o_coarse", d_o_coarse)):
+        _need(t, name, torch.float32, (B, H, plan.n_tiles, D))
+    scale = D ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = tuple(torch.empty_like(qbar) for _ in range(3))
+    _check(lib().vsa_coarse_backward(plan.handle, _ptr(qbar), _ptr(kbar), _ptr(vbar),
+                                     _ptr(d_o_coarse), B, H, D, scale, _ptr(out[0]), _ptr(out[1]),
+                                     _ptr(out[2]), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream)))
+    return out
+
+
+def vsa_sparse_attn_backward(plan: Plan, q_t, k_t, v_t, d_out_t, topk_idx, k: int, lse, delta, ws,
+                             topk_ref=None, k_ref: Optional[int] = None, d_bar=None,
+                             scale: Optional[float] = None, out=None, stream=None):
+    """Backward of the block-sparse attention (plus the pooling term when
+    ``d_bar`` = (d_qbar, d_kbar, d_vbar) is given).  k_ref None: every
+    reference tile is a key of every video query tile.  Returns (dq_t, dk_t,
+    dv_t), bf16 [B,H,N_pad,D]."""
+    B, H, _, D = q_t.shape
+    tiled = (B, H, plan.n_padded, D)
+    for name, t in (("q_t", q_t), ("k_t", k_t), ("v_t", v_t), ("d_out_t", d_out_t)):
+        _need(t, name, torch.bfloat16, tiled)
+    _need(lse, "lse", torch.float32, (B, H, plan.n_padded))
+    _need(delta, "delta", torch.float32, (B, H, plan.n_padded))
+    scale = D ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = tuple(torch.empty(tiled, dtype=torch.bfloat16, device=q_t.device) for _ in range(3))
+    kr = plan.n_prefix_tiles if k_ref is None else int(k_ref)
+    ref = None if k_ref is None or topk_ref is None or topk_ref.numel() == 0 else _ptr(topk_ref)
+    db = (None, None, None) if d_bar is None else tuple(_ptr(t) for t in d_bar)
+    _check(lib().vsa_sparse_attn_backward(
+        plan.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(d_out_t),
+        _ptr(topk_idx) if topk_idx is not None and topk_idx.numel() else None, k, ref, kr,
+        _ptr(lse), _ptr(delta), db[0], db[1], db[2], B, H, D, scale, _ptr(out[0]), _ptr(out[1]),
+        _ptr(out[2]), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return out
 
 
 class Layer:
@@ -369,8 +497,10 @@ class Layer:
     are allocated once and reused by every call."""
 
     def __init__(self, plan: Plan, B: int, H: int, D: int, k: int, scale: Optional[float] = None,
-                 device=None, fused: bool = True):
+                 device=None, fused: bool = True, k_ref: Optional[int] = None):
         self.plan, self.B, self.H, self.D, self.k, self.fused = plan, B, H, D, k, fused
+        # k_ref: reference tiles each video query tile keeps (None: all of them)
+        self.k_ref = k_ref
         self.scale = D ** -0.5 if scale is None else float(scale)
         dev = torch.device("cuda", plan.device) if device is None else torch.device(device)
         tiled = (B, H, plan.n_padded, D)
@@ -382,6 +512,8 @@ class Layer:
         self.topk_idx = torch.empty(B, H, plan.n_video_tiles, max(k, 0), dtype=torch.int32, device=dev)
         self.ws = torch.empty(max(plan.workspace_size(B, H, D, k), 16), dtype=torch.uint8, device=dev)
         self.out = torch.empty(B, H, plan.n_tokens, D, dtype=torch.bfloat16, device=dev)
+        self.topk_ref = (torch.empty(B, H, plan.n_video_tiles, max(k_ref, 0), dtype=torch.int32, device=dev)
+                         if k_ref is not None else None)
 
     def __call__(self, q, k, v, g, stream=None):
         p = self.plan
@@ -392,6 +524,13 @@ class Layer:
             vsa_permute_pool(p, v, self.v_t, vbar, stream)
             vsa_coarse_topk_pooled(p, self.B, self.H, self.D, self.k, self.ws, self.scale,
                                    o_coarse=self.o_coarse, topk_idx=self.topk_idx, stream=stream)
+            if self.k_ref is not None:
+                vsa_select_reference(p, self.B, self.H, self.D, self.k_ref, self.ws, self.scale,
+                                     out=self.topk_ref, stream=stream)
+                vsa_sparse_attn_ref(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k,
+                                    self.topk_ref, self.k_ref, self.scale, gate=g,
+                                    o_coarse=self.o_coarse, out=self.out, stream=stream)
+                return self.out
             vsa_sparse_attn_combine(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, g,
                                     self.o_coarse, self.scale, out=self.out, stream=stream)
             return self.out
@@ -401,8 +540,14 @@ class Layer:
         vsa_coarse_topk(p, self.q_t, self.k_t, self.v_t, self.k, self.scale, ws=self.ws,
                         o_coarse=self.o_coarse, topk_idx=self.topk_idx, stream=stream)
         vsa_permute(p, g, self.g_t, stream)
-        vsa_sparse_attn(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, self.scale,
-                        out=self.o_fine_t, stream=stream)
+        if self.k_ref is not None:
+            vsa_select_reference(p, self.B, self.H, self.D, self.k_ref, self.ws, self.scale,
+                                 out=self.topk_ref, stream=stream)
+            vsa_sparse_attn_ref(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k,
+                                self.topk_ref, self.k_ref, self.scale, out=self.o_fine_t, stream=stream)
+        else:
+            vsa_sparse_attn(p, self.q_t, self.k_t, self.v_t, self.topk_idx, self.k, self.scale,
+                            out=self.o_fine_t, stream=stream)
         vsa_gate_combine(p, self.o_fine_t, self.g_t, self.o_coarse, natural=True, out=self.out,
                          stream=stream)
         return self.out
@@ -470,3 +615,77 @@ class LayerPipeline:
             end_event.record(self.s_out)
         here.wait_event(ev_out[n - 1])
         return ev_out[n - 1]
+
+
+class TrainingLayer:
+    """Forward and backward of the layer for training.  ``forward`` runs the
+    unfused chain and keeps what the backward needs (tiled Q, K, V, G, the
+    pooled means, o_coarse, the selection, o_fine and its log-sum-exp);
+    ``backward(d_out)`` returns (dq, dk, dv, dg) in natural order [B,H,N,D],
+    bf16: permute d_out, combine backward, coarse backward, attention backward
+    (with the pooling term), and four unpermutes.  The selection passes no
+    gradient.  Buffers are allocated once and reused."""
+
+    def __init__(self, plan: Plan, B: int, H: int, D: int, k: int, scale: Optional[float] = None,
+                 device=None, k_ref: Optional[int] = None):
+        self.plan, self.B, self.H, self.D, self.k, self.k_ref = plan, B, H, D, k, k_ref
+        self.scale = D ** -0.5 if scale is None else float(scale)
+        dev = torch.device("cuda", plan.device) if device is None else torch.device(device)
+        tiled = (B, H, plan.n_padded, D)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.q_t, self.k_t, self.v_t, self.g_t, self.o_fine_t, self.d_out_t = (
+            torch.empty(tiled, **bf) for _ in range(6))
+        self.o_coarse = torch.empty(B, H, plan.n_tiles, D, **f32)
+        self.lse = torch.empty(B, H, plan.n_padded, **f32)
+        self.topk_idx = torch.empty(B, H, plan.n_video_tiles, max(k, 0), dtype=torch.int32, device=dev)
+        self.topk_ref = (torch.empty(B, H, plan.n_video_tiles, max(k_ref, 0), dtype=torch.int32, device=dev)
+                         if k_ref is not None else None)
+        self.ws = torch.empty(max(plan.workspace_size(B, H, D, k), 16), dtype=torch.uint8, device=dev)
+        self.bws = torch.empty(max(vsa_backward_workspace_size(plan, B, H, D), 16), dtype=torch.uint8,
+                               device=dev)
+        self.out = torch.empty(B, H, plan.n_tokens, D, **bf)
+        self.delta = torch.empty(B, H, plan.n_padded, **f32)
+        self.d_o_coarse = torch.empty(B, H, plan.n_tiles, D, **f32)
+        self.d_bar = tuple(torch.empty(B, H, plan.n_tiles, D, **f32) for _ in range(3))
+        self.dq_t, self.dk_t, self.dv_t, self.dg_t = (torch.empty(tiled, **bf) for _ in range(4))
+        self.grads = tuple(torch.empty(B, H, plan.n_tokens, D, **bf) for _ in range(4))
+
+    def forward(self, q, k, v, g, stream=None):
+        p = self.plan
+        qbar, kbar, vbar = pooled_slots(p, self.ws, self.B, self.H, self.D)
+        vsa_permute_pool(p, q, self.q_t, qbar, stream)
+        vsa_permute_pool(p, k, self.k_t, kbar, stream)
+        vsa_permute_pool(p, v, self.v_t, vbar, stream)
+        vsa_coarse_topk_pooled(p, self.B, self.H, self.D, self.k, self.ws, self.scale,
+                               o_coarse=self.o_coarse, topk_idx=self.topk_idx, stream=stream)
+        vsa_permute(p, g, self.g_t, stream)
+        kr = p.n_prefix_tiles if self.k_ref is None else self.k_ref
+        if self.k_ref is not None:
+            vsa_select_reference(p, self.B, self.H, self.D, self.k_ref, self.ws, self.scale,
+                                 out=self.topk_ref, stream=stream)
+        _check(lib().vsa_sparse_attn_ref(
+            p.handle, _ptr(self.q_t), _ptr(self.k_t), _ptr(self.v_t),
+            _ptr(self.topk_idx) if self.topk_idx.numel() else None, self.k,
+            _ptr(self.topk_ref) if self.topk_ref is not None and self.topk_ref.numel() else None, kr,
+            self.B, self.H, self.D, self.scale, None, None, _ptr(self.o_fine_t), _ptr(self.lse),
+            _stream(stream)))
+        vsa_gate_combine(p, self.o_fine_t, self.g_t, self.o_coarse, natural=True, out=self.out,
+                         stream=stream)
+        return self.out
+
+    def backward(self, d_out, stream=None):
+        p = self.plan
+        vsa_permute(p, d_out, self.d_out_t, stream)
+        vsa_combine_backward(p, self.d_out_t, self.o_fine_t, self.g_t, self.o_coarse, self.delta,
+                             self.dg_t, self.d_o_coarse, stream)
+        qbar, kbar, vbar = pooled_slots(p, self.ws, self.B, self.H, self.D)
+        vsa_coarse_backward(p, qbar, kbar, vbar, self.d_o_coarse, self.bws, self.scale,
+                            out=self.d_bar, stream=stream)
+        vsa_sparse_attn_backward(p, self.q_t, self.k_t, self.v_t, self.d_out_t, self.topk_idx,
+                                 self.k, self.lse, self.delta, self.bws, topk_ref=self.topk_ref,
+                                 k_ref=self.k_ref, d_bar=self.d_bar, scale=self.scale,
+                                 out=(self.dq_t, self.dk_t, self.dv_t), stream=stream)
+        for src, dst in zip((self.dq_t, self.dk_t, self.dv_t, self.dg_t), self.grads):
+            vsa_unpermute(p, src, dst, stream)
+        return self.grads
