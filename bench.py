@@ -263,6 +263,74 @@ def projection_timing(w: Workload, plan, dev, stream, steps: int) -> dict:
             "cublas_ms": round(ref_ms, 4), "gpu_launches_per_call": 1}
 
 
+def backward_timing(w: Workload, plan, dev, stream, inp_dev, k: int, kept_flop: float,
+                    steps: int) -> dict:
+    """The layer's backward pass (vsa.TrainingLayer.backward: permute of
+    d_out, combine backward, coarse backward, attention backward with the
+    pooling term, four unpermutes) at this workload's shape, after one
+    forward, inputs resident, CUDA events around each phase.  The attention
+    backward's algorithmic work is five products per kept tile pair (S, dP,
+    dQ, dK, dV: 2.5x the forward's two)."""
+    from tile_sparse_video_b200 import vsa
+    layer = vsa.TrainingLayer(plan, w.B, w.H, w.D, k)
+    layer.forward(*inp_dev)
+    g = torch.Generator(device=dev).manual_seed(w.seed_base + 5555)
+    d_out = torch.randn(layer.out.shape, device=dev, generator=g).to(torch.bfloat16)
+    p = plan
+    qbar, kbar, vbar = vsa.pooled_slots(p, layer.ws, w.B, w.H, w.D)
+
+    def bstep(ev=None):
+        mark = (lambda j: ev[j].record(stream)) if ev is not None else (lambda j: None)
+        mark(0)
+        vsa.vsa_permute(p, d_out, layer.d_out_t)
+        mark(1)
+        vsa.vsa_combine_backward(p, layer.d_out_t, layer.o_fine_t, layer.g_t, layer.o_coarse,
+                                 layer.delta, layer.dg_t, layer.d_o_coarse)
+        mark(2)
+        vsa.vsa_coarse_backward(p, qbar, kbar, vbar, layer.d_o_coarse, layer.bws, layer.scale,
+                                out=layer.d_bar)
+        mark(3)
+        vsa.vsa_sparse_attn_backward(p, layer.q_t, layer.k_t, layer.v_t, layer.d_out_t,
+                                     layer.topk_idx, k, layer.lse, layer.delta, layer.bws,
+                                     d_bar=layer.d_bar, scale=layer.scale,
+                                     out=(layer.dq_t, layer.dk_t, layer.dv_t))
+        mark(4)
+        for src, dst in zip((layer.dq_t, layer.dk_t, layer.dv_t, layer.dg_t), layer.grads):
+            vsa.vsa_unpermute(p, src, dst)
+        mark(5)
+
+    for _ in range(3):
+        bstep()
+    vsa.vsa_sync_status(plan)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        bstep(events[i])
+    torch.cuda.synchronize()
+    vsa.vsa_sync_status(plan)
+    parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(5)] for e in events]).mean(axis=0)
+    names = ("permute_d_out", "combine_backward", "coarse_backward", "sparse_attn_backward",
+             "unpermute_dq_dk_dv_dg")
+    peaks = load_peaks()
+    flop = 2.5 * kept_flop
+    attn_ms = float(parts[3])
+    achieved = flop / (attn_ms * 1e-3) / 1e12
+    tiled_bytes = w.B * w.H * plan.n_padded * w.D * 2
+    res = {"ms_per_layer": round(float(parts.sum()), 4),
+           "kernels_ms": {n: round(float(x), 4) for n, x in zip(names, parts)},
+           "combine_backward_hbm_gbs": round(4 * tiled_bytes / (parts[1] * 1e-3) / 1e9, 1),
+           "roofline": {"kernel": "sparse_attn_backward (dQ and dK/dV kernels)", "bound": "tensor",
+                        "achieved": round(achieved, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                        "frac": round(achieved / peaks["bf16"], 4),
+                        "algorithmic_tflop": round(flop / 1e12, 3)},
+           "gpu_launches_per_layer": 16,
+           "memsets_per_layer": 1,
+           "steps": steps}
+    del layer
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     from tile_sparse_video_b200 import vsa
     import torch.distributed as dist
@@ -385,6 +453,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     }
     if not args.no_projection:
         res["projection"] = projection_timing(w, plan, dev, stream, max(3, min(args.steps, 10)))
+    if not args.no_backward:
+        del layer
+        torch.cuda.empty_cache()
+        res["backward"] = backward_timing(w, plan, dev, stream, (q, kk, v, g), k, acct["kept_flop"],
+                                          max(3, min(args.steps, 5)))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = oracle_sample(w, inp)
     if rank == 0:
@@ -426,6 +499,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
     ap.add_argument("--no-projection", action="store_true", help="skip the gate projection timing")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
     ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
                     help="profiling runs only: another named workload")
     ap.add_argument("--heads", type=int, default=0, help="profiling runs only: fewer heads")

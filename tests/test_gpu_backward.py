@@ -161,3 +161,62 @@ def test_backward_rejects_bad_arguments():
                                      d_bar=(layer.d_bar[0], None, None))
     assert e.value.status == 1
     vsa.vsa_sync_status(plan)
+
+
+def test_backward_full_size_sampled():
+    """The 104,704-token, 42-head Veda layer in the benchmark's launch
+    configuration (vsa.TrainingLayer): for two heads, the oracle computes the
+    coarse backward of the whole head and, one tile at a time, dq of sampled
+    query tiles (prefix and video), dk and dv of a sampled video key tile
+    (summing over every query tile that attends to it) and d_gate of the
+    sampled query tiles' rows."""
+    from tile_sparse_video_b200.inputs import VEDA_104K
+    w = VEDA_104K
+    inp = make_inputs(w)
+    d_out = make_grad_output(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    layer = vsa.TrainingLayer(plan, w.B, w.H, w.D, k)
+    layer.forward(*(inp[x].cuda() for x in "qkvg"))
+    layer.backward(d_out.cuda())
+    vsa.vsa_sync_status(plan)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    R, n_p, T = p.R, p.n_prefix_tiles, p.n_tiles
+    scale = w.D ** -0.5
+    sel_all = layer.topk_idx.cpu().numpy().astype(np.int64)
+    rng = np.random.default_rng(5)
+    for h in (0, w.H - 1):
+        q_t, k_t, v_t, g_t = (O.permute(inp[x][0, h].to(torch.float64).numpy(), p) for x in "qkvg")
+        d_t = O.permute(d_out[0, h].to(torch.float64).numpy(), p)
+        qbar, kbar, vbar = O.pool(q_t, p), O.pool(k_t, p), O.pool(v_t, p)
+        _, o_coarse = O.coarse_attention(qbar, kbar, vbar, scale)
+        _, dg_t, d_oc = O.gate_combine_backward(d_t, np.zeros_like(d_t), g_t, o_coarse, p)
+        d_qbar, d_kbar, d_vbar = O.coarse_attention_backward(qbar, kbar, vbar, scale, d_oc)
+        sel = sel_all[0, h]
+        keys = lambda i: O.key_tiles(p, i, sel[i - n_p] if i >= n_p else None)
+        gq, gk, gv, gg = (f64(t[0, h]) for t in (layer.dq_t, layer.dk_t, layer.dv_t, layer.dg_t))
+        # dq of sampled query tiles
+        for i in [0, n_p, T - 1] + list(rng.choice(np.arange(n_p, T), 2, replace=False)):
+            n = p.block_len[i]
+            rows = slice(i * R, i * R + n)
+            _, dq, _, _ = O.fine_tile_backward(q_t, k_t, v_t, p, i, keys(i), scale, d_t[rows])
+            assert_rel(gq[rows], dq + d_qbar[i] / n, what=f"dq h{h} tile {i}")
+            assert_rel(gg[rows], dg_t[rows], 2 ** -8, 2 ** -8, f"d_gate h{h} tile {i}")
+        # dk, dv of a sampled video key tile (a prefix key tile is attended by all
+        # 818 query tiles, too many for the oracle here; the small layouts cover it)
+        for j in [int(rng.integers(n_p, T))]:
+            n = p.block_len[j]
+            dk = np.zeros((n, w.D))
+            dv = np.zeros((n, w.D))
+            for i in range(T):
+                ks = keys(i)
+                if j not in ks:
+                    continue
+                rows_i = slice(i * R, i * R + p.block_len[i])
+                key_rows, _, dki, dvi = O.fine_tile_backward(q_t, k_t, v_t, p, i, ks, scale, d_t[rows_i])
+                at = np.searchsorted(key_rows, j * R)
+                dk += dki[at: at + n]
+                dv += dvi[at: at + n]
+            rows = slice(j * R, j * R + n)
+            assert_rel(gk[rows], dk + d_kbar[j] / n, what=f"dk h{h} tile {j}")
+            assert_rel(gv[rows], dv + d_vbar[j] / n, what=f"dv h{h} tile {j}")

@@ -341,61 +341,66 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
 template <int R, int D, bool kKeyMajor>
 struct BwdCfg {
   static constexpr int N = R;                       // rows of a column-side tile
+  static constexpr int NH = 64;                     // score columns of a half-step
+  static constexpr int HS = N / NH;                 // half-steps per step
+  static constexpr int NS = HS == 1 ? 3 : 2;        // column-side ring stages
   static constexpr int XBYTES = kBwdM * D * 2;      // one row-side tile (128-row box)
   static constexpr int YBYTES = N * D * 2;          // one column-side tile
   static constexpr int CBYTES = 2 * N * 4;          // key-major: lse and delta of the column tile
   static constexpr int OFF_X1 = 0;
   static constexpr int OFF_X2 = XBYTES;
   static constexpr int OFF_Y = 2 * XBYTES;          // stage s: Y1 at + s*2*YBYTES, Y2 at + YBYTES
-  static constexpr int OFF_C = OFF_Y + 4 * YBYTES;  // stage s: + s*CBYTES
-  static constexpr int OFF_BAR = OFF_C + 2 * CBYTES;
-  // barriers: x_full, y_full[2], s_full, p_ready, mm2_done, acc_full, list_full,
-  //           epi_done, drain
-  static constexpr int NBAR = 10;
+  static constexpr int OFF_C = OFF_Y + NS * 2 * YBYTES;   // stage s: + s*CBYTES
+  static constexpr int OFF_BAR = OFF_C + NS * CBYTES;
+  // barriers: x_full, y_full[NS], s_full[2], p_ready[2], acc_done[2], acc_full,
+  //           list_full, epi_done, drain
+  static constexpr int NBAR = 1 + NS + 6 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;   // tmem slot, abort flag, list count
   static constexpr int OFF_LIST = OFF_MISC + 16;
-  // TMEM columns: accumulators first (dQ; or dK then dV), then S and dP
+  // TMEM columns: accumulators (dQ; or dK then dV), then two half-step
+  // buffers, each S [NH columns] then dP [NH columns]
   static constexpr uint32_t COL_ACC0 = 0;
   static constexpr uint32_t COL_ACC1 = D;
-  static constexpr uint32_t COL_S = kKeyMajor ? 2 * D : D;
-  static constexpr uint32_t COL_DP = COL_S + N;
-  static constexpr uint32_t TMEM_COLS = (COL_DP + N) <= 256 ? 256u : 512u;
-  static_assert(COL_DP + N <= 512, "TMEM columns");
-  static constexpr uint32_t IDESC_SS = idesc_bf16(kBwdM, N, false, false);
+  static constexpr uint32_t COL_BUF = kKeyMajor ? 2 * D : D;
+  static constexpr uint32_t TMEM_COLS = (COL_BUF + 4 * NH) <= 256 ? 256u : 512u;
+  static_assert(COL_BUF + 4 * NH <= 512, "TMEM columns");
+  static_assert(N % NH == 0, "tile rows");
+  static constexpr uint32_t IDESC_SS = idesc_bf16(kBwdM, NH, false, false);
   static constexpr uint32_t IDESC_ACC = idesc_bf16(kBwdM, D, false, true);
-  static size_t bytes(int T) { return size_t(OFF_LIST) + size_t(4) * ((T + 3) & ~3); }
+  // the list: column tile of each step int32[T], then its block_len int32[T]
+  static size_t bytes(int T) { return size_t(OFF_LIST) + size_t(8) * ((T + 3) & ~3); }
 };
 
-// TMEM column of the bf16 pair holding K index kappa of a P / dS operand:
-// warp half h writes the packed values of score columns [h N/2, (h+1) N/2)
-// into the first N/4 columns of that same range (only columns it has read).
-template <int N>
-__device__ __forceinline__ constexpr uint32_t packed_col(int kappa) {
-  return uint32_t((kappa / (N / 2)) * (N / 2) + (kappa % (N / 2)) / 2);
-}
-
-// Work item -> (b*h, row tile): every head's prefix tiles first (the longest
-// items in both modes), then the video tiles head by head.
+// Work item -> (b*h, row tile): the video tiles head by head first, so that
+// the CTAs share one head's column-side tiles in L2, then every head's prefix
+// tiles (the longest items in both modes: each streams a whole head).  Run
+// first, the prefix items spread the concurrent reads over all heads and the
+// column-side tiles no longer stayed in L2 (measured: 17x the algorithmic
+// DRAM reads).
 __device__ __forceinline__ void decode_bwd_item(int item, int BH, int n_p, int T, int64_t& bh,
                                                 int& t) {
-  const int first = BH * n_p;
+  const int n_v = T - n_p;
+  const int first = BH * n_v;
   if (item < first) {
-    bh = item / n_p;
-    t = item % n_p;
+    bh = item / n_v;
+    t = n_p + item % n_v;
   } else {
-    const int n_v = T - n_p;
-    bh = (item - first) / n_v;
-    t = n_p + (item - first) % n_v;
+    bh = (item - first) / n_p;
+    t = (item - first) % n_p;
   }
 }
 
+// Half-step u of an item covers score columns [c*NH, (c+1)*NH) (c = u % HS)
+// of step n = u / HS.  Half-steps alternate between the two elementwise
+// warpgroups and their two TMEM buffers (w = global half-step & 1), so that
+// one warpgroup's exponentials overlap the tensor core's work on the other's.
 template <int R, int D, bool kKeyMajor>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ CUtensorMap tm_x2,
                     const __grid_constant__ CUtensorMap tm_y1, const __grid_constant__ CUtensorMap tm_y2,
                     const BwdArgs a) {
   using C = BwdCfg<R, D, kKeyMajor>;
-  constexpr int N = C::N;
+  constexpr int N = C::N, NH = C::NH, HS = C::HS, NS = C::NS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -403,18 +408,20 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   const uint32_t sX1 = s_base + C::OFF_X1, sX2 = s_base + C::OFF_X2, sY = s_base + C::OFF_Y;
   const uint32_t bar0 = s_base + C::OFF_BAR;
   // x_full: row-side tiles of an item.  y_full[s]: column-side tiles (and, key-
-  // major, their lse / delta) of the steps using stage s.  s_full, p_ready and
-  // mm2_done complete once per step; acc_full once per item with steps;
-  // list_full and epi_done once per item.  The issuer waits for mm2_done of a
-  // step before it issues the next step's products or reloads its stage, so no
-  // waiter can fall two phases behind on any of them.
-  const uint32_t x_full = bar0, y_full = bar0 + 8, s_full = bar0 + 24, p_ready = bar0 + 32,
-                 mm2_done = bar0 + 40, acc_full = bar0 + 48, list_full = bar0 + 56,
-                 epi_done = bar0 + 64, drain = bar0 + 72;
+  // major, their lse / delta) of the steps using stage s.  s_full[w],
+  // p_ready[w] and acc_done[w] complete once per half-step of buffer w;
+  // acc_full once per item with steps; list_full and epi_done once per item.
+  // The issuer reuses buffer w (and reloads a stage) only after acc_done of
+  // its previous half-step, which follows that half-step's p_ready, so no
+  // waiter can fall two phases behind.
+  const uint32_t x_full = bar0, y_full = bar0 + 8, s_full = y_full + 8 * NS, p_ready = s_full + 16,
+                 acc_done = p_ready + 16, acc_full = acc_done + 16, list_full = acc_full + 8,
+                 epi_done = list_full + 8, drain = epi_done + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* s_cnt = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   int32_t* s_list = reinterpret_cast<int32_t*>(smem + C::OFF_LIST);
+  int32_t* s_blen = s_list + ((a.T + 3) & ~3);
   const float* s_c = reinterpret_cast<const float*>(smem + C::OFF_C);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -422,11 +429,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(x_full, 1);
-    mbar_init(y_full, 1);
-    mbar_init(y_full + 8, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_ready, 8);
-    mbar_init(mm2_done, 1);
+    for (int s = 0; s < NS; ++s) mbar_init(y_full + 8 * s, 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(s_full + 8 * w, 1);
+      mbar_init(p_ready + 8 * w, 4);
+      mbar_init(acc_done + 8 * w, 1);
+    }
     mbar_init(acc_full, 1);
     mbar_init(list_full, 1);
     mbar_init(epi_done, 8);
@@ -455,9 +463,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
   if (warp == kWarpIssue) {
     // ------------------------------------------------------------ lists, TMA, MMA
-    uint32_t g = 0;                   // steps of earlier items (stage = step & 1)
-    uint32_t x_loads = 0;             // row-side loads issued
-    uint32_t y_issued[2] = {0, 0}, y_seen[2] = {0, 0};
+    uint32_t G = 0, Gs = 0;           // half-steps / steps of earlier items
+    uint32_t hw[2] = {0, 0};          // half-steps of each buffer so far
+    uint32_t x_loads = 0;
+    uint32_t y_issued[NS] = {}, y_seen[NS] = {};
     bool x_pending = false;
     int t = 0;
     bool ok = true;
@@ -472,8 +481,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         // query tiles whose key set holds key tile rt, ascending
         const uint32_t* row = a.colmask + (bh * a.T + rt) * int64_t(a.W);
         for (int base = 0; base < a.W; base += 32) {
-          const int w = base + lane;
-          uint32_t word = w < a.W ? __ldg(row + w) : 0u;
+          const int wd = base + lane;
+          uint32_t word = wd < a.W ? __ldg(row + wd) : 0u;
           const int c = __popc(word);
           int incl = c;
 #pragma unroll
@@ -483,7 +492,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           }
           int pos = cnt + incl - c;
           while (word != 0u) {
-            s_list[pos++] = 32 * w + (__ffs(word) - 1);
+            s_list[pos++] = 32 * wd + (__ffs(word) - 1);
             word &= word - 1u;
           }
           cnt += __shfl_sync(0xFFFFFFFFu, incl, 31);
@@ -506,13 +515,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           s_list[x] = j;
         }
       }
+      __syncwarp();
+      for (int x = lane; x < cnt; x += 32) s_blen[x] = __ldg(a.block_len + s_list[x]);
       __threadfence_block();
       __syncwarp();
       if (lane == 0) {
         *s_cnt = cnt;
         mbar_arrive(list_full);
         const int64_t row0 = bh * a.n_pad;
-        auto load_y = [&](int n, uint32_t s) {
+        const int U = cnt * HS;
+        auto load_y = [&](int n) {
+          const uint32_t s = (Gs + n) % NS;
           const int j = s_list[n];
           const int r = int(row0 + int64_t(j) * R);
           const uint32_t bar = y_full + 8 * s;
@@ -530,86 +543,110 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           }
           ++y_issued[s];
         };
+        // S (or S^T) and dP (or dP^T) of half-step u into buffer (G + u) & 1
+        auto issue_sd = [&](int u) -> bool {
+          const int n = u / HS, c = u % HS;
+          const uint32_t s = (Gs + n) % NS, w = (G + u) & 1;
+          if (u == 0) {
+            if (!wait_bar(x_full, (x_loads - 1) & 1, abort_flag, a.status, 41)) return false;
+            x_pending = false;
+          }
+          if (c == 0) {
+            if (!wait_bar(y_full + 8 * s, ((Gs + n) / NS) & 1, abort_flag, a.status, 42)) return false;
+            ++y_seen[s];
+          }
+          tc_fence_after();
+          const uint32_t y1 = sY + s * 2 * C::YBYTES, y2 = y1 + C::YBYTES;
+          const uint32_t buf = tmem + C::COL_BUF + w * 2 * NH;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t ko = (ks / 4) * 128u * 128u + (ks % 4) * 32u;
+            const uint32_t kn = (ks / 4) * uint32_t(N) * 128u + uint32_t(c * NH) * 128u + (ks % 4) * 32u;
+            umma_bf16(buf, sdesc_sw128(sX1 + ko, 16, 1024), sdesc_sw128(y1 + kn, 16, 1024), C::IDESC_SS,
+                      ks > 0 ? 1u : 0u);
+            umma_bf16(buf + NH, sdesc_sw128(sX2 + ko, 16, 1024), sdesc_sw128(y2 + kn, 16, 1024),
+                      C::IDESC_SS, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full + 8 * w);
+          return true;
+        };
         if (cnt > 0) {
           mbar_expect_tx(x_full, 2 * C::XBYTES);
           const int r = int(row0 + int64_t(rt) * R);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(sX1 + c * kBwdM * 128, &tm_x1, x_full, c * 64, r);
-            tma_load_2d(sX2 + c * kBwdM * 128, &tm_x2, x_full, c * 64, r);
+            tma_load_2d_hint(sX1 + c * kBwdM * 128, &tm_x1, x_full, c * 64, r, l2_evict_first_policy());
+            tma_load_2d_hint(sX2 + c * kBwdM * 128, &tm_x2, x_full, c * 64, r, l2_evict_first_policy());
           }
           ++x_loads;
           x_pending = true;
-          for (int n = 0; n < cnt && n < 2; ++n) load_y(n, (g + n) & 1);
+          for (int n = 0; n < cnt && n < NS; ++n) load_y(n);
+          ok = issue_sd(0) && (U < 2 || issue_sd(1));
         }
-        for (int n = 0; n < cnt; ++n) {
-          const uint32_t gs = g + n, s = gs & 1;
-          if (n == 0) {
-            if (!wait_bar(x_full, (x_loads - 1) & 1, abort_flag, a.status, 41)) { ok = false; break; }
-            x_pending = false;
-          }
-          if (!wait_bar(y_full + 8 * s, (gs >> 1) & 1, abort_flag, a.status, 42)) { ok = false; break; }
-          ++y_seen[s];
+        for (int u = 0; u < U && ok; ++u) {
+          const int n = u / HS, c = u % HS;
+          const uint32_t s = (Gs + n) % NS, w = (G + u) & 1;
+          const uint32_t idx = hw[w]++;
+          if (!wait_bar(p_ready + 8 * w, idx & 1, abort_flag, a.status, 43)) { ok = false; break; }
           tc_fence_after();
           const uint32_t y1 = sY + s * 2 * C::YBYTES, y2 = y1 + C::YBYTES;
+          const uint32_t buf = tmem + C::COL_BUF + w * 2 * NH;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t ko = (ks / 4) * 128u * 128u + (ks % 4) * 32u;
-            const uint32_t kn = (ks / 4) * uint32_t(N) * 128u + (ks % 4) * 32u;
-            umma_bf16(tmem + C::COL_S, sdesc_sw128(sX1 + ko, 16, 1024), sdesc_sw128(y1 + kn, 16, 1024),
-                      C::IDESC_SS, ks > 0 ? 1u : 0u);
-            umma_bf16(tmem + C::COL_DP, sdesc_sw128(sX2 + ko, 16, 1024),
-                      sdesc_sw128(y2 + kn, 16, 1024), C::IDESC_SS, ks > 0 ? 1u : 0u);
-          }
-          umma_commit(s_full);
-          if (!wait_bar(p_ready, gs & 1, abort_flag, a.status, 43)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < N / 16; ++ks) {
-            const uint32_t pc = packed_col<N>(ks * 16);
-            const uint32_t acc = (n > 0 || ks > 0) ? 1u : 0u;
+          for (int ks = 0; ks < NH / 16; ++ks) {
+            const uint32_t boff = uint32_t(c * NH + ks * 16) * 128u;
+            const uint32_t acc = (u > 0 || ks > 0) ? 1u : 0u;
             if (kKeyMajor) {
-              // dK += dS^T Q_i,  dV += P^T dO_i   (B operands MN-major)
-              umma_bf16_ts(tmem + C::COL_ACC0, tmem + C::COL_DP + pc,
-                           sdesc_sw128(y1 + ks * 16 * 128, N * 128, 1024), C::IDESC_ACC, acc);
-              umma_bf16_ts(tmem + C::COL_ACC1, tmem + C::COL_S + pc,
-                           sdesc_sw128(y2 + ks * 16 * 128, N * 128, 1024), C::IDESC_ACC, acc);
+              // dK += dS^T Q_i,  dV += P^T dO_i   (B operands MN-major; bf16 pairs in
+              // the first NH/2 columns of the dP and S halves of the buffer)
+              umma_bf16_ts(tmem + C::COL_ACC0, buf + NH + ks * 8,
+                           sdesc_sw128(y1 + boff, N * 128, 1024), C::IDESC_ACC, acc);
+              umma_bf16_ts(tmem + C::COL_ACC1, buf + ks * 8, sdesc_sw128(y2 + boff, N * 128, 1024),
+                           C::IDESC_ACC, acc);
             } else {
               // dQ += dS K_j
-              umma_bf16_ts(tmem + C::COL_ACC0, tmem + C::COL_S + pc,
-                           sdesc_sw128(y1 + ks * 16 * 128, N * 128, 1024), C::IDESC_ACC, acc);
+              umma_bf16_ts(tmem + C::COL_ACC0, buf + ks * 8, sdesc_sw128(y1 + boff, N * 128, 1024),
+                           C::IDESC_ACC, acc);
             }
           }
-          umma_commit(mm2_done);
-          if (n == cnt - 1) umma_commit(acc_full);
-          if (!wait_bar(mm2_done, gs & 1, abort_flag, a.status, 44)) { ok = false; break; }
-          if (n + 2 < cnt) load_y(n + 2, s);
+          umma_commit(acc_done + 8 * w);
+          if (u == U - 1) umma_commit(acc_full);
+          if (u + 2 < U) {
+            // buffer w (and, after a step's last half, its stage) is free once
+            // this half-step's products have read it
+            if (!wait_bar(acc_done + 8 * w, idx & 1, abort_flag, a.status, 44)) { ok = false; break; }
+            if (c == HS - 1 && n + NS < cnt) load_y(n + NS);
+            if (!issue_sd(u + 2)) { ok = false; break; }
+          }
         }
-        g += cnt;
+        G += U;
+        Gs += cnt;
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      g = __shfl_sync(0xFFFFFFFFu, g, 0);
+      G = __shfl_sync(0xFFFFFFFFu, G, 0);
+      Gs = __shfl_sync(0xFFFFFFFFu, Gs, 0);
       __syncwarp();
     }
     if (lane == 0 && !ok) {
       // Abort: let every MMA issued above complete and every TMA copy land.
       umma_commit(drain);
       wait_bar_drain(drain, 0);
-      for (int s = 0; s < 2; ++s)
+      for (int s = 0; s < NS; ++s)
         if (y_issued[s] > y_seen[s]) wait_bar_drain(y_full + 8 * s, (y_issued[s] - 1) & 1);
       if (x_pending) wait_bar_drain(x_full, (x_loads - 1) & 1);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise + epilogue
-    // Thread = row of the row tile = TMEM lane; warp half h takes score
-    // columns [h N/2, (h+1) N/2) and accumulator columns [h D/2, (h+1) D/2).
+    // Warpgroup wg (warps 4wg .. 4wg+3) takes the half-steps of buffer wg;
+    // thread = row of the row tile = TMEM lane.  In the epilogue warpgroup wg
+    // writes accumulator columns [wg D/2, (wg+1) D/2).
     constexpr float kLog2e = 1.4426950408889634f;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, wg = warp >> 2;
     const int row = quad * 32 + lane;
     const bool rows_active = (R == 128) || (quad < 2);
     const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
-    uint32_t g = 0, accs = 0;
+    const uint32_t buf = t_lane + C::COL_BUF + wg * 2 * NH;
+    uint32_t G = 0, Gs = 0, mine = 0, accs = 0;
     int t = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
@@ -618,6 +655,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       decode_bwd_item(item, BH, a.n_p, a.T, bh, rt);
       if (!wait_warp(list_full, t & 1, abort_flag, a.status, 45)) { ok = false; break; }
       const int cnt = *s_cnt;
+      const int U = cnt * HS;
       const int blen_row = __ldg(a.block_len + rt);
       float lse2_row = 0.f, delta_row = 0.f;
       if (!kKeyMajor && rows_active && row < blen_row) {
@@ -625,35 +663,36 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         lse2_row = __ldg(a.lse + r) * kLog2e;
         delta_row = __ldg(a.delta + r);
       }
-      for (int n = 0; n < cnt; ++n) {
-        const uint32_t gs = g + n, s = gs & 1;
-        if (!wait_warp(s_full, gs & 1, abort_flag, a.status, 46)) { ok = false; break; }
-        if (kKeyMajor && !wait_warp(y_full + 8 * s, (gs >> 1) & 1, abort_flag, a.status, 47)) {
+      for (int u = int((uint32_t(wg) - G) & 1u); u < U; u += 2) {
+        const int n = u / HS, c = u % HS;
+        const uint32_t s = (Gs + n) % NS;
+        if (!wait_warp(s_full + 8 * wg, mine & 1, abort_flag, a.status, 46)) { ok = false; break; }
+        ++mine;
+        if (kKeyMajor && !wait_warp(y_full + 8 * s, ((Gs + n) / NS) & 1, abort_flag, a.status, 47)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int blen_col = __ldg(a.block_len + s_list[n]);
+        const int blen_col = s_blen[n];
         if (rows_active) {
-          const float* c_lse = s_c + s * (C::CBYTES / 4);
+          const float* c_lse = s_c + s * (C::CBYTES / 4) + c * NH;
           const float* c_del = c_lse + N;
 #pragma unroll
-          for (int cc = 0; cc < N / 64; ++cc) {
-            const int c0 = half * (N / 2) + cc * 32;
+          for (int cc = 0; cc < NH / 32; ++cc) {
             uint32_t sr[32], dr[32];
-            tmem_ld32(t_lane + C::COL_S + c0, sr);
+            tmem_ld32(buf + cc * 32, sr);
             tmem_wait_ld(sr);
-            tmem_ld32(t_lane + C::COL_DP + c0, dr);
+            tmem_ld32(buf + NH + cc * 32, dr);
             tmem_wait_ld(dr);
             uint32_t pp[16], dd[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
               float pv[2], dv[2];
 #pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int col = c0 + e + u;
-                const float sv = __uint_as_float(sr[e + u]);
-                const float dp = __uint_as_float(dr[e + u]);
+              for (int q = 0; q < 2; ++q) {
+                const int col = cc * 32 + e + q;             // within the half-step
+                const float sv = __uint_as_float(sr[e + q]);
+                const float dp = __uint_as_float(dr[e + q]);
                 float l2, dl;
                 if (kKeyMajor) {
                   l2 = c_lse[col] * kLog2e;
@@ -662,28 +701,30 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
                   l2 = lse2_row;
                   dl = delta_row;
                 }
-                const float p = col < blen_col ? ex2f(fmaf(sv, a.scale_log2, -l2)) : 0.f;
-                pv[u] = p;
-                dv[u] = p * (dp - dl);
+                const float p = c * NH + col < blen_col ? ex2f(fmaf(sv, a.scale_log2, -l2)) : 0.f;
+                pv[q] = p;
+                dv[q] = p * (dp - dl);
               }
               pp[e / 2] = pack_bf16(pv[0], pv[1]);
               dd[e / 2] = pack_bf16(dv[0], dv[1]);
             }
+            // bf16 pairs into columns this thread has already read
             if (kKeyMajor) {
-              tmem_st16(t_lane + C::COL_S + packed_col<N>(c0), pp);
-              tmem_st16(t_lane + C::COL_DP + packed_col<N>(c0), dd);
+              tmem_st16(buf + cc * 16, pp);
+              tmem_st16(buf + NH + cc * 16, dd);
             } else {
-              tmem_st16(t_lane + C::COL_S + packed_col<N>(c0), dd);
+              tmem_st16(buf + cc * 16, dd);
             }
           }
           tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_ready);
+        if (lane == 0) mbar_arrive(p_ready + 8 * wg);
       }
       if (!ok) break;
-      g += cnt;
+      G += U;
+      Gs += cnt;
       // epilogue: accumulator (x scale for dQ, dK) + pooled gradient / block_len
       if (cnt > 0) {
         if (!wait_warp(acc_full, accs & 1, abort_flag, a.status, 48)) { ok = false; break; }
@@ -702,7 +743,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           const uint32_t col_acc = o == 0 ? C::COL_ACC0 : C::COL_ACC1;
 #pragma unroll
           for (int cc = 0; cc < D / 64; ++cc) {
-            const int c0 = half * (D / 2) + cc * 32;
+            const int c0 = wg * (D / 2) + cc * 32;
             uint32_t v[32];
             if (cnt > 0) {
               tmem_ld32(t_lane + col_acc + c0, v);
