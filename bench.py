@@ -48,7 +48,7 @@ UNIT = "ms/layer"
 # one-pass ncu capture at the benchmark size summarised in
 # profiles/sparse_attn_veda_h8.md, valid only for the kernel source it was
 # taken on.
-ATTN_TRAFFIC = {"source_sha256_16": "740cc30a2ff525cc", "bytes": 18.70e9}
+ATTN_TRAFFIC = {"source_sha256_16": "0af39b16e1e9c15c", "bytes": 20.28e9}
 
 
 # ----------------------------------------------------------------- accounting

@@ -299,6 +299,7 @@ struct BwdArgs {
   uint16_t* out;              // dQ_t (query-major) or dK_t (key-major), bf16 [BH, N_pad, D]
   uint16_t* out2;             // key-major: dV_t
   unsigned int* status;
+  unsigned int* next_item;    // work counter (zero at launch)
   int T, n_p, k, k_ref, n_sink, W, n_items;
   int64_t n_pad;
   float scale, scale_log2;
@@ -371,23 +372,16 @@ struct BwdCfg {
   static size_t bytes(int T) { return size_t(OFF_LIST) + size_t(8) * ((T + 3) & ~3); }
 };
 
-// Work item -> (b*h, row tile): the video tiles head by head first, so that
-// the CTAs share one head's column-side tiles in L2, then every head's prefix
-// tiles (the longest items in both modes: each streams a whole head).  Run
-// first, the prefix items spread the concurrent reads over all heads and the
-// column-side tiles no longer stayed in L2 (measured: 17x the algorithmic
-// DRAM reads).
-__device__ __forceinline__ void decode_bwd_item(int item, int BH, int n_p, int T, int64_t& bh,
-                                                int& t) {
-  const int n_v = T - n_p;
-  const int first = BH * n_v;
-  if (item < first) {
-    bh = item / n_v;
-    t = n_p + item % n_v;
-  } else {
-    bh = (item - first) / n_p;
-    t = (item - first) % n_p;
-  }
+// Work items are (b*h, row tile) in head-major order (each head's prefix
+// tiles, then its video tiles), handed out in that order from a global
+// counter.  The items' lengths vary (a key tile is attended by as many query
+// tiles as selected it), and under a static round-robin split the CTAs drifted
+// apart by several heads, whose column-side tiles then no longer shared the
+// L2 (measured: 20x the algorithmic DRAM reads of the key-major kernel).
+// Taken in order, the concurrent items stay within one or two heads.
+__device__ __forceinline__ void decode_bwd_item(int item, int T, int64_t& bh, int& t) {
+  bh = item / T;
+  t = item % T;
 }
 
 // Half-step u of an item covers score columns [c*NH, (c+1)*NH) (c = u % HS)
@@ -420,12 +414,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* s_cnt = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  volatile int* s_item = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 12);
   int32_t* s_list = reinterpret_cast<int32_t*>(smem + C::OFF_LIST);
   int32_t* s_blen = s_list + ((a.T + 3) & ~3);
   const float* s_c = reinterpret_cast<const float*>(smem + C::OFF_C);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = a.n_items / a.T;
 
   if (threadIdx.x == 0) {
     mbar_init(x_full, 1);
@@ -470,12 +464,22 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     bool x_pending = false;
     int t = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
-      int64_t bh;
-      int rt;
-      decode_bwd_item(item, BH, a.n_p, a.T, bh, rt);
+    for (; ok; ++t) {
       // the previous item's epilogue is done with the accumulators and the list
       if (t > 0 && !wait_warp(epi_done, (t - 1) & 1, abort_flag, a.status, 40)) { ok = false; break; }
+      int item = 0;
+      if (lane == 0) item = int(atomicAdd(a.next_item, 1u));
+      item = __shfl_sync(0xFFFFFFFFu, item, 0);
+      if (item >= a.n_items) {
+        if (lane == 0) {
+          *s_item = -1;               // tells the elementwise warps to stop
+          mbar_arrive(list_full);
+        }
+        break;
+      }
+      int64_t bh;
+      int rt;
+      decode_bwd_item(item, a.T, bh, rt);
       int cnt = 0;
       if (kKeyMajor) {
         // query tiles whose key set holds key tile rt, ascending
@@ -521,6 +525,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       __syncwarp();
       if (lane == 0) {
         *s_cnt = cnt;
+        *s_item = item;
         mbar_arrive(list_full);
         const int64_t row0 = bh * a.n_pad;
         const int U = cnt * HS;
@@ -649,11 +654,13 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     uint32_t G = 0, Gs = 0, mine = 0, accs = 0;
     int t = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+    for (; ok; ++t) {
+      if (!wait_warp(list_full, t & 1, abort_flag, a.status, 45)) { ok = false; break; }
+      const int item = *s_item;
+      if (item < 0) break;
       int64_t bh;
       int rt;
-      decode_bwd_item(item, BH, a.n_p, a.T, bh, rt);
-      if (!wait_warp(list_full, t & 1, abort_flag, a.status, 45)) { ok = false; break; }
+      decode_bwd_item(item, a.T, bh, rt);
       const int cnt = *s_cnt;
       const int U = cnt * HS;
       const int blen_row = __ldg(a.block_len + rt);
@@ -821,7 +828,10 @@ vsa_status launch_bwd_pair(const vsa_plan_s* p, const void* q_t, const void* k_t
                            const void* d_out_t, BwdArgs a, const float* d_qbar, const float* d_kbar,
                            const float* d_vbar, void* dq_t, void* dk_t, void* dv_t, int64_t bh,
                            cudaStream_t stream) {
+  // a.next_item holds the two kernels' counters
+  unsigned int* const counters = a.next_item;
   // dQ: rows = query tile (Q, dO), columns = its key tiles (K, V)
+  a.next_item = counters;
   a.dbar = d_qbar;
   a.dbar2 = nullptr;
   a.out = static_cast<uint16_t*>(dq_t);
@@ -829,6 +839,7 @@ vsa_status launch_bwd_pair(const vsa_plan_s* p, const void* q_t, const void* k_t
   vsa_status st = launch_bwd_rd<R, D, false>(p, q_t, d_out_t, k_t, v_t, a, bh, stream);
   if (st != VSA_OK) return st;
   // dK, dV: rows = key tile (K, V), columns = the query tiles attending to it (Q, dO)
+  a.next_item = counters + 1;
   a.dbar = d_kbar;
   a.dbar2 = d_vbar;
   a.out = static_cast<uint16_t*>(dk_t);
@@ -840,10 +851,14 @@ inline int grid_of(int64_t warps) { return int((warps + 7) / 8); }
 
 }  // namespace
 
-size_t colmask_bytes(const vsa_plan_s* p, int64_t bh) {
+// The attention backward's workspace: the selection bitmap, then the two
+// kernels' work counters (16 bytes), all zeroed by one memset per call.
+static size_t bitmap_bytes(const vsa_plan_s* p, int64_t bh) {
   const int W = (p->n_tiles + 31) / 32;
-  return size_t(bh) * p->n_tiles * W * 4;
+  return (size_t(bh) * p->n_tiles * W * 4 + 15) & ~size_t(15);
 }
+
+size_t colmask_bytes(const vsa_plan_s* p, int64_t bh) { return bitmap_bytes(p, bh) + 16; }
 
 size_t coarse_bwd_bytes(const vsa_plan_s* p, int64_t bh) {
   return size_t(2) * bh * p->n_tiles * p->n_tiles * 4;
@@ -912,6 +927,7 @@ vsa_status launch_sparse_attn_backward(const vsa_plan_s* p, const void* q_t, con
   a.topk = topk_idx;
   a.topk_ref = k_ref < 0 ? nullptr : topk_ref;
   a.colmask = static_cast<const uint32_t*>(ws);
+  a.next_item = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + bitmap_bytes(p, bh));
   a.lse = lse_t;
   a.delta = delta;
   a.status = p->d_status;
