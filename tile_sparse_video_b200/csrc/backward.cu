@@ -339,6 +339,58 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// P and dS of 32 score columns of one row: P = 2^(S scale log2(e) - lse
+// log2(e)) (0 at or past column `lim`), dS = P (dP - delta), as bf16 pairs.
+// Query-major: lse and delta are the row's (nl2_row = -lse log2(e));
+// key-major: the columns' (c_lse, c_del: 32 floats each in shared memory).
+template <bool kKeyMajor, bool kMask>
+__device__ __forceinline__ void p_and_ds_cols(const uint32_t (&sr)[32], const uint32_t (&dr)[32],
+                                              float scale_log2, float nl2_row, float delta_row,
+                                              const float* c_lse, const float* c_del, int lim,
+                                              uint32_t (&pp)[16], uint32_t (&dd)[16]) {
+  constexpr float kLog2e = 1.4426950408889634f;
+#pragma unroll
+  for (int q4 = 0; q4 < 8; ++q4) {
+    float nl[4], dl[4];
+    if (kKeyMajor) {
+      const float4 l4 = *reinterpret_cast<const float4*>(c_lse + 4 * q4);
+      const float4 d4 = *reinterpret_cast<const float4*>(c_del + 4 * q4);
+      nl[0] = -l4.x * kLog2e; nl[1] = -l4.y * kLog2e; nl[2] = -l4.z * kLog2e; nl[3] = -l4.w * kLog2e;
+      dl[0] = d4.x; dl[1] = d4.y; dl[2] = d4.z; dl[3] = d4.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        nl[e] = nl2_row;
+        dl[e] = delta_row;
+      }
+    }
+    float pv[4], dv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int col = 4 * q4 + e;
+      float p = ex2f(fmaf(__uint_as_float(sr[col]), scale_log2, nl[e]));
+      if (kMask && col >= lim) p = 0.f;
+      pv[e] = p;
+      dv[e] = p * (__uint_as_float(dr[col]) - dl[e]);
+    }
+    pp[2 * q4] = pack_bf16(pv[0], pv[1]);
+    pp[2 * q4 + 1] = pack_bf16(pv[2], pv[3]);
+    dd[2 * q4] = pack_bf16(dv[0], dv[1]);
+    dd[2 * q4 + 1] = pack_bf16(dv[2], dv[3]);
+  }
+}
+
+template <bool kKeyMajor>
+__device__ __forceinline__ void p_and_ds(const uint32_t (&sr)[32], const uint32_t (&dr)[32],
+                                         float scale_log2, float nl2_row, float delta_row,
+                                         const float* c_lse, const float* c_del, int lim,
+                                         uint32_t (&pp)[16], uint32_t (&dd)[16]) {
+  if (lim >= 32)   // every column live (the common case): no mask
+    p_and_ds_cols<kKeyMajor, false>(sr, dr, scale_log2, nl2_row, delta_row, c_lse, c_del, lim, pp, dd);
+  else
+    p_and_ds_cols<kKeyMajor, true>(sr, dr, scale_log2, nl2_row, delta_row, c_lse, c_del, lim, pp, dd);
+}
+
 template <int R, int D, bool kKeyMajor>
 struct BwdCfg {
   static constexpr int N = R;                       // rows of a column-side tile
@@ -664,10 +716,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int cnt = *s_cnt;
       const int U = cnt * HS;
       const int blen_row = __ldg(a.block_len + rt);
-      float lse2_row = 0.f, delta_row = 0.f;
+      float nl2_row = 0.f, delta_row = 0.f;       // query-major: -lse*log2(e) and delta of the row
       if (!kKeyMajor && rows_active && row < blen_row) {
         const int64_t r = bh * a.n_pad + int64_t(rt) * R + row;
-        lse2_row = __ldg(a.lse + r) * kLog2e;
+        nl2_row = -__ldg(a.lse + r) * kLog2e;
         delta_row = __ldg(a.delta + r);
       }
       for (int u = int((uint32_t(wg) - G) & 1u); u < U; u += 2) {
@@ -684,37 +736,16 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (rows_active) {
           const float* c_lse = s_c + s * (C::CBYTES / 4) + c * NH;
           const float* c_del = c_lse + N;
+          const int lim = blen_col - c * NH;           // live score columns of this half-step
 #pragma unroll
           for (int cc = 0; cc < NH / 32; ++cc) {
-            uint32_t sr[32], dr[32];
+            uint32_t sr[32], dr[32], pp[16], dd[16];
             tmem_ld32(buf + cc * 32, sr);
-            tmem_wait_ld(sr);
             tmem_ld32(buf + NH + cc * 32, dr);
+            tmem_wait_ld(sr);
             tmem_wait_ld(dr);
-            uint32_t pp[16], dd[16];
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float pv[2], dv[2];
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const int col = cc * 32 + e + q;             // within the half-step
-                const float sv = __uint_as_float(sr[e + q]);
-                const float dp = __uint_as_float(dr[e + q]);
-                float l2, dl;
-                if (kKeyMajor) {
-                  l2 = c_lse[col] * kLog2e;
-                  dl = c_del[col];
-                } else {
-                  l2 = lse2_row;
-                  dl = delta_row;
-                }
-                const float p = c * NH + col < blen_col ? ex2f(fmaf(sv, a.scale_log2, -l2)) : 0.f;
-                pv[q] = p;
-                dv[q] = p * (dp - dl);
-              }
-              pp[e / 2] = pack_bf16(pv[0], pv[1]);
-              dd[e / 2] = pack_bf16(dv[0], dv[1]);
-            }
+            p_and_ds<kKeyMajor>(sr, dr, a.scale_log2, nl2_row, delta_row, c_lse + cc * 32,
+                                c_del + cc * 32, lim - cc * 32, pp, dd);
             // bf16 pairs into columns this thread has already read
             if (kKeyMajor) {
               tmem_st16(buf + cc * 16, pp);
