@@ -257,10 +257,27 @@ def projection_timing(w: Workload, plan, dev, stream, steps: int) -> dict:
     ref_ms = timed(lambda: torch.matmul(x2, wt.t()))
     flop = 2.0 * N * C * HD
     peaks = load_peaks()
-    return {"shape": f"x[{N}x{C}] W[{HD}x{C}] -> [{w.H},{N},{w.D}]", "ms": round(ms, 4),
-            "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
-            "frac": round(flop / (ms * 1e-3) / 1e12 / peaks["bf16"], 4),
-            "cublas_ms": round(ref_ms, 4), "gpu_launches_per_call": 1}
+    # tile before projecting: the layer input permuted once, then Q, K, V and
+    # the gate projected on the tiled rows (vsa.TiledInputProjection)
+    del y
+    proj = vsa.TiledInputProjection(plan, 1, w.H, w.D, C, dev)
+    perm_ms = timed(lambda: vsa.vsa_permute_rows(plan, x, proj.x_t))
+    tiled_ms = timed(lambda: proj(x, wt, wt, wt, wt))
+    vsa.vsa_sync_status(plan)
+    x_bytes = 2.0 * (N + plan.n_padded) * C
+    res = {"shape": f"x[{N}x{C}] W[{HD}x{C}] -> [{w.H},{N},{w.D}]", "ms": round(ms, 4),
+           "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+           "frac": round(flop / (ms * 1e-3) / 1e12 / peaks["bf16"], 4),
+           "cublas_ms": round(ref_ms, 4), "gpu_launches_per_call": 1,
+           "tiled_input_projection": {
+               "what": "vsa_permute_rows(x) + vsa_project_tiled for Q, K, V and the gate",
+               "ms": round(tiled_ms, 4), "permute_rows_ms": round(perm_ms, 4),
+               "permute_rows_gbs": round(x_bytes / (perm_ms * 1e-3) / 1e9, 1),
+               "gemm_tflops": round(4 * flop / ((tiled_ms - perm_ms) * 1e-3) / 1e12, 1),
+               "gpu_launches_per_call": 5}}
+    del proj
+    torch.cuda.empty_cache()
+    return res
 
 
 def backward_timing(w: Workload, plan, dev, stream, inp_dev, k: int, kept_flop: float,

@@ -203,6 +203,20 @@ vsa_status vsa_sparse_attn_ref(vsa_plan plan, const void* q_t, const void* k_t, 
 vsa_status vsa_project(vsa_plan plan, const void* x, const void* w, int B, int H, int D, int C,
                        int act, void* y, void* stream);
 
+/* Tile before projecting (SnackOnAI, "The Code, Annotated", snippet two: the
+ * layer input x is tiled first and the tiled x_t is projected, so that Q, K, V
+ * and the gate come out in tile order without four sequence-sized copies).
+ * vsa_permute_rows: x_t[b, untile[n], :] = x[b, n, :], pad rows 0; x bf16
+ * [B,N,C] natural order, x_t bf16 [B,N_pad,C]; C a multiple of 8, pointers
+ * 16-byte aligned.  vsa_project_tiled: vsa_project on the tiled rows,
+ * x_t bf16 [B,N_pad,C] -> y_t bf16 [B,H,N_pad,D] (pad rows of a zero-padded x_t
+ * hold act(0): 0 for the identity).  A row permutation commutes with the
+ * row-wise product, so vsa_project_tiled(vsa_permute_rows(x)) equals
+ * vsa_permute(vsa_project(x)) element for element. */
+vsa_status vsa_permute_rows(vsa_plan plan, const void* x, void* x_t, int B, int C, void* stream);
+vsa_status vsa_project_tiled(vsa_plan plan, const void* x_t, const void* w, int B, int H, int D,
+                             int C, int act, void* y_t, void* stream);
+
 /* Allocation-free variant of vsa_coarse_topk (the pages have no counterpart:
  * this is a library convenience).  For callers that cannot call cudaMalloc --
  * a host application that owns all device memory and gives plugins no

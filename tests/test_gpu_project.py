@@ -86,3 +86,62 @@ def test_projection_rejects_bad_arguments():
         vsa.vsa_project(plan, x, wt, 2, 128)
     assert e.value.status == 1
     vsa.vsa_sync_status(plan)
+
+
+# --------------------------------------------------------------------------
+# Tile before projecting: vsa_permute_rows + vsa_project_tiled
+# --------------------------------------------------------------------------
+
+TILED_CASES = [
+    _case("tiled_tiny", TINY.prefix, TINY.grid, TINY.tile, 1, 2, 128, 64, 21),
+    _case("tiled_ragged_b2", (5, 0, 64, 65), (5, 6, 7), (4, 4, 4), 2, 3, 64, 200, 22),
+    _case("tiled_r128", (256, 3), (8, 17, 9), (4, 8, 4), 1, 3, 128, 520, 23),
+]
+
+
+@pytest.mark.parametrize("w", TILED_CASES, ids=lambda c: c.name)
+def test_permute_rows_bit_exact(w):
+    """x_t[b, untile[n]] = x[b, n], pad rows zero, for rows of any width."""
+    inp = make_projection_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    x_t = vsa.vsa_permute_rows(plan, inp["x"].cuda())
+    vsa.vsa_sync_status(plan)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    assert np.array_equal(x_t.cpu().to(torch.float64).numpy(), O.permute(inp["x"].to(torch.float64).numpy(), p))
+
+
+@pytest.mark.parametrize("w,sig", [(TILED_CASES[0], False), (TILED_CASES[1], True), (TILED_CASES[2], False)],
+                         ids=lambda c: getattr(c, "name", str(c)))
+def test_project_tiled_equals_project_then_permute(w, sig):
+    """Projecting the tiled input gives the tiled projection: bit-identical to
+    vsa_permute(vsa_project(x)) on live rows (the same row products in the same
+    order), act(0) on pad rows, and within the projection bound of the oracle."""
+    inp = make_projection_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    x, wt = inp["x"].cuda(), inp["w"].cuda()
+    y_t = vsa.vsa_project_tiled(plan, vsa.vsa_permute_rows(plan, x), wt, w.H, w.D, sigmoid=sig)
+    ref = vsa.vsa_permute(plan, vsa.vsa_project(plan, x, wt, w.H, w.D, sigmoid=sig))
+    vsa.vsa_sync_status(plan)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    live = torch.from_numpy(p.row_src >= 0).cuda()
+    assert torch.equal(y_t[:, :, live], ref[:, :, live])
+    pad = y_t[:, :, ~live].to(torch.float32)
+    assert torch.all(pad == (0.5 if sig else 0.0))
+    want = O.permute(O.project(inp["x"], inp["w"], w.H, w.D, act="sigmoid" if sig else None), p)
+    got = y_t.cpu().to(torch.float64).numpy()[:, :, p.row_src >= 0]
+    _check(torch.from_numpy(got), want[:, :, p.row_src >= 0])
+
+
+def test_tiled_input_projection_full_size():
+    """The Veda layer input (104,704 tokens x 5,376) through
+    vsa.TiledInputProjection: q_t equals vsa_permute(vsa_project(x, w_q))
+    element for element."""
+    w = VEDA_104K
+    inp = make_projection_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    x, wt = inp["x"].cuda(), inp["w"].cuda()
+    proj = vsa.TiledInputProjection(plan, w.B, w.H, w.D, w.gate_width)
+    q_t, k_t, v_t, g_t = proj(x, wt, wt, wt, wt)
+    ref = vsa.vsa_permute(plan, vsa.vsa_project(plan, x, wt, w.H, w.D))
+    vsa.vsa_sync_status(plan)
+    assert torch.equal(q_t, ref) and torch.equal(g_t, ref)

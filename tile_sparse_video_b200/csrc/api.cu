@@ -290,7 +290,38 @@ vsa_status vsa_project(vsa_plan p, const void* x, const void* w, int B, int H, i
   VSA_TRY(check_ptr(x, "x"));
   VSA_TRY(check_ptr(w, "w"));
   VSA_TRY(check_ptr(y, "y"));
-  return launch_project(p, x, w, B, H, D, C, act, y, static_cast<cudaStream_t>(stream));
+  return launch_project(p, x, w, B, H, D, C, act, 0, y, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_project_tiled(vsa_plan p, const void* x_t, const void* w, int B, int H, int D, int C,
+                             int act, void* y_t, void* stream) {
+  bool empty = false;
+  VSA_TRY(check_launch(p, B, H, D, &empty));
+  if (C <= 0 || C % 8 != 0) return fail(VSA_ERR_INVALID_ARG, "C must be a positive multiple of 8");
+  if (act != 0 && act != 1) return fail(VSA_ERR_INVALID_ARG, "act must be 0 (identity) or 1 (sigmoid)");
+  if (empty) return VSA_OK;
+  VSA_TRY(check_ptr(x_t, "x_t"));
+  VSA_TRY(check_ptr(w, "w"));
+  VSA_TRY(check_ptr(y_t, "y_t"));
+  return launch_project(p, x_t, w, B, H, D, C, act, 1, y_t, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_permute_rows(vsa_plan p, const void* x, void* x_t, int B, int C, void* stream) {
+  if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
+  if (p->device < 0) return fail(VSA_ERR_INVALID_ARG, "host-only plan (device = -1) cannot launch");
+  if (B < 0) return fail(VSA_ERR_INVALID_ARG, "B must be >= 0");
+  if (C <= 0 || C % 8 != 0) return fail(VSA_ERR_INVALID_ARG, "C must be a positive multiple of 8");
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur != p->device)
+    return fail(VSA_ERR_INVALID_ARG, "current CUDA device differs from the plan's device");
+  if (B == 0 || p->n_tokens == 0) return VSA_OK;
+  VSA_TRY(check_ptr(x, "x"));
+  VSA_TRY(check_ptr(x_t, "x_t"));
+  e = launch_gather_wide(static_cast<const uint16_t*>(x), static_cast<uint16_t*>(x_t), p->d_row_src,
+                         B, p->n_tokens, p->n_padded, C, p->num_sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "permute_rows launch");
 }
 
 vsa_status vsa_sparse_attn(vsa_plan p, const void* q_t, const void* k_t, const void* v_t,

@@ -57,6 +57,39 @@ __global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint4* __re
   }
 }
 
+// Rows of any width (C bf16, C a multiple of 8): dst[b, r, :] = map[r] >= 0 ?
+// src[b, map[r], :] : 0.  One warp per destination row; the lanes walk its
+// 16-byte chunks with kUnroll loads in flight.  Used to put the layer input
+// into tile order before its projections.
+__global__ void __launch_bounds__(kThreads) gather_wide_kernel(const uint4* __restrict__ src,
+                                                               uint4* __restrict__ dst,
+                                                               const int32_t* __restrict__ map,
+                                                               int64_t src_rows, int64_t dst_rows,
+                                                               int64_t n_rows, int cpr) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = int64_t(gridDim.x) * (kThreads / 32);
+  for (int64_t w = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); w < n_rows;
+       w += warps) {
+    const int64_t b = w / dst_rows, r = w % dst_rows;
+    const int32_t m = __ldg(map + r);
+    uint4* d = dst + w * cpr;
+    const uint4* s = src + (b * src_rows + (m >= 0 ? m : 0)) * cpr;
+    for (int c0 = lane; c0 < cpr; c0 += 32 * kUnroll) {
+      uint4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int c = c0 + 32 * u;
+        v[u] = (m >= 0 && c < cpr) ? ldg_nc(s + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < cpr) d[c] = v[u];
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -271,6 +304,20 @@ cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, const int32_t
     gather_rows_kernel<8><<<grid, kThreads, 0, stream>>>(reinterpret_cast<const uint4*>(src),
                                                          reinterpret_cast<uint4*>(dst), map,
                                                          src_rows, dst_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_wide(const uint16_t* src, uint16_t* dst, const int32_t* map, int64_t B,
+                               int64_t src_rows, int64_t dst_rows, int C, int num_sms,
+                               cudaStream_t stream) {
+  const int64_t n_rows = B * dst_rows;
+  if (n_rows == 0) return cudaSuccess;
+  const int64_t want = int64_t(num_sms > 0 ? num_sms : 148) * 8;
+  int64_t blocks = (n_rows + 7) / 8;
+  if (blocks > want) blocks = want;
+  gather_wide_kernel<<<unsigned(blocks), kThreads, 0, stream>>>(
+      reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), map, src_rows, dst_rows,
+      n_rows, C / 8);
   return cudaGetLastError();
 }
 

@@ -225,8 +225,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
 }  // namespace
 
 vsa_status launch_project(const vsa_plan_s* p, const void* x, const void* w, int B, int H, int D,
-                          int C, int act, void* y, cudaStream_t stream) {
-  const int64_t M = int64_t(B) * p->n_tokens;
+                          int C, int act, int tiled, void* y, cudaStream_t stream) {
+  const int64_t rows_per_b = tiled ? p->n_padded : p->n_tokens;
+  const int64_t M = int64_t(B) * rows_per_b;
   const int HD = H * D;
   if (M >= (int64_t(1) << 31) || HD >= (1 << 20))
     return fail(VSA_ERR_UNSUPPORTED, "projection too large for 32-bit TMA coordinates");
@@ -240,7 +241,7 @@ vsa_status launch_project(const vsa_plan_s* p, const void* x, const void* w, int
   a.y = static_cast<uint16_t*>(y);
   a.status = p->d_status;
   a.M = M;
-  a.N = p->n_tokens;
+  a.N = rows_per_b;
   a.H = H;
   a.D = D;
   a.C = C;

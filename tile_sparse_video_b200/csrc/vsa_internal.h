@@ -41,6 +41,10 @@ vsa_status build_plan(const vsa_geometry& g, vsa_plan_s* p);
 cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, const int32_t* map,
                                int64_t bh, int64_t src_rows, int64_t dst_rows, int D,
                                int num_sms, cudaStream_t stream);
+// Rows of C bf16 (C a multiple of 8): dst[b, r] = map[r] >= 0 ? src[b, map[r]] : 0.
+cudaError_t launch_gather_wide(const uint16_t* src, uint16_t* dst, const int32_t* map, int64_t B,
+                               int64_t src_rows, int64_t dst_rows, int C, int num_sms,
+                               cudaStream_t stream);
 cudaError_t launch_pool(const uint16_t* q_t, const uint16_t* k_t, const uint16_t* v_t,
                         const int32_t* block_len, float* qbar, float* kbar, float* vbar,
                         int64_t bh, int T, int R, int D, int num_sms, cudaStream_t stream);
@@ -71,8 +75,10 @@ vsa_status launch_sparse_attn(const vsa_plan_s* p, const void* q_t, const void* 
                               const float* o_coarse, const int32_t* topk_ref, int k_ref,
                               cudaStream_t stream);
 
+// tiled = 0: x [B, N, C] natural rows -> y [B, H, N, D]; tiled = 1: x [B, N_pad, C]
+// in tile order -> y [B, H, N_pad, D] (pad rows hold act(0)).
 vsa_status launch_project(const vsa_plan_s* p, const void* x, const void* w, int B, int H, int D,
-                          int C, int act, void* y, cudaStream_t stream);
+                          int C, int act, int tiled, void* y, cudaStream_t stream);
 
 // Backward (backward.cu).
 size_t colmask_bytes(const vsa_plan_s* p, int64_t bh);

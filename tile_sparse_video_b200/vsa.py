@@ -28,7 +28,8 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_coun
            "vsa_plan_destroy", "vsa_workspace_size", "vsa_permute", "vsa_unpermute",
            "vsa_permute_pool", "vsa_coarse_topk", "vsa_coarse_topk_pooled",
            "vsa_coarse_topk_noalloc", "vsa_sparse_attn", "vsa_sparse_attn_combine",
-           "vsa_gate_combine", "vsa_project", "vsa_keep_count_ref", "vsa_select_reference",
+           "vsa_gate_combine", "vsa_project", "vsa_project_tiled", "vsa_permute_rows",
+           "vsa_keep_count_ref", "vsa_select_reference",
            "vsa_sparse_attn_ref", "vsa_backward_workspace_size", "vsa_combine_backward",
            "vsa_coarse_backward", "vsa_sparse_attn_backward", "vsa_sync_status", "vsa_last_error")
 
@@ -73,6 +74,8 @@ def lib():
             "vsa_sparse_attn_combine": [P, V, V, V, V, I, I, I, I, F, V, V, V, V, V],
             "vsa_gate_combine": [P, V, V, V, V, I, I, I, I, V],
             "vsa_project": [P, V, V, I, I, I, I, I, V, V],
+            "vsa_project_tiled": [P, V, V, I, I, I, I, I, V, V],
+            "vsa_permute_rows": [P, V, V, I, I, V],
             "vsa_keep_count_ref": [P, D, I32, ctypes.POINTER(I32)],
             "vsa_select_reference": [P, I, I, I, F, I, V, V, Z, V],
             "vsa_sparse_attn_ref": [P, V, V, V, V, I, V, I, I, I, I, F, V, V, V, V, V],
@@ -363,6 +366,57 @@ def vsa_project(plan: Plan, x: torch.Tensor, w: torch.Tensor, H: int, D: int, si
     _check(lib().vsa_project(plan.handle, _ptr(x), _ptr(w), B, H, D, C, 1 if sigmoid else 0, _ptr(y),
                              _stream(stream)))
     return y
+
+
+def vsa_permute_rows(plan: Plan, x: torch.Tensor, x_t: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Tile order for rows of any width: x bf16 [B,N,C] -> x_t bf16 [B,N_pad,C]
+    (pad rows 0), the layer input before its projections."""
+    B, N, C = x.shape
+    _need(x, "x", torch.bfloat16, (B, plan.n_tokens, C))
+    if x_t is None:
+        x_t = torch.empty(B, plan.n_padded, C, dtype=torch.bfloat16, device=x.device)
+    _need(x_t, "x_t", torch.bfloat16, (B, plan.n_padded, C))
+    _check(lib().vsa_permute_rows(plan.handle, _ptr(x), _ptr(x_t), B, C, _stream(stream)))
+    return x_t
+
+
+def vsa_project_tiled(plan: Plan, x_t: torch.Tensor, w: torch.Tensor, H: int, D: int,
+                      sigmoid: bool = False, y_t: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """vsa_project on tiled rows: x_t bf16 [B,N_pad,C] (from vsa_permute_rows),
+    w bf16 [H*D,C]; returns y_t bf16 [B,H,N_pad,D] in tile order."""
+    B, Np, C = x_t.shape
+    _need(x_t, "x_t", torch.bfloat16, (B, plan.n_padded, C))
+    _need(w, "w", torch.bfloat16, (H * D, C))
+    if y_t is None:
+        y_t = torch.empty(B, H, plan.n_padded, D, dtype=torch.bfloat16, device=x_t.device)
+    _need(y_t, "y_t", torch.bfloat16, (B, H, plan.n_padded, D))
+    _check(lib().vsa_project_tiled(plan.handle, _ptr(x_t), _ptr(w), B, H, D, C, 1 if sigmoid else 0,
+                                   _ptr(y_t), _stream(stream)))
+    return y_t
+
+
+class TiledInputProjection:
+    """Q, K, V and the gate of a layer from its input x [B,N,C], tiled before
+    projecting: one vsa_permute_rows of x, then four tcgen05 GEMMs on the tiled
+    rows (vsa_project_tiled) writing q_t, k_t, v_t and g_t [B,H,N_pad,D] in tile
+    order, ready for vsa_coarse_topk, vsa_sparse_attn and vsa_gate_combine.
+    Weights are nn.Linear layout [H*D, C], bias-free."""
+
+    def __init__(self, plan: Plan, B: int, H: int, D: int, C: int, device=None):
+        self.plan, self.B, self.H, self.D, self.C = plan, B, H, D, C
+        dev = torch.device("cuda", plan.device) if device is None else torch.device(device)
+        self.x_t = torch.empty(B, plan.n_padded, C, dtype=torch.bfloat16, device=dev)
+        self.out = tuple(torch.empty(B, H, plan.n_padded, D, dtype=torch.bfloat16, device=dev)
+                         for _ in range(4))
+
+    def __call__(self, x, w_q, w_k, w_v, w_g, stream=None):
+        p = self.plan
+        vsa_permute_rows(p, x, self.x_t, stream)
+        for w, y in zip((w_q, w_k, w_v, w_g), self.out):
+            vsa_project_tiled(p, self.x_t, w, self.H, self.D, y_t=y, stream=stream)
+        return self.out
 
 
 def vsa_keep_count_ref(plan: Plan, keep_ratio: Optional[float] = None,
