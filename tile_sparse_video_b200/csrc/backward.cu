@@ -27,14 +27,17 @@
 //   colmask_kernel       for every key tile, the bitmap of the query tiles
 //                        that attend to it (the transpose of the selection).
 //   attn_bwd_kernel<R, D, kKeyMajor>: tcgen05 kernel, one persistent CTA per
-//                        SM.  Query-major (dQ): work item = (b*h, query tile
-//                        i), loop over its key tiles.  Key-major (dK, dV):
-//                        item = (b*h, key tile j), loop over the query tiles
-//                        whose key set holds j.  Per step the two score-side
-//                        products go to TMEM (S and dP, M=128, N=R, K=D), the
-//                        elementwise warps turn them into bf16 P / dS in TMEM,
-//                        and TS-MMAs accumulate dQ (or dK and dV) in TMEM.
-//                        The epilogue adds the pooling term and writes bf16.
+//                        SM taking work items from a global counter.
+//                        Query-major (dQ): item = (b*h, query tile i), loop
+//                        over its key tiles.  Key-major (dK, dV): item = (b*h,
+//                        key tile j), loop over the query tiles whose key set
+//                        holds j.  Each step is split into 64-column
+//                        half-steps that alternate between two elementwise
+//                        warpgroups and two TMEM buffers: the score-side
+//                        products go to TMEM (S and dP, M=128, N=64, K=D), the
+//                        warpgroup turns them into bf16 P / dS in TMEM, and
+//                        TS-MMAs accumulate dQ (or dK and dV) in TMEM.  The
+//                        epilogue adds the pooling term and writes bf16.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
