@@ -340,6 +340,14 @@ vsa_status vsa_sparse_attn_backward(vsa_plan plan, const void* q_t, const void* 
                                     float scale, void* dq_t, void* dk_t, void* dv_t, void* ws,
                                     size_t ws_bytes, void* stream);
 
+/* Self-test of the bounded device wait every kernel of the library uses: one
+ * CTA whose two waiting threads wait on an mbarrier that nothing completes.
+ * The waits give up after their bound (2 s of wall time), the kernel records
+ * VSA_ERR_DEVICE_TIMEOUT in the plan's status word (read it with
+ * vsa_sync_status) and returns; result (device int32[2], 16-byte aligned)
+ * receives 0 for each wait that gave up.  The context stays usable. */
+vsa_status vsa_check_bounded_wait(vsa_plan plan, int32_t* result, void* stream);
+
 /* Synchronise `stream`, then read and clear the plan's device status word.
  * Returns VSA_OK, VSA_ERR_DEVICE_TIMEOUT, VSA_ERR_DEVICE_INDEX or VSA_ERR_CUDA. */
 vsa_status vsa_sync_status(vsa_plan plan, void* stream);

@@ -262,6 +262,26 @@ def test_bad_kept_index_is_reported():
     vsa.vsa_sync_status(plan)       # cleared
 
 
+def test_bounded_wait_gives_up_and_reports():
+    """The bounded device wait every kernel uses, on an mbarrier nothing
+    completes (vsa_check_bounded_wait): both waiters give up within the bound,
+    the timeout is reported through the status word, and the context still
+    runs a layer correctly afterwards."""
+    import time
+    w = TINY
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    t0 = time.perf_counter()
+    res = vsa.vsa_check_bounded_wait(plan)
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_sync_status(plan)
+    elapsed = time.perf_counter() - t0
+    assert e.value.status == 6                  # VSA_ERR_DEVICE_TIMEOUT
+    assert res.cpu().tolist() == [0, 0]          # both waits gave up
+    assert 1.5 < elapsed < 30.0, elapsed         # the 2 s bound, not a hang
+    vsa.vsa_sync_status(plan)                    # cleared
+    _check_layer(w, make_inputs(w))              # the context is still usable
+
+
 def test_empty_batch_is_a_no_op():
     plan = vsa.Plan(TINY.prefix, TINY.grid, TINY.tile)
     x = torch.empty(0, 2, plan.n_tokens, 64, dtype=torch.bfloat16, device="cuda")

@@ -564,6 +564,20 @@ vsa_status vsa_sparse_attn_backward(vsa_plan p, const void* q_t, const void* k_t
                                      dq_t, dk_t, dv_t, ws, static_cast<cudaStream_t>(stream));
 }
 
+vsa_status vsa_check_bounded_wait(vsa_plan p, int32_t* result, void* stream) {
+  if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
+  if (p->device < 0) return fail(VSA_ERR_INVALID_ARG, "host-only plan (device = -1) cannot launch");
+  VSA_TRY(check_ptr(result, "result"));
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur != p->device)
+    return fail(VSA_ERR_INVALID_ARG, "current CUDA device differs from the plan's device");
+  e = launch_bounded_wait_check(p->d_status, reinterpret_cast<int*>(result),
+                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "bounded-wait check launch");
+}
+
 vsa_status vsa_sync_status(vsa_plan p, void* stream) {
   if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
   if (p->device < 0) return VSA_OK;

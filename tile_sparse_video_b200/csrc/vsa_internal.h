@@ -100,6 +100,9 @@ vsa_status launch_sparse_attn_backward(const vsa_plan_s* p, const void* q_t, con
                                        void* dq_t, void* dk_t, void* dv_t, void* ws,
                                        cudaStream_t stream);
 
+// Self-test of the bounded wait (selftest.cu): result int32[2], 0 = the wait gave up.
+cudaError_t launch_bounded_wait_check(unsigned int* status, int* result, cudaStream_t stream);
+
 // Device status codes written by kernels into vsa_plan_s::d_status.
 enum : unsigned int { kStatusOk = 0, kStatusTimeout = 1, kStatusBadIndex = 2 };
 

@@ -31,7 +31,8 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_coun
            "vsa_gate_combine", "vsa_project", "vsa_project_tiled", "vsa_permute_rows",
            "vsa_keep_count_ref", "vsa_select_reference",
            "vsa_sparse_attn_ref", "vsa_backward_workspace_size", "vsa_combine_backward",
-           "vsa_coarse_backward", "vsa_sparse_attn_backward", "vsa_sync_status", "vsa_last_error")
+           "vsa_coarse_backward", "vsa_sparse_attn_backward", "vsa_check_bounded_wait",
+           "vsa_sync_status", "vsa_last_error")
 
 
 class VsaError(RuntimeError):
@@ -84,6 +85,7 @@ def lib():
             "vsa_coarse_backward": [P, V, V, V, V, I, I, I, F, V, V, V, V, Z, V],
             "vsa_sparse_attn_backward": [P, V, V, V, V, V, I, V, I, V, V, V, V, V, I, I, I, F,
                                          V, V, V, V, Z, V],
+            "vsa_check_bounded_wait": [P, V, V],
             "vsa_sync_status": [P, V],
         }
         for name, args in sig.items():
@@ -466,6 +468,15 @@ def vsa_sparse_attn_ref(plan: Plan, q_t, k_t, v_t, topk_idx, k: int, topk_ref, k
 
 def vsa_sync_status(plan: Plan, stream=None):
     _check(lib().vsa_sync_status(plan.handle, _stream(stream)))
+
+
+def vsa_check_bounded_wait(plan: Plan, stream=None) -> torch.Tensor:
+    """Launch the bounded-wait self-test (its waits give up after 2 s); returns
+    the device int32[2] result (0 = that wait gave up).  Read the recorded
+    timeout with vsa_sync_status, which raises VsaError(VSA_ERR_DEVICE_TIMEOUT)."""
+    result = torch.full((4,), -1, dtype=torch.int32, device=torch.device("cuda", plan.device))
+    _check(lib().vsa_check_bounded_wait(plan.handle, _ptr(result), _stream(stream)))
+    return result[:2]
 
 
 # ---------------------------------------------------------------- backward
