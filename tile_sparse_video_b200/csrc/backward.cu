@@ -286,9 +286,10 @@ __global__ void __launch_bounds__(256) colmask_kernel(
 
 // ---------------------------------------------------------------- fine backward (tcgen05)
 
-constexpr int kThreadsBwd = 288;   // warps 0-7 elementwise + epilogue, warp 8 lists, TMA and MMA
+constexpr int kThreadsBwd = 320;   // warps 0-7 elementwise + epilogue, 8 lists/TMA/S-dP MMA, 9 accumulating MMA
 constexpr int kBwdM = 128;         // MMA rows: one row tile (rows at or past R are ignored)
 constexpr int kWarpIssue = 8;
+constexpr int kWarpAcc = 9;
 
 struct BwdArgs {
   const int32_t* block_len;   // [T]
@@ -409,8 +410,8 @@ struct BwdCfg {
   static constexpr int OFF_C = OFF_Y + NS * 2 * YBYTES;   // stage s: + s*CBYTES
   static constexpr int OFF_BAR = OFF_C + NS * CBYTES;
   // barriers: x_full, y_full[NS], s_full[2], p_ready[2], acc_done[2], acc_full,
-  //           list_full, epi_done, drain
-  static constexpr int NBAR = 1 + NS + 6 + 4;
+  //           list_full, epi_done, drain, drain2
+  static constexpr int NBAR = 1 + NS + 6 + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;   // tmem slot, abort flag, list count
   static constexpr int OFF_LIST = OFF_MISC + 16;
   // TMEM columns: accumulators (dQ; or dK then dV), then two half-step
@@ -465,7 +466,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   // waiter can fall two phases behind.
   const uint32_t x_full = bar0, y_full = bar0 + 8, s_full = y_full + 8 * NS, p_ready = s_full + 16,
                  acc_done = p_ready + 16, acc_full = acc_done + 16, list_full = acc_full + 8,
-                 epi_done = list_full + 8, drain = epi_done + 8;
+                 epi_done = list_full + 8, drain = epi_done + 8, drain2 = drain + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* s_cnt = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
@@ -488,6 +489,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     mbar_init(list_full, 1);
     mbar_init(epi_done, 8);
     mbar_init(drain, 1);
+    mbar_init(drain2, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -645,6 +647,51 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         }
         for (int u = 0; u < U && ok; ++u) {
           const int n = u / HS, c = u % HS;
+          const uint32_t w = (G + u) & 1;
+          const uint32_t idx = hw[w]++;
+          if (u + 2 < U) {
+            // buffer w (and, after a step's last half, its stage) is free once
+            // the accumulating products of half-step u (warp kWarpAcc) have read it
+            if (!wait_bar(acc_done + 8 * w, idx & 1, abort_flag, a.status, 44)) { ok = false; break; }
+            if (c == HS - 1 && n + NS < cnt) load_y(n + NS);
+            if (!issue_sd(u + 2)) { ok = false; break; }
+          }
+        }
+        G += U;
+        Gs += cnt;
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      G = __shfl_sync(0xFFFFFFFFu, G, 0);
+      Gs = __shfl_sync(0xFFFFFFFFu, Gs, 0);
+      __syncwarp();
+    }
+    if (lane == 0 && !ok) {
+      // Abort: let every MMA issued above complete and every TMA copy land.
+      umma_commit(drain);
+      wait_bar_drain(drain, 0);
+      for (int s = 0; s < NS; ++s)
+        if (y_issued[s] > y_seen[s]) wait_bar_drain(y_full + 8 * s, (y_issued[s] - 1) & 1);
+      if (x_pending) wait_bar_drain(x_full, (x_loads - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == kWarpAcc) {
+    // ------------------------------------------------------------ accumulating MMAs
+    // dQ += dS K_j (or dK += dS^T Q_i, dV += P^T dO_i) of each half-step once
+    // its warpgroup has written P / dS; a warp of its own, so that one
+    // buffer's accumulation never waits behind the other buffer's products.
+    uint32_t G = 0, Gs = 0;
+    uint32_t hw[2] = {0, 0};
+    int t = 0;
+    bool ok = true;
+    for (; ok; ++t) {
+      if (!wait_warp(list_full, t & 1, abort_flag, a.status, 50)) { ok = false; break; }
+      const int item = *s_item;
+      if (item < 0) break;
+      const int cnt = *s_cnt;
+      const int U = cnt * HS;
+      if (lane == 0) {
+        for (int u = 0; u < U; ++u) {
+          const int n = u / HS, c = u % HS;
           const uint32_t s = (Gs + n) % NS, w = (G + u) & 1;
           const uint32_t idx = hw[w]++;
           if (!wait_bar(p_ready + 8 * w, idx & 1, abort_flag, a.status, 43)) { ok = false; break; }
@@ -670,29 +717,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           }
           umma_commit(acc_done + 8 * w);
           if (u == U - 1) umma_commit(acc_full);
-          if (u + 2 < U) {
-            // buffer w (and, after a step's last half, its stage) is free once
-            // this half-step's products have read it
-            if (!wait_bar(acc_done + 8 * w, idx & 1, abort_flag, a.status, 44)) { ok = false; break; }
-            if (c == HS - 1 && n + NS < cnt) load_y(n + NS);
-            if (!issue_sd(u + 2)) { ok = false; break; }
-          }
         }
-        G += U;
-        Gs += cnt;
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      G = __shfl_sync(0xFFFFFFFFu, G, 0);
-      Gs = __shfl_sync(0xFFFFFFFFu, Gs, 0);
+      G += U;
+      Gs += cnt;
       __syncwarp();
     }
     if (lane == 0 && !ok) {
-      // Abort: let every MMA issued above complete and every TMA copy land.
-      umma_commit(drain);
-      wait_bar_drain(drain, 0);
-      for (int s = 0; s < NS; ++s)
-        if (y_issued[s] > y_seen[s]) wait_bar_drain(y_full + 8 * s, (y_issued[s] - 1) & 1);
-      if (x_pending) wait_bar_drain(x_full, (x_loads - 1) & 1);
+      // Abort: let every MMA this warp issued complete.
+      umma_commit(drain2);
+      wait_bar_drain(drain2, 0);
     }
     __syncwarp();
   } else {
