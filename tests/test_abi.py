@@ -93,5 +93,20 @@ def test_host_only_plan_refuses_launches(libvsa):
     assert libvsa.vsa_workspace_size(p.handle, 1, 2, 64, 2, ctypes.byref(n)) == 0
     assert n.value == 3 * 1 * 2 * p.n_tiles * 64 * 4
     assert libvsa.vsa_workspace_size(p.handle, 1, 2, 96, 2, ctypes.byref(n)) == 2
+    # the calls added for training and tile-before-projecting refuse a host-only plan too
+    vp = ctypes.cast(buf, ctypes.c_void_p)
+    assert libvsa.vsa_permute_rows(p.handle, vp, vp, 1, 64, None) == 1
+    assert libvsa.vsa_project_tiled(p.handle, vp, vp, 1, 2, 64, 64, 0, vp, None) == 1
+    assert libvsa.vsa_combine_backward(p.handle, vp, vp, vp, vp, 1, 2, 64, vp, vp, vp, None) == 1
+    assert libvsa.vsa_check_bounded_wait(p.handle, vp, None) == 1
+    assert b"host-only" in libvsa.vsa_last_error()
+    # backward workspace: the larger of the coarse backward's P and dS (2 x [B*H, T, T]
+    # fp32) and the attention backward's bitmap (B*H*T*ceil(T/32) words, 16-byte
+    # rounded) plus its two work counters (16 bytes)
+    assert libvsa.vsa_backward_workspace_size(p.handle, 1, 2, 64, ctypes.byref(n)) == 0
+    T = p.n_tiles
+    bitmap = (2 * T * ((T + 31) // 32) * 4 + 15) // 16 * 16 + 16
+    assert n.value == max(2 * 2 * T * T * 4, bitmap)
+    assert libvsa.vsa_backward_workspace_size(p.handle, 1, 2, 96, ctypes.byref(n)) == 2
     assert libvsa.vsa_plan_destroy(None) == 0
     p.close()
