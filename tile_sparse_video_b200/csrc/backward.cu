@@ -460,7 +460,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   // x_full: row-side tiles of an item.  y_full[s]: column-side tiles (and, key-
   // major, their lse / delta) of the steps using stage s.  s_full[w],
   // p_ready[w] and acc_done[w] complete once per half-step of buffer w;
-  // acc_full once per item with steps; list_full and epi_done once per item.
+  // acc_full once per item with steps; list_full and epi_done once per item
+  // (epi_done: the eight elementwise warps after the epilogue and the
+  // accumulating warp after its last product of the item).
   // The issuer reuses buffer w (and reloads a stage) only after acc_done of
   // its previous half-step, which follows that half-step's p_ready, so no
   // waiter can fall two phases behind.
@@ -487,7 +489,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(list_full, 1);
-    mbar_init(epi_done, 8);
+    mbar_init(epi_done, 9);          // 8 elementwise warps + the accumulating warp
     mbar_init(drain, 1);
     mbar_init(drain2, 1);
     *abort_flag = 0;
@@ -722,7 +724,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       G += U;
       Gs += cnt;
+      // this warp is done with the item's list: the next one may be published
+      // (without this arrival an item with no steps could let the list barrier
+      // run two phases ahead of this warp)
       __syncwarp();
+      if (ok && lane == 0) mbar_arrive(epi_done);
     }
     if (lane == 0 && !ok) {
       // Abort: let every MMA this warp issued complete.
