@@ -336,6 +336,7 @@ def backward_timing(w: Workload, plan, dev, stream, inp_dev, k: int, kept_flop: 
     res = {"ms_per_layer": round(float(parts.sum()), 4),
            "kernels_ms": {n: round(float(x), 4) for n, x in zip(names, parts)},
            "combine_backward_hbm_gbs": round(4 * tiled_bytes / (parts[1] * 1e-3) / 1e9, 1),
+           "combine_backward_hbm_frac": round(4 * tiled_bytes / (parts[1] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
            "roofline": {"kernel": "sparse_attn_backward (dQ and dK/dV kernels)", "bound": "tensor",
                         "achieved": round(achieved, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
                         "frac": round(achieved / peaks["bf16"], 4),
@@ -455,6 +456,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                        "coarse_topk": round(float(part_ms[1]), 4),
                        "sparse_attn_combine": round(attn_ms, 4)},
         "kernels_hbm_gbs": {"permute_pool_q_k_v": round(acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9, 1)},
+        "kernels_hbm_frac": {"permute_pool_q_k_v": round(
+            acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
         "roofline": {"kernel": "sparse_attn_combine", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
                      "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),
