@@ -39,7 +39,8 @@ sys.path.insert(0, ROOT)
 
 from dataclasses import replace  # noqa: E402
 
-from tile_sparse_video_b200.inputs import VEDA_104K, WORKLOADS, Workload, make_inputs  # noqa: E402
+from tile_sparse_video_b200.inputs import (VEDA_104K, WORKLOADS, Workload, make_inputs,  # noqa: E402
+                                           sweep_workloads)
 
 METRIC = "ms/layer & kept-FLOP TFLOP/s (% bf16 peak) at 104k tokens, 90% tile sparsity"
 UNIT = "ms/layer"
@@ -349,6 +350,80 @@ def backward_timing(w: Workload, plan, dev, stream, inp_dev, k: int, kept_flop: 
     return res
 
 
+def sweep_timing(args) -> None:
+    """The layer step of the benchmark (permute + pool of Q, K, V, coarse +
+    top-k, attention with the fused combine) timed on every sweep workload
+    (the small and reference-to-video shapes at sparsity 0.50 / 0.75 / 0.90 /
+    0.95 and k = 24, several video lengths, B = 2), one JSON line each.  The
+    inputs are drawn on the device from a seeded generator with the workloads'
+    laws (N(0, 1); the reference-to-video family scaled per head by U[0.5, 2];
+    the gate with its marginal law): drawing them on the host as the parity
+    tests do would take minutes per shape, and the timing depends on the
+    values only through the selection they induce."""
+    from tile_sparse_video_b200 import vsa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    steps = max(3, min(args.steps, 10))
+    for w in sweep_workloads():
+        plan = vsa.Plan(w.prefix, w.grid, w.tile, device=0)
+        k = plan.keep_count(keep_ratio=w.keep_ratio, keep_tiles=w.keep_tiles)
+        acct = geometry_counts(w, plan.n_prefix_tiles, plan.n_tiles, k)
+        gen = torch.Generator(device=dev).manual_seed(w.seed_base)
+        shape = (w.B, w.H, plan.n_tokens, w.D)
+        scale = torch.ones(w.B, w.H, 1, 1, device=dev)
+        if w.values == "head_scaled":
+            scale = 0.5 + 1.5 * torch.rand(w.B, w.H, 1, 1, device=dev, generator=gen)
+        q, kk, v = ((torch.randn(shape, device=dev, generator=gen) * scale).to(torch.bfloat16)
+                    for _ in range(3))
+        g = (torch.randn(shape, device=dev, generator=gen) *
+             (w.gate_std * w.gate_width ** 0.5)).to(torch.bfloat16)
+        layer = vsa.Layer(plan, w.B, w.H, w.D, k)
+        slots = vsa.pooled_slots(plan, layer.ws, w.B, w.H, w.D)
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record()
+            for src, dst, pooled in zip((q, kk, v), (layer.q_t, layer.k_t, layer.v_t), slots):
+                vsa.vsa_permute_pool(plan, src, dst, pooled)
+            if ev is not None:
+                ev[1].record()
+            vsa.vsa_coarse_topk_pooled(plan, w.B, w.H, w.D, k, layer.ws, layer.scale,
+                                       o_coarse=layer.o_coarse, topk_idx=layer.topk_idx)
+            if ev is not None:
+                ev[2].record()
+            vsa.vsa_sparse_attn_combine(plan, layer.q_t, layer.k_t, layer.v_t, layer.topk_idx, k, g,
+                                        layer.o_coarse, layer.scale, out=layer.out)
+            if ev is not None:
+                ev[3].record()
+
+        for _ in range(args.warmup):
+            step()
+        vsa.vsa_sync_status(plan)
+        events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            step(events[i])
+        torch.cuda.synchronize()
+        vsa.vsa_sync_status(plan)
+        parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in events]).mean(axis=0)
+        layer_ms = float(parts.sum())
+        attn = acct["kept_flop"] / (parts[2] * 1e-3) / 1e12
+        print(json.dumps({
+            "sweep": w.name, "B": w.B, "H": w.H, "D": w.D, "tokens": w.n_tokens,
+            "tile": "x".join(map(str, w.tile)), "grid": list(w.grid), "sparsity": w.sparsity,
+            "kept_video_tiles": k, "kept_pair_fraction": round(acct["pair_fraction"], 4),
+            "ms_per_layer": round(layer_ms, 4), "steps": steps, "warmup": args.warmup,
+            "kernels_ms": {"permute_pool_q_k_v": round(float(parts[0]), 4),
+                           "coarse_topk": round(float(parts[1]), 4),
+                           "sparse_attn_combine": round(float(parts[2]), 4)},
+            "attn_kept_tflops": round(attn, 2), "attn_frac": round(attn / peaks["bf16"], 4),
+            "dense_equiv_tflops": round(acct["dense_flop"] / (layer_ms * 1e-3) / 1e12, 2),
+            "data": "synthetic (seeded, drawn on the device)"}), flush=True)
+        del layer, slots, q, kk, v, g
+        torch.cuda.empty_cache()
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     from tile_sparse_video_b200 import vsa
     import torch.distributed as dist
@@ -523,6 +598,8 @@ def main():
     ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
                     help="profiling runs only: another named workload")
     ap.add_argument("--heads", type=int, default=0, help="profiling runs only: fewer heads")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the layer on every sweep workload (one GPU; one JSON line each)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", "0"))
@@ -530,6 +607,11 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.sweep:
+        if world > 1:
+            raise SystemExit("--sweep runs on one GPU")
+        sweep_timing(args)
         return
     import torch.distributed as dist
     from datetime import timedelta
