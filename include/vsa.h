@@ -229,9 +229,14 @@ vsa_status vsa_project_tiled(vsa_plan plan, const void* x_t, const void* w, int 
  * VSA_ERR_WORKSPACE, launching nothing, when that exceeds 16 MiB.
  * The first call on a device resolves the array's device address with
  * cudaGetSymbolAddress (once per device, that device current); make that first
- * call before any stream capture.  All calls share the array, which keeps the
- * last call's contents (nothing in it needs to start at zero); calls that
- * overlap on the GPU race on it and must be serialised by the caller. */
+ * call before any stream capture.  The address is cached per device together
+ * with the CUDA context that was current when it was resolved, and resolved
+ * again when a call finds another context current.  cudaDeviceReset
+ * invalidates every device resource the library holds, plans included:
+ * destroy and recreate plans after a reset.  All calls share the array, which
+ * keeps the last call's contents (nothing in it needs to start at zero);
+ * calls that overlap on the GPU race on it and must be serialised by the
+ * caller. */
 vsa_status vsa_coarse_topk_noalloc(vsa_plan plan, const void* q_t, const void* k_t,
                                    const void* v_t, int B, int H, int D, float scale, int k,
                                    float* o_coarse, int32_t* topk_idx, float* topk_score,
@@ -246,8 +251,9 @@ vsa_status vsa_coarse_topk_noalloc(vsa_plan plan, const void* q_t, const void* k
  * [B,H,N_pad,D], pad rows written 0.  lse_t (nullable): fp32 [B,H,N_pad],
  * natural-log log-sum-exp of each live row's scaled scores (0 on pad rows).
  * topk_idx must hold valid, distinct video tile indices (as vsa_coarse_topk
- * writes them); a kernel that meets an index outside [n_p, T) skips it and
- * records VSA_ERR_DEVICE_INDEX.  ws may be NULL. */
+ * writes them).  A kernel that meets an index outside [n_p, T) replaces it
+ * with tile n_p, so the outputs of that query tile are then undefined, and
+ * records VSA_ERR_DEVICE_INDEX for vsa_sync_status.  ws may be NULL. */
 vsa_status vsa_sparse_attn(vsa_plan plan, const void* q_t, const void* k_t, const void* v_t,
                            const int32_t* topk_idx, int B, int H, int D, int k, float scale,
                            void* o_fine_t, float* lse_t, void* ws, size_t ws_bytes,

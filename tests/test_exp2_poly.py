@@ -1,7 +1,9 @@
 """The FMA-pipe exp2 of the attention kernel, checked against its error bound.
 
-The kernel takes one exponential in four off the MUFU unit with its own
-Cody-Waite + degree-3 polynomial.  This test reads the shipped coefficients
+The attention kernel has an optional FMA-pipe exp2 (off by default: the
+VSA_EXP2_FMA_SHARE build knob selects which share of the exponentials it
+takes off the MUFU unit), a Cody-Waite + degree-3 polynomial of its own.  This
+test reads the coefficients
 from the kernel source, replays the same float32 operations in numpy and
 checks the relative error against 2^x over the whole range the softmax feeds
 it (x in [-125, 8]: scores minus a running max, which may lag by up to 8)."""

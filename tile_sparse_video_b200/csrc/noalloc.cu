@@ -12,7 +12,8 @@
 // module holds its kStaticScratchBytes until the process exits.  Host code
 // cannot use the array's name as a device address (it names a host-side
 // stand-in), so the first call on each device, with that device current,
-// resolves the real address with cudaGetSymbolAddress and caches it.  That
+// resolves the real address with cudaGetSymbolAddress and caches it (again
+// when a later call finds another CUDA context current, as after a reset).  That
 // first call on a device therefore does a one-time runtime query; make it
 // before any stream capture.
 //
@@ -20,6 +21,8 @@
 // it needs to start at zero: the pooling kernel overwrites every value it later
 // reads.  Calls whose executions overlap on the GPU (different streams, or
 // different threads) race on the array and must be serialised by the caller.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "vsa_internal.h"
@@ -32,19 +35,42 @@ static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / si
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};   // context current when the address was taken
 
-// Device address of g_static_scratch on `device`, which must be current.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, found through the runtime (the library links
+// no driver stub); nullptr when the driver does not provide it.
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_static_scratch on `device`, which must be current.  The
+// address is cached with the context it was taken in and taken again when
+// another context is current (a reset device gets a new primary context).
 vsa_status static_scratch(int device, void** out) {
   if (device < 0 || device >= kMaxDevices)
     return vsa::fail(VSA_ERR_UNSUPPORTED, "device ordinal beyond the static scratch table");
+  CUcontext ctx = nullptr;
+  if (CtxGetCurrentFn get = ctx_get_current_fn()) get(&ctx);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[device] == nullptr) {
+  if (g_scratch_addr[device] == nullptr || g_scratch_ctx[device] != ctx) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess || p == nullptr)
       return vsa::fail(VSA_ERR_CUDA, std::string("cudaGetSymbolAddress of the static scratch: ") +
                                          cudaGetErrorString(e));
     g_scratch_addr[device] = p;
+    g_scratch_ctx[device] = ctx;
   }
   *out = g_scratch_addr[device];
   return VSA_OK;
