@@ -354,6 +354,18 @@ vsa_status vsa_sparse_attn_backward(vsa_plan plan, const void* q_t, const void* 
  * receives 0 for each wait that gave up.  The context stays usable. */
 vsa_status vsa_check_bounded_wait(vsa_plan plan, int32_t* result, void* stream);
 
+/* Test hook for the attention kernels' failure path (the pages have no
+ * counterpart).  Sets the bound of every mbarrier wait of the kernels that
+ * vsa_sparse_attn, vsa_sparse_attn_combine, vsa_sparse_attn_ref and
+ * vsa_sparse_attn_backward launch from then on, process-wide, in ns of wall
+ * time; 0 (or anything above it) restores the 2 s default.  With a bound of
+ * a few microseconds their waits run out: the kernel records
+ * VSA_ERR_DEVICE_TIMEOUT in the plan's status word, drains its own TMA loads
+ * and MMAs, frees its tensor memory and returns, and the outputs of that
+ * launch are undefined.  Not for production use; not thread safe against
+ * launches running concurrently in other host threads.  Returns VSA_OK. */
+vsa_status vsa_debug_set_wait_limit(uint64_t ns);
+
 /* Synchronise `stream`, then read and clear the plan's device status word.
  * Returns VSA_OK, VSA_ERR_DEVICE_TIMEOUT, VSA_ERR_DEVICE_INDEX or VSA_ERR_CUDA. */
 vsa_status vsa_sync_status(vsa_plan plan, void* stream);

@@ -19,7 +19,7 @@ import pytest
 import torch
 
 import oracle as O
-from tests.parity import f64
+from tests.parity import RECORDS, bf16_floor, f64
 from tile_sparse_video_b200 import vsa
 from tile_sparse_video_b200.inputs import SMALL, TINY, Workload, make_grad_output, make_inputs
 
@@ -55,6 +55,9 @@ def assert_rel(got, want, rel_max=REL_MAX, rel_mean=REL_MEAN, what=""):
     if want.size == 0:
         return
     err = np.abs(got - want)
+    fmx, fmn = bf16_floor(want)
+    from tests import parity
+    RECORDS.append((f"{parity.CURRENT_TEST[0]}: {what}", float(err.max()), float(err.mean()), fmx, fmn))
     scale_max = float(np.abs(want).max())
     scale_mean = float(np.abs(want).mean())
     assert err.max() <= rel_max * scale_max + 1e-30, (

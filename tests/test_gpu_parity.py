@@ -217,6 +217,17 @@ def _sampled(w: Workload, heads, n_video_samples, seed):
     assert n_near <= max(2, w.B * len(heads) * p.n_video_tiles // 50)
 
 
+# the reference-to-video family of the sweep at its shortest clip (24 x 42
+# grid: partial w-cubes; six-segment prefix; B = 2), at 75 % and at k = 24
+REF2VA_SWEEP = [w for w in sweep_workloads()
+                if w.grid[:2] == (16, 24) and (w.name.endswith("_s75_b2") or "_k24_" in w.name)]
+
+
+@pytest.mark.parametrize("w", REF2VA_SWEEP, ids=lambda w: w.name)
+def test_ref2va_sweep_sampled(w):
+    _sampled(w, (0, 29, 41), 12, seed=5)
+
+
 @pytest.mark.parametrize("w,heads,n", [(REF2VA, (0, 17, 41), 24), (VEDA_104K, (0, 23, 41), 16),
                                        (replace(VEDA_104K, name="veda_h56", H=56), (0, 55), 8)],
                          ids=["ref2va_full", "veda_104k_full", "veda_h56_full"])
@@ -280,6 +291,55 @@ def test_bounded_wait_gives_up_and_reports():
     assert 1.5 < elapsed < 30.0, elapsed         # the 2 s bound, not a hang
     vsa.vsa_sync_status(plan)                    # cleared
     _check_layer(w, make_inputs(w))              # the context is still usable
+
+
+@pytest.mark.parametrize("w", [
+    TINY,                                                                  # 64-row tiles (pairs)
+    _w("abort_r128", 1, 2, 128, (256,), (8, 16, 8), (4, 8, 4), keep_tiles=3),
+], ids=lambda w: w.name)
+def test_attention_abort_path(w):
+    """The attention kernels' own failure path, run on the GPU without a
+    fault: with their wait bound cut to 100 ns (vsa_debug_set_wait_limit) the
+    forward kernel's and the backward kernels' waits run out, each records
+    VSA_ERR_DEVICE_TIMEOUT, drains its TMA loads and MMAs, frees its tensor
+    memory and returns well within a second; with the bound restored the same
+    context runs the layer, forward and backward, correctly."""
+    import time
+    inp = make_inputs(w)
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    q, kk, v, g = (inp[x].cuda() for x in "qkvg")
+    train = vsa.TrainingLayer(plan, w.B, w.H, w.D, k)
+    train.forward(q, kk, v, g)
+    d_out = torch.randn(train.out.shape, device="cuda").to(torch.bfloat16)
+    vsa.vsa_sync_status(plan)
+    try:
+        vsa.vsa_debug_set_wait_limit(100)
+        for what in ("forward", "backward"):
+            timed_out = False
+            for _ in range(5):             # a wait that happened to finish in time: try again
+                t0 = time.perf_counter()
+                if what == "forward":
+                    vsa.vsa_sparse_attn(plan, train.q_t, train.k_t, train.v_t, train.topk_idx, k)
+                else:
+                    train.backward(d_out)
+                try:
+                    vsa.vsa_sync_status(plan)
+                except vsa.VsaError as e:
+                    assert e.status == 6, e              # VSA_ERR_DEVICE_TIMEOUT
+                    timed_out = True
+                elapsed = time.perf_counter() - t0
+                assert elapsed < 1.0, (what, elapsed)
+                if timed_out:
+                    break
+            assert timed_out, f"the {what} kernels never gave up under a 100 ns bound"
+    finally:
+        vsa.vsa_debug_set_wait_limit(0)
+    vsa.vsa_sync_status(plan)
+    _check_layer(w, inp)
+    grads = train.backward(d_out)
+    vsa.vsa_sync_status(plan)
+    assert all(torch.isfinite(x.float()).all() for x in grads)
 
 
 def test_empty_batch_is_a_no_op():

@@ -1,15 +1,23 @@
 // libvsa C ABI: argument checks, plan lifetime and dispatch to the kernels.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <new>
 #include <string>
 
+#include "sm100.cuh"
 #include "vsa_internal.h"
 
 namespace vsa {
 
 static thread_local std::string g_last_error;
+
+// Bound of the attention kernels' mbarrier waits (process-wide; a test
+// shortens it through vsa_debug_set_wait_limit to make the abort path run).
+static std::atomic<unsigned long long> g_wait_limit_ns{sm100::kWaitLimitNs};
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(); }
 
 void set_error(const std::string& msg) { g_last_error = msg; }
 
@@ -576,6 +584,14 @@ vsa_status vsa_check_bounded_wait(vsa_plan p, int32_t* result, void* stream) {
   e = launch_bounded_wait_check(p->d_status, reinterpret_cast<int*>(result),
                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "bounded-wait check launch");
+}
+
+vsa_status vsa_debug_set_wait_limit(uint64_t ns) {
+  // 0 restores the default; anything above the default is capped to it
+  const unsigned long long lim =
+      (ns == 0 || ns > sm100::kWaitLimitNs) ? sm100::kWaitLimitNs : (unsigned long long)ns;
+  g_wait_limit_ns.store(lim);
+  return VSA_OK;
 }
 
 vsa_status vsa_sync_status(vsa_plan p, void* stream) {

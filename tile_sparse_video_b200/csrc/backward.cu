@@ -303,6 +303,7 @@ struct BwdArgs {
   uint16_t* out;              // dQ_t (query-major) or dK_t (key-major), bf16 [BH, N_pad, D]
   uint16_t* out2;             // key-major: dV_t
   unsigned int* status;
+  unsigned long long wait_ns; // bound of every mbarrier wait
   unsigned int* next_item;    // work counter (zero at launch)
   int T, n_p, k, k_ref, n_sink, W, n_items;
   int64_t n_pad;
@@ -338,8 +339,9 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // only if all of them saw the phase (so that no lane is left behind at the
 // warp-collective tcgen05 instructions that follow when the CTA aborts).
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* status, unsigned int where) {
-  const bool ok = wait_bar(bar, parity, abort_flag, status, where);
+                                          unsigned int* status, unsigned int where,
+                                          unsigned long long limit_ns) {
+  const bool ok = wait_bar(bar, parity, abort_flag, status, where, limit_ns);
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     bool ok = true;
     for (; ok; ++t) {
       // the previous item's epilogue is done with the accumulators and the list
-      if (t > 0 && !wait_warp(epi_done, (t - 1) & 1, abort_flag, a.status, 40)) { ok = false; break; }
+      if (t > 0 && !wait_warp(epi_done, (t - 1) & 1, abort_flag, a.status, 40, a.wait_ns)) { ok = false; break; }
       int item = 0;
       if (lane == 0) item = int(atomicAdd(a.next_item, 1u));
       item = __shfl_sync(0xFFFFFFFFu, item, 0);
@@ -612,11 +614,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           const int n = u / HS, c = u % HS;
           const uint32_t s = (Gs + n) % NS, w = (G + u) & 1;
           if (u == 0) {
-            if (!wait_bar(x_full, (x_loads - 1) & 1, abort_flag, a.status, 41)) return false;
+            if (!wait_bar(x_full, (x_loads - 1) & 1, abort_flag, a.status, 41, a.wait_ns)) return false;
             x_pending = false;
           }
           if (c == 0) {
-            if (!wait_bar(y_full + 8 * s, ((Gs + n) / NS) & 1, abort_flag, a.status, 42)) return false;
+            if (!wait_bar(y_full + 8 * s, ((Gs + n) / NS) & 1, abort_flag, a.status, 42, a.wait_ns)) return false;
             ++y_seen[s];
           }
           tc_fence_after();
@@ -654,7 +656,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           if (u + 2 < U) {
             // buffer w (and, after a step's last half, its stage) is free once
             // the accumulating products of half-step u (warp kWarpAcc) have read it
-            if (!wait_bar(acc_done + 8 * w, idx & 1, abort_flag, a.status, 44)) { ok = false; break; }
+            if (!wait_bar(acc_done + 8 * w, idx & 1, abort_flag, a.status, 44, a.wait_ns)) { ok = false; break; }
             if (c == HS - 1 && n + NS < cnt) load_y(n + NS);
             if (!issue_sd(u + 2)) { ok = false; break; }
           }
@@ -686,7 +688,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     int t = 0;
     bool ok = true;
     for (; ok; ++t) {
-      if (!wait_warp(list_full, t & 1, abort_flag, a.status, 50)) { ok = false; break; }
+      if (!wait_warp(list_full, t & 1, abort_flag, a.status, 50, a.wait_ns)) { ok = false; break; }
       const int item = *s_item;
       if (item < 0) break;
       const int cnt = *s_cnt;
@@ -696,7 +698,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           const int n = u / HS, c = u % HS;
           const uint32_t s = (Gs + n) % NS, w = (G + u) & 1;
           const uint32_t idx = hw[w]++;
-          if (!wait_bar(p_ready + 8 * w, idx & 1, abort_flag, a.status, 43)) { ok = false; break; }
+          if (!wait_bar(p_ready + 8 * w, idx & 1, abort_flag, a.status, 43, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t y1 = sY + s * 2 * C::YBYTES, y2 = y1 + C::YBYTES;
           const uint32_t buf = tmem + C::COL_BUF + w * 2 * NH;
@@ -751,7 +753,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     int t = 0;
     bool ok = true;
     for (; ok; ++t) {
-      if (!wait_warp(list_full, t & 1, abort_flag, a.status, 45)) { ok = false; break; }
+      if (!wait_warp(list_full, t & 1, abort_flag, a.status, 45, a.wait_ns)) { ok = false; break; }
       const int item = *s_item;
       if (item < 0) break;
       int64_t bh;
@@ -769,9 +771,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       for (int u = int((uint32_t(wg) - G) & 1u); u < U; u += 2) {
         const int n = u / HS, c = u % HS;
         const uint32_t s = (Gs + n) % NS;
-        if (!wait_warp(s_full + 8 * wg, mine & 1, abort_flag, a.status, 46)) { ok = false; break; }
+        if (!wait_warp(s_full + 8 * wg, mine & 1, abort_flag, a.status, 46, a.wait_ns)) { ok = false; break; }
         ++mine;
-        if (kKeyMajor && !wait_warp(y_full + 8 * s, ((Gs + n) / NS) & 1, abort_flag, a.status, 47)) {
+        if (kKeyMajor && !wait_warp(y_full + 8 * s, ((Gs + n) / NS) & 1, abort_flag, a.status, 47, a.wait_ns)) {
           ok = false;
           break;
         }
@@ -809,7 +811,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       Gs += cnt;
       // epilogue: accumulator (x scale for dQ, dK) + pooled gradient / block_len
       if (cnt > 0) {
-        if (!wait_warp(acc_full, accs & 1, abort_flag, a.status, 48)) { ok = false; break; }
+        if (!wait_warp(acc_full, accs & 1, abort_flag, a.status, 48, a.wait_ns)) { ok = false; break; }
         ++accs;
         tc_fence_after();
       }
@@ -1006,6 +1008,7 @@ vsa_status launch_sparse_attn_backward(const vsa_plan_s* p, const void* q_t, con
   a.lse = lse_t;
   a.delta = delta;
   a.status = p->d_status;
+  a.wait_ns = wait_limit_ns();
   a.T = p->n_tiles;
   a.n_p = p->n_prefix_tiles;
   a.k = k;

@@ -170,6 +170,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       VSA_I8(0), VSA_I8(8), VSA_I8(16), VSA_I8(24)
       : "memory");
 }
+// One fp32 column of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -191,15 +195,18 @@ __device__ __forceinline__ void record(unsigned int* status, unsigned int code, 
 // cycles per wait on B200 even when the phase had long completed).  The timer
 // and the abort flag are looked at every 16 polls; mbarrier.try_wait itself
 // suspends the thread for a while when the phase is not complete.
+// limit_ns: the bound (the launch's wait limit; kWaitLimitNs unless a test
+// shortened it to make the abort path run).
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned int* status, unsigned int where) {
+                                         unsigned int* status, unsigned int where,
+                                         unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         record(status, kStatusTimeout, where);
         return false;

@@ -38,13 +38,23 @@
 //                    goes to TMEM as bf16 pairs.  The epilogue adds the two
 //                    warpgroups' row sums and stores bf16 rows (and the LSE), or
 //                    the gated combine in natural order.
-// TMEM columns: O [0,D), S_w [D + w*R, D + (w+1)*R), P_w [D + 2R + w*R/2,
-// D + 2R + (w+1)*R/2) (two bf16 per 32-bit column, key order, row = lane).
+// TMEM columns: O [0,D), S_w [D + w*128, D + (w+1)*128), P_w [D + 256 + w*64,
+// D + 256 + (w+1)*64) (two bf16 per 32-bit column, key order, row = lane).
 // S_{n+2} depends only on S_n having been read, P_n only on PV_{n-2}, so MMA
 // latency stays off the softmax's path, and no P tile takes shared memory.
-// With R = 64 the MMA still runs with M = 128 (rows 64..127 of the Q box are
-// the next rows of the tensor, or zero past its end); their results are never
-// stored and the warps of those rows skip the softmax work.
+//
+// 64-row tiles (VSA 4x4x4 cubes) run in pairs, so that every MMA keeps its
+// 128 x 128 shape: an item is a pair of consecutive query tiles (2m, 2m+1) of
+// one head (MMA rows 0-63 and 64-127; their 128 rows are contiguous in the
+// tiled layout, so one Q box loads both), and a step is a pair of key tiles
+// taken in ascending order from the union of the two query tiles' key sets.
+// Each entry of that list carries a mask of the query tiles whose set holds
+// it; the softmax warps of the other query tile treat its keys as masked, and
+// warps whose query tile holds neither key tile of a step write P = 0 without
+// exponentials.  A key tile both query tiles kept is loaded once for both.
+// The list is built per item by the K producer warp (two bitmaps over the T
+// tiles, then a ballot compaction) into one of two shared-memory slots that
+// the other roles read.
 //
 // Every mbarrier wait is bounded (kWaitLimitNs of wall time); on expiry the
 // CTA raises an abort flag, records VSA_ERR_DEVICE_TIMEOUT in the status word,
@@ -216,12 +226,13 @@ struct AttnArgs {
   uint16_t* out;              // bf16 [BH, N_pad, D], or [BH, N, D] natural when fused
   float* lse;                 // [BH, N_pad] or null
   unsigned int* status;       // device status word
+  unsigned long long wait_ns; // bound of every mbarrier wait (kWaitLimitNs unless shortened)
   // fused gated combine (step 5) in the epilogue: out[row_src[r]] =
   // o_fine[r] + sigmoid(gate[row_src[r]]) * o_coarse[tile(r)]
   const uint16_t* gate;       // bf16 [BH, N, D] natural order, or null (unfused)
   const float* o_coarse;      // fp32 [BH, T, D]
   const int32_t* row_src;     // [N_pad] padded row -> token, -1 for a pad row
-  int T, n_p, k, n_items;
+  int T, n_p, k, n_items, BH;
   int64_t n_pad, n_tok;
   float scale_log2;           // scale * log2(e)
   // reference thinning: the kept reference tiles of each video query tile
@@ -240,11 +251,13 @@ __device__ __forceinline__ float sigmoid_fast(float g) {
 
 template <int R, int D>
 struct Cfg {
-  static constexpr int BN = R;
-  static constexpr int NSK = (R == 128) ? VSA_NSK128 : 4;   // K ring stages
-  static constexpr int NSV = (R == 128) ? VSA_NSV128 : 4;   // V ring stages
+  // 64-row tiles run in pairs: two query tiles per item, two key tiles per step
+  static constexpr bool kPair = (R == 64);
+  static constexpr int BN = 128;                         // key rows per step
+  static constexpr int NSK = VSA_NSK128;                 // K ring stages
+  static constexpr int NSV = VSA_NSV128;                 // V ring stages
   static constexpr int QBYTES = kBM * D * 2;
-  static constexpr int TBYTES = BN * D * 2;              // one K (or V) tile
+  static constexpr int TBYTES = BN * D * 2;              // one step's K (or V) rows
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_V = OFF_K + NSK * TBYTES;
@@ -254,8 +267,8 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_X + (2 + 4) * 128 * 4;
   // barriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV],
   //           s_full[2], s_empty[2], p_full[2], pv_done[2], dec[4], o_full, o_empty,
-  //           drain, drain2
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 4;
+  //           drain, drain2, list_full[2], list_empty[2] (paired tiles)
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 4 + (kPair ? 4 : 0);
   static constexpr int TAIL = NBAR * 8 + 16;              // barriers + tmem slot + abort flag
   // TMEM columns: O [0, D), S_w [D + w*BN, D + (w+1)*BN), P_w (bf16 pairs)
   // [D + 2*BN + w*BN/2, D + 2*BN + (w+1)*BN/2)
@@ -266,12 +279,42 @@ struct Cfg {
   static_assert(D + 3 * BN <= 512, "TMEM columns");
   static constexpr uint32_t IDESC_QK = idesc_bf16(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16(kBM, D, false, true);
-  // bytes: tiles, exchanges, barriers/misc, then the lists (blen uint8[T],
-  // two int32[k] kept-tile lists)
+  // bytes: tiles, exchanges, barriers/misc, then the lists: blen uint8[T] and
+  // two int32[k] kept-tile lists; paired tiles: the two list lengths, two
+  // bitmaps of ceil(T/32) words and two list slots of list_cap(T) entries
+  __host__ __device__ static int list_cap(int T) { return (T + 3) & ~3; }
+  __host__ __device__ static int bitmap_words(int T) { return (T + 31) >> 5; }
   static size_t bytes(int T, int k) {
+    if (kPair)
+      return size_t(OFF_BAR) + TAIL + 16 + size_t(8) * ((bitmap_words(T) + 3) & ~3) +
+             size_t(8) * list_cap(T);
     return size_t(OFF_BAR) + TAIL + size_t((T + 15) & ~15) + size_t(8) * ((k + 3) & ~3);
   }
 };
+
+// List entry of the paired kernel: key tile index | mask << 16 (bit h: query
+// tile 2m+h holds it) | (block_len - 1) << 18.
+constexpr uint32_t kEntryTile = 0xFFFFu;
+__device__ __forceinline__ int entry_tile(uint32_t e) { return int(e & kEntryTile); }
+__device__ __forceinline__ bool entry_has(uint32_t e, int half) { return (e >> (16 + half)) & 1u; }
+__device__ __forceinline__ int entry_blen(uint32_t e) { return int((e >> 18) & 63u) + 1; }
+
+// Pair item -> (b*h, pair m): the pairs made of video tiles only first, head
+// by head, then the pairs that hold a prefix tile (dense, T key tiles long),
+// as decode_item orders single tiles.
+__device__ __forceinline__ void decode_pair(int item, int BH, int n_pp, int n_pairs, int64_t& bh,
+                                            int& m) {
+  const int nvp = n_pairs - n_pp;
+  const int first = BH * nvp;
+  if (item < first) {
+    bh = item / nvp;
+    m = n_pp + item % nvp;
+  } else {
+    const int v = item - first;
+    bh = v / n_pp;
+    m = v % n_pp;
+  }
+}
 
 // Work item -> (b*h, query tile i).  kItemOrder 0: every head's prefix query
 // tiles first, then the video query tiles head by head; 1: the video tiles
@@ -376,7 +419,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
       const int64_t row0 = bh * a.n_pad;
       if (kIsK) {
         VSA_TR(8, 1, g);
-        if (t > 0) ok = wait_bar(q_empty, (t - 1) & 1, abort_flag, a.status, 1);
+        if (t > 0) ok = wait_bar(q_empty, (t - 1) & 1, abort_flag, a.status, 1, a.wait_ns);
         if (ok) {
           ++q_issued;
           mbar_expect_tx(q_full, C::QBYTES);
@@ -393,7 +436,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
         const uint32_t s = g % NS;
         VSA_TL(kIsK ? 3 : 4, 'x', g);
         if (g >= uint32_t(NS)) {
-          ok = wait_bar(empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, kIsK ? 2 : 11);
+          ok = wait_bar(empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, kIsK ? 2 : 11, a.wait_ns);
           if (!ok) break;
         }
         VSA_TL(kIsK ? 3 : 4, kIsK ? 'K' : 'V', g);
@@ -430,6 +473,155 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
   }
 }
 
+// Union key list of pair m of head bh (whole warp): bit j of bitmap h is set
+// when query tile 2m+h attends to key tile j (every tile for a dense prefix
+// query tile; its reference tiles and kept video tiles otherwise; none when
+// 2m+h = T); the list holds every j with a bit set, ascending, as packed
+// entries.  Returns its length.  Out-of-range kept indices are clamped and
+// recorded as by kept_tile / sink_tile.
+template <bool kRef>
+__device__ int build_pair_list(const AttnArgs& a, int64_t bh, int m, uint32_t* bm, uint32_t* list,
+                               int lane) {
+  const int T = a.T, W = (T + 31) >> 5;
+  for (int h = 0; h < 2; ++h) {
+    const int i = 2 * m + h;
+    uint32_t* b = bm + h * W;
+    const bool dense = i < a.n_p;
+    for (int w = lane; w < W; w += 32) {
+      const int rem = T - 32 * w;
+      b[w] = !dense ? 0u : (rem >= 32 ? 0xFFFFFFFFu : ((1u << rem) - 1u));
+    }
+    __syncwarp();
+    if (!dense && i < T) {
+      const int ns = n_sink<kRef>(a);
+      for (int x = lane; x < ns + a.k; x += 32) {
+        const int j = x < ns ? (kRef ? sink_tile(a, bh, i, x) : x) : kept_tile(a, bh, i, x - ns);
+        atomicOr(b + (j >> 5), 1u << (j & 31));
+      }
+    }
+    __syncwarp();
+  }
+  int count = 0;
+  for (int w = 0; w < W; ++w) {
+    const uint32_t w0 = bm[w], w1 = bm[W + w];
+    const uint32_t mask = ((w0 >> lane) & 1u) | (((w1 >> lane) & 1u) << 1);
+    const uint32_t ball = __ballot_sync(0xFFFFFFFFu, mask != 0u);
+    if (mask != 0u) {
+      const int j = 32 * w + lane;              // < T: no bit past T is ever set
+      list[count + __popc(ball & ((1u << lane) - 1u))] =
+          uint32_t(j) | (mask << 16) | (uint32_t(__ldg(a.block_len + j) - 1) << 18);
+    }
+    count += __popc(ball);
+  }
+  if (lane == 0 && (count & 1)) list[count] = 0u;   // an odd list's last step: no tile b
+  __syncwarp();
+  return count;
+}
+
+// Producers of the paired kernel (64-row tiles).  The K warp builds each
+// item's union list into list slot t & 1 (after every reader has released
+// the slot's previous item) and publishes it; the V warp waits for it.  Lane
+// 0 then loads, per step, key tiles 2n and 2n+1 of the list into one ring slot
+// (rows 0-63 and 64-127 of each 64-column box); the second tile of an
+// odd-length list's last step is read from the rows before the tensor, which
+// load as zeros.  The K warp also loads the item's 128 query rows (tiles 2m,
+// 2m+1).  Both release the list slot once their loads are issued.
+template <int D, int NS, bool kIsK, bool kRef>
+__device__ __forceinline__ void producer_pair(const AttnArgs& a, const CUtensorMap* tm_q,
+                                              const CUtensorMap* tm_t, uint32_t sQ, uint32_t sT,
+                                              uint32_t full, uint32_t empty, uint32_t q_full,
+                                              uint32_t q_empty, uint32_t list_full,
+                                              uint32_t list_empty, uint32_t* lists, int* counts,
+                                              uint32_t* bm, int cap, volatile int* abort_flag,
+                                              int lane) {
+  using C = Cfg<64, D>;
+  const int n_pairs = (a.T + 1) >> 1, n_pp = (a.n_p + 1) >> 1;
+  uint32_t g = 0, q_issued = 0;
+  int t = 0;
+  bool ok = true;
+  for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+    int64_t bh;
+    int m;
+    decode_pair(item, a.BH, n_pp, n_pairs, bh, m);
+    const int slot = t & 1;
+    uint32_t* list = lists + slot * cap;
+    int count;
+    if (kIsK) {
+      if (t >= 2)
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(list_empty + 8 * slot, ((t >> 1) - 1) & 1, abort_flag,
+                                              a.status, 22, a.wait_ns));
+      if (!ok) break;
+      count = build_pair_list<kRef>(a, bh, m, bm, list, lane);
+      if (lane == 0) {
+        counts[slot] = count;
+        mbar_arrive(list_full + 8 * slot);
+      }
+      __syncwarp();
+    } else {
+      ok = __all_sync(0xFFFFFFFFu,
+                      wait_bar(list_full + 8 * slot, (t >> 1) & 1, abort_flag, a.status, 23, a.wait_ns));
+      if (!ok) break;
+      count = counts[slot];
+    }
+    const int nk = (count + 1) >> 1;
+    if (lane == 0) {
+      const int64_t row0 = bh * a.n_pad;
+      if (kIsK) {
+        if (t > 0) ok = wait_bar(q_empty, (t - 1) & 1, abort_flag, a.status, 1, a.wait_ns);
+        if (ok) {
+          ++q_issued;
+          mbar_expect_tx(q_full, C::QBYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d_hint(sQ + c * kBM * 128, tm_q, q_full, c * 64, int(row0 + int64_t(m) * 128),
+                             l2_evict_first_policy());
+        }
+      }
+      for (int n = 0; n < nk && ok; ++n, ++g) {
+        const uint32_t s = g % NS;
+        if (g >= uint32_t(NS)) {
+          ok = wait_bar(empty + 8 * s, ((g / NS) - 1) & 1, abort_flag, a.status, kIsK ? 2 : 11, a.wait_ns);
+          if (!ok) break;
+        }
+        const int row_a = int(row0 + int64_t(entry_tile(list[2 * n])) * 64);
+        const int row_b =
+            2 * n + 1 < count ? int(row0 + int64_t(entry_tile(list[2 * n + 1])) * 64) : -64;
+        mbar_expect_tx(full + 8 * s, C::TBYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          const uint32_t dst = sT + s * C::TBYTES + c * C::BN * 128;
+          tma_load_2d(dst, tm_t, full + 8 * s, c * 64, row_a);
+          tma_load_2d(dst + 64 * 128, tm_t, full + 8 * s, c * 64, row_b);
+        }
+      }
+    }
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(list_empty + 8 * slot);
+  }
+  if (lane == 0 && !ok) {
+    // Abort: make sure none of our TMA writes is still in flight.
+    for (uint32_t x = (g > uint32_t(NS) ? g - NS : 0); x < g; ++x)
+      wait_bar_drain(full + 8 * (x % NS), (x / NS) & 1);
+    if (kIsK && q_issued > 0) wait_bar_drain(q_full, (q_issued - 1) & 1);
+  }
+}
+
+// Score columns of the key rows past block_len of a partial 64-row key tile
+// (tile a: columns [0, 64), tile b: [64, 128) of the S row at taddr) set to
+// -inf in TMEM, so that the row max and the exponentials need no mask.  A
+// call, not inline code: partial tiles are rare and the softmax's common
+// path stays as compact as it is without them.  Whole warp, warp-uniform
+// arguments.
+__device__ __noinline__ void mask_partial_tiles(uint32_t taddr, int bla, int blb) {
+  const uint32_t ninf = __float_as_uint(-INFINITY);
+  if (bla > 0)
+    for (int col = bla; col < 64; ++col) tmem_st1(taddr + col, ninf);
+  if (blb > 0)
+    for (int col = blb; col < 64; ++col) tmem_st1(taddr + 64 + col, ninf);
+  tmem_wait_st();
+}
+
 template <int R, int D, bool kRef>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -452,9 +644,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   // phase whose predecessor is already complete and whose successor cannot
   // complete before the waiter has observed it, so the parity test never
   // aliases.
+  // Paired tiles: list_full[slot] completes once per item that uses the list
+  // slot (the K warp published its list), list_empty[slot] once every reader
+  // has released it (K and V warps, the two issuers, the eight softmax warps).
   const uint32_t s_full = v_empty + 8 * NSV, s_empty = s_full + 16, p_full = s_empty + 16,
                  pv_done = p_full + 16, dec = pv_done + 16, o_full = dec + 32,
-                 o_empty = o_full + 8, drain = o_empty + 8, drain2 = drain + 8;
+                 o_empty = o_full + 8, drain = o_empty + 8, drain2 = drain + 8,
+                 list_full = drain2 + 8, list_empty = list_full + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + C::NBAR * 8 + 4);
   float* mbox = reinterpret_cast<float*>(smem + C::OFF_X);       // [2][128]
@@ -463,10 +659,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* s_blen = smem + C::OFF_BAR + C::TAIL;                  // [T]
   int32_t* s_klist = reinterpret_cast<int32_t*>(s_blen + ((a.T + 15) & ~15));
   int32_t* s_vlist = s_klist + ((a.k + 3) & ~3);
+  // paired tiles: list lengths [2], bitmaps [2][W], list slots [2][cap]
+  int* p_counts = reinterpret_cast<int*>(smem + C::OFF_BAR + C::TAIL);
+  uint32_t* p_bm = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::TAIL + 16);
+  const int p_cap = C::list_cap(a.T);
+  uint32_t* p_lists = p_bm + 2 * ((C::bitmap_words(a.T) + 3) & ~3);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_v = a.T - a.n_p;
-  const int BH = a.n_items / a.T;
+  const int BH = a.n_items / (C::kPair ? (a.T + 1) >> 1 : a.T);
+  const int n_pairs = (a.T + 1) >> 1, n_pp = (a.n_p + 1) >> 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -490,6 +692,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
     mbar_init(drain2, 1);
+    if constexpr (C::kPair) {
+      for (int sl = 0; sl < 2; ++sl) {
+        mbar_init(list_full + 8 * sl, 1);
+        mbar_init(list_empty + 8 * sl, 12);
+      }
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -512,11 +720,21 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   if (threadIdx.x == 0) VSA_TR(10, 21, tmem);
 
   if (warp == kWarpTmaK) {
-    producer<R, D, NSK, true, kRef>(a, &tm_q, &tm_k, &tm_v, sQ, sK, k_full, k_empty, q_full, q_empty,
-                              s_klist, abort_flag, lane, BH, n_v);
+    if constexpr (C::kPair)
+      producer_pair<D, NSK, true, kRef>(a, &tm_q, &tm_k, sQ, sK, k_full, k_empty, q_full, q_empty,
+                                        list_full, list_empty, p_lists, p_counts, p_bm, p_cap,
+                                        abort_flag, lane);
+    else
+      producer<R, D, NSK, true, kRef>(a, &tm_q, &tm_k, &tm_v, sQ, sK, k_full, k_empty, q_full,
+                                      q_empty, s_klist, abort_flag, lane, BH, n_v);
   } else if (warp == kWarpTmaV) {
-    producer<R, D, NSV, false, kRef>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full, q_empty,
-                               s_vlist, abort_flag, lane, BH, n_v);
+    if constexpr (C::kPair)
+      producer_pair<D, NSV, false, kRef>(a, &tm_q, &tm_v, sQ, sV, v_full, v_empty, q_full, q_empty,
+                                         list_full, list_empty, p_lists, p_counts, p_bm, p_cap,
+                                         abort_flag, lane);
+    else
+      producer<R, D, NSV, false, kRef>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full,
+                                       q_empty, s_vlist, abort_flag, lane, BH, n_v);
   } else if (warp == kWarpMmaS) {
     // ------------------------------------------------------------ S issuer
     // S_n = Q K_n^T into S_w (w = n & 1) as soon as K_n is in and warpgroup w
@@ -529,20 +747,30 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       int t = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
-        int64_t bh;
-        int i;
-        decode_item(item, BH, a.n_p, n_v, bh, i);
-        const int nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
-        if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5)) { ok = false; break; }
+        int nk;
+        if constexpr (C::kPair) {
+          if (!wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag, a.status, 24, a.wait_ns)) {
+            ok = false;
+            break;
+          }
+          nk = (p_counts[t & 1] + 1) >> 1;
+          mbar_arrive(list_empty + 8 * (t & 1));
+        } else {
+          int64_t bh;
+          int i;
+          decode_item(item, BH, a.n_p, n_v, bh, i);
+          nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
+        }
+        if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5, a.wait_ns)) { ok = false; break; }
         for (int n = 0; n < nk; ++n) {
           const int w = n & 1;
           if (si[w] > 0 &&
-              !wait_bar(s_empty + 8 * w, (si[w] - 1) & 1, abort_flag, a.status, 7)) {
+              !wait_bar(s_empty + 8 * w, (si[w] - 1) & 1, abort_flag, a.status, 7, a.wait_ns)) {
             ok = false;
             break;
           }
           const uint32_t s = gk % NSK;
-          if (!wait_bar(k_full + 8 * s, (gk / NSK) & 1, abort_flag, a.status, 6)) { ok = false; break; }
+          if (!wait_bar(k_full + 8 * s, (gk / NSK) & 1, abort_flag, a.status, 6, a.wait_ns)) { ok = false; break; }
           VSA_TL(0, 'S', g + n);
           tc_fence_after();
 #pragma unroll
@@ -579,20 +807,30 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       int t = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
-        int64_t bh;
-        int i;
-        decode_item(item, BH, a.n_p, n_v, bh, i);
-        const int nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
-        for (int n = 0; n < nk; ++n) {
-          const int w = n & 1;
-          if (n == 0 && t > 0 && !wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3)) {
+        int nk;
+        if constexpr (C::kPair) {
+          if (!wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag, a.status, 25, a.wait_ns)) {
             ok = false;
             break;
           }
-          if (!wait_bar(p_full + 8 * w, pf[w] & 1, abort_flag, a.status, 4)) { ok = false; break; }
+          nk = (p_counts[t & 1] + 1) >> 1;
+          mbar_arrive(list_empty + 8 * (t & 1));
+        } else {
+          int64_t bh;
+          int i;
+          decode_item(item, BH, a.n_p, n_v, bh, i);
+          nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
+        }
+        for (int n = 0; n < nk; ++n) {
+          const int w = n & 1;
+          if (n == 0 && t > 0 && !wait_bar(o_empty, (t - 1) & 1, abort_flag, a.status, 3, a.wait_ns)) {
+            ok = false;
+            break;
+          }
+          if (!wait_bar(p_full + 8 * w, pf[w] & 1, abort_flag, a.status, 4, a.wait_ns)) { ok = false; break; }
           ++pf[w];
           const uint32_t sv = gv % NSV;
-          if (!wait_bar(v_full + 8 * sv, (gv / NSV) & 1, abort_flag, a.status, 12)) {
+          if (!wait_bar(v_full + 8 * sv, (gv / NSV) & 1, abort_flag, a.status, 12, a.wait_ns)) {
             ok = false;
             break;
           }
@@ -617,172 +855,162 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warpgroups
-    // Warpgroup wg takes the tiles n = wg (mod 2) of an item; both add into
-    // one O, scaled by one reference max m_ref per row.  m_ref after tile n is
-    // decided by the warp that runs tile n from m_ref after tile n-1 (read
-    // from the mailbox its partner warp on the same TMEM lanes wrote) and its
-    // own row max, and published in turn; it moves only when a row grew by
-    // more than 2^8 (exact: p <= 256), and then that warp rescales its O rows
-    // once PV_{n-1} is complete.
-    VSA_TL_DECL;
-    const int wg = warp >> 2;                            // 0 or 1
-    const int quad = warp & 3;
-    const bool rows_active = (R == 128) || (quad < 2);
-    const int row = quad * 32 + lane;                    // = TMEM lane
-    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
-    const uint32_t col_s = C::COL_S + wg * BN;
-    const uint32_t col_p = C::COL_P + wg * (BN / 2);
-    const uint32_t dbar = dec + 8 * quad;
-    uint32_t G = 0;              // global index of the item's first tile
-    uint32_t cnt[2] = {0, 0};    // tiles of each warpgroup in earlier items
-    uint32_t cw = 0;             // tiles processed by this warpgroup
-    int t = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
-      int64_t bh;
-      int i;
-      decode_item(item, BH, a.n_p, n_v, bh, i);
-      const bool dense = i < a.n_p;
-      const int nk = dense ? a.T : n_sink<kRef>(a) + a.k;
-      // Group barrier of the 256 softmax threads around the per-item list.  A
-      // warp that sees the abort flag leaves instead: the others then also see
-      // it before they could block here (they wait on the same mbarrier phases
-      // first).
-      if (*abort_flag) { ok = false; break; }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      for (int x = threadIdx.x; x < nk; x += 256) {
-        const int j = step_tile_global<kRef>(a, bh, i, dense, x);
-        s_blen[x] = uint8_t(__ldg(a.block_len + j) - 1);
-      }
-      if (*abort_flag) { ok = false; break; }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const int q_live = __ldg(a.block_len + i);
-
-      float m_mine = -INFINITY, l = 0.f;   // l: this warpgroup's row sum, relative to m_mine
-      for (int n = wg; n < nk; n += 2, ++cw) {
-        const uint32_t Gn = G + n;
-        if (lane == 0) VSA_TR(quad + 4 * wg, 13, Gn);
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'a', Gn);
-        ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * wg, cw & 1, abort_flag, a.status, 8));
+    if constexpr (C::kPair) {
+      // Paired 64-row tiles.  Warps 0-1 and 4-5 hold the rows of query tile
+      // 2m (half 0), warps 2-3 and 6-7 those of tile 2m+1 (half 1).  A step's
+      // S tile spans key tiles a = entry 2n and b = entry 2n+1 of the item's
+      // list (columns [0, 64) and [64, 128)); a key tile outside this half's
+      // set counts as fully masked.  The protocol is the one of the 128-row
+      // kernel below (one O, a reference max shared through the mailbox,
+      // lazy rescale).  Key tiles outside the set skip their exponentials and
+      // write P = 0.
+      VSA_TL_DECL;
+      const int wg = warp >> 2;                            // 0 or 1
+      const int quad = warp & 3;
+      const int half = quad >> 1;
+      const int row = quad * 32 + lane;                    // = TMEM lane
+      const int row_t = row - 64 * half;                   // row within the query tile
+      const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
+      const uint32_t col_s = C::COL_S + wg * BN;
+      const uint32_t col_p = C::COL_P + wg * (BN / 2);
+      const uint32_t dbar = dec + 8 * quad;
+      const uint32_t s_lists =
+          s_base + C::OFF_BAR + C::TAIL + 16 + 8 * ((C::bitmap_words(a.T) + 3) & ~3);
+      uint32_t G = 0;              // global index of the item's first step
+      uint32_t cnt[2] = {0, 0};    // steps of each warpgroup in earlier items
+      uint32_t cw = 0;             // steps processed by this warpgroup
+      int t = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+        int64_t bh;
+        int m;
+        decode_pair(item, BH, n_pp, n_pairs, bh, m);
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag,
+                                              a.status, 26, a.wait_ns));
         if (!ok) break;
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 's', Gn);
-        tc_fence_after();
-        uint32_t r[BN / 32][32];
-        if (rows_active) {
+        int count;
+        asm volatile("ld.shared.u32 %0, [%1];"
+                     : "=r"(count)
+                     : "r"(s_base + C::OFF_BAR + C::TAIL + 4 * (t & 1)));
+        const int nk = (count + 1) >> 1;
+        const uint32_t plist = s_lists + 4 * (t & 1) * C::list_cap(a.T);
+        const int i = 2 * m + half;                         // this warp's query tile
+        const bool rows_active = i < a.T;                   // warp-uniform
+        const int q_live = rows_active ? __ldg(a.block_len + i) : 0;
+
+        float m_mine = -INFINITY, l = 0.f;   // l: this warpgroup's row sum, relative to m_mine
+        for (int n = wg; n < nk; n += 2, ++cw) {
+          const uint32_t Gn = G + n;
+          ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * wg, cw & 1, abort_flag, a.status, 8, a.wait_ns));
+          if (!ok) break;
+          tc_fence_after();
+          // block_len of key tiles a and b for this half, 0 when outside its set
+          // (an odd list ends with a zero entry)
+          uint32_t ea, eb;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(ea), "=r"(eb) : "r"(plist + 8 * n));
+          const int bl2[2] = {entry_has(ea, half) ? entry_blen(ea) : 0,
+                              entry_has(eb, half) ? entry_blen(eb) : 0};
+          // S row into registers, then S is released at once so that S_{n+2}
+          // can be issued during this step's exponentials
+          // key rows past block_len of a partial key tile (rare): their score
+          // columns are overwritten with -inf in TMEM, one column per store, so
+          // that the row max and the exponentials below need no mask
+          if (((bl2[0] | bl2[1]) & 63) != 0) mask_partial_tiles(t_lane + col_s, bl2[0], bl2[1]);
+          uint32_t r[4][32];
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + col_s + 32 * c, r[c]);
+          for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + col_s + 32 * c, r[c]);
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) tmem_wait_ld(r[c]);
-        }
-        tc_fence_before();
-        mbar_arrive(s_empty + 8 * wg);
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'l', Gn);
-        // row max over raw scores (scale > 0 commutes with max), four chains
-        float mx = -INFINITY;
-        if (rows_active) {
-          const int bl = int(s_blen[n]) + 1;
-          if (bl < BN) {
+          for (int c = 0; c < 4; ++c) tmem_wait_ld(r[c]);
+          tc_fence_before();
+          mbar_arrive(s_empty + 8 * wg);
+          // row max over raw scores (scale > 0 commutes with max), four chains;
+          // a key tile outside this half's set is left out
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c)
+          for (int c2 = 0; c2 < 2; ++c2) {
+            if (bl2[c2] == 0) continue;                     // warp-uniform
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (32 * c + e >= bl) r[c][e] = __float_as_uint(-INFINITY);
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int e = 0; e < 32; e += 2)
+                mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(r[2 * c2 + h][e]),
+                                          __uint_as_float(r[2 * c2 + h][e + 1]));
           }
-          float mx4[4];
+          const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
+          // m_ref after step n-1 (the previous global step's decision; an
+          // item's first step starts from -inf), then this step's decision
+          float m_prev = -INFINITY;
+          if (Gn > 0) {
+            ok = __all_sync(0xFFFFFFFFu, wait_bar(dbar, (Gn - 1) & 1, abort_flag, a.status, 14, a.wait_ns));
+            if (!ok) break;
+            if (n > 0) m_prev = mbox[((Gn - 1) & 1) * 128 + row];
+          }
+          const float m_cand = fmaxf(m_prev, mx * a.scale_log2);
+          const bool rescale = __any_sync(0xFFFFFFFFu, m_cand > m_prev + 8.0f);
+          const float m_new = rescale ? m_cand : m_prev;
+          if (m_new != -INFINITY) {
+            // this warpgroup's row sum follows the reference max (-inf only
+            // while no key of the item has reached these rows)
+            l *= ex2(m_mine - m_new);
+            m_mine = m_new;
+          }
+          // P_w is free once this warpgroup's previous PV is complete
+          if (cw > 0) {
+            ok = __all_sync(0xFFFFFFFFu,
+                            wait_bar(pv_done + 8 * wg, (cw - 1) & 1, abort_flag, a.status, 9, a.wait_ns));
+            if (!ok) break;
+          }
+          tc_fence_after();
+          bool published = false;            // warp-uniform
+          {
+            const float m_use = m_new == -INFINITY ? 0.f : m_new;
+            const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(-m_use, -m_use);
+            uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) mx4[q] = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; e += 2)
-              mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(r[c][e]),
-                                        __uint_as_float(r[c][e + 1]));
-          mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
-        }
-        // m_ref after tile n-1 (the previous global tile's decision; an item's
-        // first tile starts from -inf), then this tile's decision
-        float m_prev = -INFINITY;
-        if (Gn > 0) {
-          ok = __all_sync(0xFFFFFFFFu, wait_bar(dbar, (Gn - 1) & 1, abort_flag, a.status, 14));
-          if (!ok) break;
-          if (n > 0) m_prev = mbox[((Gn - 1) & 1) * 128 + row];
-        }
-        const float m_cand = fmaxf(m_prev, mx * a.scale_log2);
-        // warp-uniform (the O rescale below uses warp-collective TMEM access)
-        const bool rescale = __any_sync(0xFFFFFFFFu, m_cand > m_prev + 8.0f);
-        const float m_new = rescale ? m_cand : m_prev;
-        bool published = false;            // warp-uniform
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'm', Gn);
-        if (rows_active) {
-          // this warpgroup's row sum follows the reference max
-          l *= ex2(m_mine - m_new);
-          m_mine = m_new;
-        }
-        // P_w is free once this warpgroup's previous PV is complete
-        if (cw > 0) {
-          ok = __all_sync(0xFFFFFFFFu,
-                          wait_bar(pv_done + 8 * wg, (cw - 1) & 1, abort_flag, a.status, 9));
-          if (!ok) break;
-        }
-        tc_fence_after();
-        if (rows_active) {
-          // exponentials on pairs: packed scale-and-subtract, two exp2, packed
-          // row sums, P packed to bf16 and stored to P_w every 64 scores.  One
-          // exponential in kExp2FmaShare runs on the FMA pipe.
-          const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(-m_new, -m_new);
-          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-          for (int c2 = 0; c2 < BN / 64; ++c2) {
-            uint32_t pw[32];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int c = 2 * c2 + h;
-              if (kPubChunk > 0 && kPubChunk < BN / 32 && c == kPubChunk) {
+            for (int c2 = 0; c2 < 2; ++c2) {
+              if (c2 == 1 && kPubChunk > 0 && kPubChunk < 4) {
                 mbox[(Gn & 1) * 128 + row] = m_new;
                 mbar_arrive(dbar);
                 published = true;
               }
+              uint32_t pw[32];
+              if (bl2[c2] == 0) {
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                float x0, x1;
-                f2unpack(ffma2(f2pack(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), sc2,
-                               nm2),
-                         x0, x1);
-                const bool fma0 = kExp2FmaShare > 0 && e % kExp2FmaShare == kExp2FmaShare - 1;
-                const bool fma1 = kExp2FmaShare > 0 && (e + 1) % kExp2FmaShare == kExp2FmaShare - 1;
-                const float p0 = fma0 ? exp2_fma(x0) : ex2(x0);
-                const float p1 = fma1 ? exp2_fma(x1) : ex2(x1);
-                acc2[(e >> 1) & 3] = fadd2(acc2[(e >> 1) & 3], f2pack(p0, p1));
-                pw[16 * h + (e >> 1)] = pack_bf16(p0, p1);
+                for (int e = 0; e < 32; ++e) pw[e] = 0u;
+              } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                  for (int e = 0; e < 32; e += 2) {
+                    float x0, x1;
+                    f2unpack(ffma2(f2pack(__uint_as_float(r[2 * c2 + h][e]),
+                                          __uint_as_float(r[2 * c2 + h][e + 1])),
+                                   sc2, nm2),
+                             x0, x1);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    acc2[(e >> 1) & 1] = fadd2(acc2[(e >> 1) & 1], f2pack(p0, p1));
+                    pw[16 * h + (e >> 1)] = pack_bf16(p0, p1);
+                  }
               }
+              tmem_st32(t_lane + col_p + 32 * c2, pw);
             }
-            tmem_st32(t_lane + col_p + 32 * c2, pw);
+            float s0, s1;
+            f2unpack(fadd2(acc2[0], acc2[1]), s0, s1);
+            l += s0 + s1;
           }
-          float s0, s1, s2, s3;
-          f2unpack(fadd2(acc2[0], acc2[1]), s0, s1);
-          f2unpack(fadd2(acc2[2], acc2[3]), s2, s3);
-          l += (s0 + s1) + (s2 + s3);
-        }
-        // Publish the decision only now: the partner warp, which shares this
-        // warp's SM sub-partition and its MUFU unit, cannot start its own
-        // exponentials before ours are done, so the two warps take turns on
-        // the MUFU and each does its loads, max and stores during the
-        // other's exponentials.
-        if (!published) {
-          mbox[(Gn & 1) * 128 + row] = m_new;
-          mbar_arrive(dbar);
-        }
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'w', Gn);
-        // O rescale when the reference max moved: O holds PV_0..PV_{n-1}
-        // relative to m_prev; PV_{n-1} (the partner's tile) must be complete,
-        // and PV_n is not issued before the p_full arrival below.
-        if (rescale && n > 0) {
-          const uint32_t idx = cnt[1 - wg] + uint32_t((n - 1) >> 1);
-          ok = __all_sync(0xFFFFFFFFu,
-                          wait_bar(pv_done + 8 * (1 - wg), idx & 1, abort_flag, a.status, 15));
-          if (!ok) break;
-          tc_fence_after();
-          if (rows_active) {
+          if (!published) {
+            mbox[(Gn & 1) * 128 + row] = m_new;
+            mbar_arrive(dbar);
+          }
+          // O rescale when the reference max moved: O holds PV_0..PV_{n-1}
+          // relative to m_prev; PV_{n-1} (the partner's step) must be complete,
+          // and PV_n is not issued before the p_full arrival below.
+          if (rescale && n > 0) {
+            const uint32_t idx = cnt[1 - wg] + uint32_t((n - 1) >> 1);
+            ok = __all_sync(0xFFFFFFFFu,
+                            wait_bar(pv_done + 8 * (1 - wg), idx & 1, abort_flag, a.status, 15, a.wait_ns));
+            if (!ok) break;
+            tc_fence_after();
             const float alpha = ex2(m_prev - m_new);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -794,89 +1022,340 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
               tmem_st32(t_lane + C::COL_O + 32 * c, o);
             }
           }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_full + 8 * wg);
         }
-        if (rows_active) tmem_wait_st();
+        if (!ok) break;
+        // ---- epilogue (as in the 128-row kernel), per query tile of the pair
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(o_full, t & 1, abort_flag, a.status, 10, a.wait_ns));
+        if (!ok) break;
+        cnt[0] += uint32_t((nk + 1) / 2);
+        cnt[1] += uint32_t(nk / 2);
+        tc_fence_after();
+        x_m[wg * 128 + row] = m_mine;
+        x_l[wg * 128 + row] = l;
+        if (*abort_flag) { ok = false; break; }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (rows_active) {
+          const float m0 = x_m[row], m1 = x_m[128 + row];
+          const float l0 = x_l[row], l1 = x_l[128 + row];
+          const float mm = fmaxf(m0, m1);
+          const float lt = (l0 > 0.f ? l0 * ex2(m0 - mm) : 0.f) + (l1 > 0.f ? l1 * ex2(m1 - mm) : 0.f);
+          const bool live = row_t < q_live;
+          const float inv = live ? 1.0f / lt : 0.f;
+          const bool fused = a.gate != nullptr;
+          const int64_t tok =
+              (fused && live) ? int64_t(__ldg(a.row_src + int64_t(i) * R + row_t)) : 0;
+          uint16_t* orow = fused ? a.out + (bh * a.n_tok + tok) * D + wg * (D / 2)
+                                 : a.out + (bh * a.n_pad + int64_t(i) * R + row_t) * D + wg * (D / 2);
+          const uint16_t* grow = fused ? a.gate + (bh * a.n_tok + tok) * D + wg * (D / 2) : nullptr;
+          const float* ocrow = fused ? a.o_coarse + (bh * a.T + i) * D + wg * (D / 2) : nullptr;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_lane + C::COL_O + wg * (D / 2) + 32 * c, o);
+            tmem_wait_ld(o);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[8 * q + e]) * inv;
+              if (fused) {
+                if (!live) continue;                  // pad rows have no natural token
+                const uint4 gv = __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
+                const float4 c0v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q));
+                const float4 c1v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q + 4));
+                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                const float cv[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  v[2 * e] = fmaf(sigmoid_fast(__uint_as_float(gw[e] << 16)), cv[2 * e], v[2 * e]);
+                  v[2 * e + 1] = fmaf(sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u)),
+                                      cv[2 * e + 1], v[2 * e + 1]);
+                }
+              }
+              uint4 u;
+              u.x = pack_bf16(v[0], v[1]);
+              u.y = pack_bf16(v[2], v[3]);
+              u.z = pack_bf16(v[4], v[5]);
+              u.w = pack_bf16(v[6], v[7]);
+              dst[q] = u;
+            }
+          }
+          if (a.lse != nullptr && wg == 0)
+            a.lse[bh * a.n_pad + int64_t(i) * R + row_t] =
+                live ? (mm + __log2f(lt)) * 0.69314718055994531f : 0.f;
+        }
         tc_fence_before();
-        mbar_arrive(p_full + 8 * wg);
-        if (lane == 0) VSA_TR(quad + 4 * wg, 16, Gn);
-        if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'W', Gn);
+        mbar_arrive(o_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(list_empty + 8 * (t & 1));   // this warp is done with the list
+        G += nk;
       }
-      if (!ok) break;
-      // ---- epilogue: once every PV of the item is complete (o_full), add the
-      // two row sums (each relative to its warpgroup's last reference max; O
-      // is relative to the larger) and store O / l (warpgroup wg: columns
-      // [wg*D/2, (wg+1)*D/2)), fused with the gated combine when a gate is given.
-      const uint32_t g_last = G + nk - 1;
-      (void)g_last;
-      if (lane == 0) VSA_TR(quad + 4 * wg, 17, g_last);
-      ok = __all_sync(0xFFFFFFFFu, wait_bar(o_full, t & 1, abort_flag, a.status, 10));
-      if (!ok) break;
-      cnt[0] += uint32_t((nk + 1) / 2);
-      cnt[1] += uint32_t(nk / 2);
-      tc_fence_after();
-      x_m[wg * 128 + row] = m_mine;
-      x_l[wg * 128 + row] = l;
-      if (*abort_flag) { ok = false; break; }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (rows_active) {
-        const float m0 = x_m[row], m1 = x_m[128 + row];
-        const float l0 = x_l[row], l1 = x_l[128 + row];
-        const float mm = fmaxf(m0, m1);
-        const float lt = (l0 > 0.f ? l0 * ex2(m0 - mm) : 0.f) + (l1 > 0.f ? l1 * ex2(m1 - mm) : 0.f);
-        const bool live = row < q_live;
-        const float inv = live ? 1.0f / lt : 0.f;
-        const bool fused = a.gate != nullptr;
-        const int64_t tok = (fused && live) ? int64_t(__ldg(a.row_src + int64_t(i) * R + row)) : 0;
-        uint16_t* orow = fused ? a.out + (bh * a.n_tok + tok) * D + wg * (D / 2)
-                               : a.out + (bh * a.n_pad + int64_t(i) * R + row) * D + wg * (D / 2);
-        const uint16_t* grow = fused ? a.gate + (bh * a.n_tok + tok) * D + wg * (D / 2) : nullptr;
-        const float* ocrow = fused ? a.o_coarse + (bh * a.T + i) * D + wg * (D / 2) : nullptr;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_lane + C::COL_O + wg * (D / 2) + 32 * c, o);
-          tmem_wait_ld(o);
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[8 * q + e]) * inv;
-            if (fused) {
-              if (!live) continue;                  // pad rows have no natural token
-              const uint4 gv =
-                  VSA_STREAM_IO ? __ldcs(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q))
-                                : __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
-              const float4 c0v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q));
-              const float4 c1v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q + 4));
-              const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-              const float cv[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                v[2 * e] = fmaf(sigmoid_fast(__uint_as_float(gw[e] << 16)), cv[2 * e], v[2 * e]);
-                v[2 * e + 1] =
-                    fmaf(sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u)), cv[2 * e + 1], v[2 * e + 1]);
+    } else {
+      // Warpgroup wg takes the tiles n = wg (mod 2) of an item; both add into
+      // one O, scaled by one reference max m_ref per row.  m_ref after tile n is
+      // decided by the warp that runs tile n from m_ref after tile n-1 (read
+      // from the mailbox its partner warp on the same TMEM lanes wrote) and its
+      // own row max, and published in turn; it moves only when a row grew by
+      // more than 2^8 (exact: p <= 256), and then that warp rescales its O rows
+      // once PV_{n-1} is complete.
+      VSA_TL_DECL;
+      const int wg = warp >> 2;                            // 0 or 1
+      const int quad = warp & 3;
+      const bool rows_active = (R == 128) || (quad < 2);
+      const int row = quad * 32 + lane;                    // = TMEM lane
+      const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
+      const uint32_t col_s = C::COL_S + wg * BN;
+      const uint32_t col_p = C::COL_P + wg * (BN / 2);
+      const uint32_t dbar = dec + 8 * quad;
+      uint32_t G = 0;              // global index of the item's first tile
+      uint32_t cnt[2] = {0, 0};    // tiles of each warpgroup in earlier items
+      uint32_t cw = 0;             // tiles processed by this warpgroup
+      int t = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+        int64_t bh;
+        int i;
+        decode_item(item, BH, a.n_p, n_v, bh, i);
+        const bool dense = i < a.n_p;
+        const int nk = dense ? a.T : n_sink<kRef>(a) + a.k;
+        // Group barrier of the 256 softmax threads around the per-item list.  A
+        // warp that sees the abort flag leaves instead: the others then also see
+        // it before they could block here (they wait on the same mbarrier phases
+        // first).
+        if (*abort_flag) { ok = false; break; }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        for (int x = threadIdx.x; x < nk; x += 256) {
+          const int j = step_tile_global<kRef>(a, bh, i, dense, x);
+          s_blen[x] = uint8_t(__ldg(a.block_len + j) - 1);
+        }
+        if (*abort_flag) { ok = false; break; }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        const int q_live = __ldg(a.block_len + i);
+
+        float m_mine = -INFINITY, l = 0.f;   // l: this warpgroup's row sum, relative to m_mine
+        for (int n = wg; n < nk; n += 2, ++cw) {
+          const uint32_t Gn = G + n;
+          if (lane == 0) VSA_TR(quad + 4 * wg, 13, Gn);
+          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'a', Gn);
+          ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * wg, cw & 1, abort_flag, a.status, 8, a.wait_ns));
+          if (!ok) break;
+          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 's', Gn);
+          tc_fence_after();
+          uint32_t r[BN / 32][32];
+          if (rows_active) {
+  #pragma unroll
+            for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + col_s + 32 * c, r[c]);
+  #pragma unroll
+            for (int c = 0; c < BN / 32; ++c) tmem_wait_ld(r[c]);
+          }
+          tc_fence_before();
+          mbar_arrive(s_empty + 8 * wg);
+          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'l', Gn);
+          // row max over raw scores (scale > 0 commutes with max), four chains
+          float mx = -INFINITY;
+          if (rows_active) {
+            const int bl = int(s_blen[n]) + 1;
+            if (bl < BN) {
+  #pragma unroll
+              for (int c = 0; c < BN / 32; ++c)
+  #pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (32 * c + e >= bl) r[c][e] = __float_as_uint(-INFINITY);
+            }
+            float mx4[4];
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) mx4[q] = -INFINITY;
+  #pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+  #pragma unroll
+              for (int e = 0; e < 32; e += 2)
+                mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(r[c][e]),
+                                          __uint_as_float(r[c][e + 1]));
+            mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
+          }
+          // m_ref after tile n-1 (the previous global tile's decision; an item's
+          // first tile starts from -inf), then this tile's decision
+          float m_prev = -INFINITY;
+          if (Gn > 0) {
+            ok = __all_sync(0xFFFFFFFFu, wait_bar(dbar, (Gn - 1) & 1, abort_flag, a.status, 14, a.wait_ns));
+            if (!ok) break;
+            if (n > 0) m_prev = mbox[((Gn - 1) & 1) * 128 + row];
+          }
+          const float m_cand = fmaxf(m_prev, mx * a.scale_log2);
+          // warp-uniform (the O rescale below uses warp-collective TMEM access)
+          const bool rescale = __any_sync(0xFFFFFFFFu, m_cand > m_prev + 8.0f);
+          const float m_new = rescale ? m_cand : m_prev;
+          bool published = false;            // warp-uniform
+          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'm', Gn);
+          if (rows_active) {
+            // this warpgroup's row sum follows the reference max
+            l *= ex2(m_mine - m_new);
+            m_mine = m_new;
+          }
+          // P_w is free once this warpgroup's previous PV is complete
+          if (cw > 0) {
+            ok = __all_sync(0xFFFFFFFFu,
+                            wait_bar(pv_done + 8 * wg, (cw - 1) & 1, abort_flag, a.status, 9, a.wait_ns));
+            if (!ok) break;
+          }
+          tc_fence_after();
+          if (rows_active) {
+            // exponentials on pairs: packed scale-and-subtract, two exp2, packed
+            // row sums, P packed to bf16 and stored to P_w every 64 scores.  One
+            // exponential in kExp2FmaShare runs on the FMA pipe.
+            const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(-m_new, -m_new);
+            uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+  #pragma unroll
+            for (int c2 = 0; c2 < BN / 64; ++c2) {
+              uint32_t pw[32];
+  #pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int c = 2 * c2 + h;
+                if (kPubChunk > 0 && kPubChunk < BN / 32 && c == kPubChunk) {
+                  mbox[(Gn & 1) * 128 + row] = m_new;
+                  mbar_arrive(dbar);
+                  published = true;
+                }
+  #pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                  float x0, x1;
+                  f2unpack(ffma2(f2pack(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), sc2,
+                                 nm2),
+                           x0, x1);
+                  const bool fma0 = kExp2FmaShare > 0 && e % kExp2FmaShare == kExp2FmaShare - 1;
+                  const bool fma1 = kExp2FmaShare > 0 && (e + 1) % kExp2FmaShare == kExp2FmaShare - 1;
+                  const float p0 = fma0 ? exp2_fma(x0) : ex2(x0);
+                  const float p1 = fma1 ? exp2_fma(x1) : ex2(x1);
+                  acc2[(e >> 1) & 3] = fadd2(acc2[(e >> 1) & 3], f2pack(p0, p1));
+                  pw[16 * h + (e >> 1)] = pack_bf16(p0, p1);
+                }
+              }
+              tmem_st32(t_lane + col_p + 32 * c2, pw);
+            }
+            float s0, s1, s2, s3;
+            f2unpack(fadd2(acc2[0], acc2[1]), s0, s1);
+            f2unpack(fadd2(acc2[2], acc2[3]), s2, s3);
+            l += (s0 + s1) + (s2 + s3);
+          }
+          // Publish the decision only now: the partner warp, which shares this
+          // warp's SM sub-partition and its MUFU unit, cannot start its own
+          // exponentials before ours are done, so the two warps take turns on
+          // the MUFU and each does its loads, max and stores during the
+          // other's exponentials.
+          if (!published) {
+            mbox[(Gn & 1) * 128 + row] = m_new;
+            mbar_arrive(dbar);
+          }
+          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'w', Gn);
+          // O rescale when the reference max moved: O holds PV_0..PV_{n-1}
+          // relative to m_prev; PV_{n-1} (the partner's tile) must be complete,
+          // and PV_n is not issued before the p_full arrival below.
+          if (rescale && n > 0) {
+            const uint32_t idx = cnt[1 - wg] + uint32_t((n - 1) >> 1);
+            ok = __all_sync(0xFFFFFFFFu,
+                            wait_bar(pv_done + 8 * (1 - wg), idx & 1, abort_flag, a.status, 15, a.wait_ns));
+            if (!ok) break;
+            tc_fence_after();
+            if (rows_active) {
+              const float alpha = ex2(m_prev - m_new);
+  #pragma unroll
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(t_lane + C::COL_O + 32 * c, o);
+                tmem_wait_ld(o);
+  #pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st32(t_lane + C::COL_O + 32 * c, o);
               }
             }
-            uint4 u;
-            u.x = pack_bf16(v[0], v[1]);
-            u.y = pack_bf16(v[2], v[3]);
-            u.z = pack_bf16(v[4], v[5]);
-            u.w = pack_bf16(v[6], v[7]);
-            if (VSA_STREAM_IO)
-              __stcs(dst + q, u);
-            else
-              dst[q] = u;
           }
+          if (rows_active) tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_full + 8 * wg);
+          if (lane == 0) VSA_TR(quad + 4 * wg, 16, Gn);
+          if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 'W', Gn);
         }
-        if (a.lse != nullptr && wg == 0)
-          a.lse[bh * a.n_pad + int64_t(i) * R + row] =
-              live ? (mm + __log2f(lt)) * 0.69314718055994531f : 0.f;
+        if (!ok) break;
+        // ---- epilogue: once every PV of the item is complete (o_full), add the
+        // two row sums (each relative to its warpgroup's last reference max; O
+        // is relative to the larger) and store O / l (warpgroup wg: columns
+        // [wg*D/2, (wg+1)*D/2)), fused with the gated combine when a gate is given.
+        const uint32_t g_last = G + nk - 1;
+        (void)g_last;
+        if (lane == 0) VSA_TR(quad + 4 * wg, 17, g_last);
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(o_full, t & 1, abort_flag, a.status, 10, a.wait_ns));
+        if (!ok) break;
+        cnt[0] += uint32_t((nk + 1) / 2);
+        cnt[1] += uint32_t(nk / 2);
+        tc_fence_after();
+        x_m[wg * 128 + row] = m_mine;
+        x_l[wg * 128 + row] = l;
+        if (*abort_flag) { ok = false; break; }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (rows_active) {
+          const float m0 = x_m[row], m1 = x_m[128 + row];
+          const float l0 = x_l[row], l1 = x_l[128 + row];
+          const float mm = fmaxf(m0, m1);
+          const float lt = (l0 > 0.f ? l0 * ex2(m0 - mm) : 0.f) + (l1 > 0.f ? l1 * ex2(m1 - mm) : 0.f);
+          const bool live = row < q_live;
+          const float inv = live ? 1.0f / lt : 0.f;
+          const bool fused = a.gate != nullptr;
+          const int64_t tok = (fused && live) ? int64_t(__ldg(a.row_src + int64_t(i) * R + row)) : 0;
+          uint16_t* orow = fused ? a.out + (bh * a.n_tok + tok) * D + wg * (D / 2)
+                                 : a.out + (bh * a.n_pad + int64_t(i) * R + row) * D + wg * (D / 2);
+          const uint16_t* grow = fused ? a.gate + (bh * a.n_tok + tok) * D + wg * (D / 2) : nullptr;
+          const float* ocrow = fused ? a.o_coarse + (bh * a.T + i) * D + wg * (D / 2) : nullptr;
+  #pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_lane + C::COL_O + wg * (D / 2) + 32 * c, o);
+            tmem_wait_ld(o);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float v[8];
+  #pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[8 * q + e]) * inv;
+              if (fused) {
+                if (!live) continue;                  // pad rows have no natural token
+                const uint4 gv =
+                    VSA_STREAM_IO ? __ldcs(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q))
+                                  : __ldg(reinterpret_cast<const uint4*>(grow + 32 * c + 8 * q));
+                const float4 c0v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q));
+                const float4 c1v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q + 4));
+                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                const float cv[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+  #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  v[2 * e] = fmaf(sigmoid_fast(__uint_as_float(gw[e] << 16)), cv[2 * e], v[2 * e]);
+                  v[2 * e + 1] =
+                      fmaf(sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u)), cv[2 * e + 1], v[2 * e + 1]);
+                }
+              }
+              uint4 u;
+              u.x = pack_bf16(v[0], v[1]);
+              u.y = pack_bf16(v[2], v[3]);
+              u.z = pack_bf16(v[4], v[5]);
+              u.w = pack_bf16(v[6], v[7]);
+              if (VSA_STREAM_IO)
+                __stcs(dst + q, u);
+              else
+                dst[q] = u;
+            }
+          }
+          if (a.lse != nullptr && wg == 0)
+            a.lse[bh * a.n_pad + int64_t(i) * R + row] =
+                live ? (mm + __log2f(lt)) * 0.69314718055994531f : 0.f;
+        }
+        tc_fence_before();
+        mbar_arrive(o_empty);
+        if (lane == 0) VSA_TR(quad + 4 * wg, 18, g_last);
+        G += nk;
       }
-      tc_fence_before();
-      mbar_arrive(o_empty);
-      if (lane == 0) VSA_TR(quad + 4 * wg, 18, g_last);
-      G += nk;
     }
   }
 
@@ -934,6 +1413,7 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   a.n_tok = p->n_tokens;
   a.lse = lse_t;
   a.status = p->d_status;
+  a.wait_ns = wait_limit_ns();
   a.T = p->n_tiles;
   a.n_p = p->n_prefix_tiles;
   a.k = k;
@@ -943,9 +1423,11 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   a.n_sink = thin ? k_ref : p->n_prefix_tiles;
   a.n_pad = p->n_padded;
   a.scale_log2 = scale * 1.4426950408889634f;
-  const int64_t items = bh * p->n_tiles;
+  // 64-row tiles: one item per pair of consecutive query tiles
+  const int64_t items = bh * (Cfg<R, D>::kPair ? (p->n_tiles + 1) / 2 : p->n_tiles);
   if (items >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "too many work items");
   a.n_items = int(items);
+  a.BH = int(bh);
   const int grid = int(std::min<int64_t>(items, p->num_sms > 0 ? p->num_sms : 148));
   kernel<<<grid, kThreadsAttn, smem, stream>>>(mq, mk, mv, a);
   e = cudaGetLastError();

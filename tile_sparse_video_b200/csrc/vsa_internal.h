@@ -30,6 +30,10 @@ struct vsa_plan_s {
 
 namespace vsa {
 
+// Bound of the attention kernels' mbarrier waits, in ns (2 s unless a test
+// shortened it through vsa_debug_set_wait_limit).
+unsigned long long wait_limit_ns();
+
 // Thread-local last error message.
 void set_error(const std::string& msg);
 vsa_status fail(vsa_status code, const std::string& msg);

@@ -86,6 +86,7 @@ def lib():
             "vsa_sparse_attn_backward": [P, V, V, V, V, V, I, V, I, V, V, V, V, V, I, I, I, F,
                                          V, V, V, V, Z, V],
             "vsa_check_bounded_wait": [P, V, V],
+            "vsa_debug_set_wait_limit": [ctypes.c_uint64],
             "vsa_sync_status": [P, V],
         }
         for name, args in sig.items():
@@ -464,6 +465,12 @@ def vsa_sparse_attn_ref(plan: Plan, q_t, k_t, v_t, topk_idx, k: int, topk_ref, k
                                      _ptr(o_coarse) if fused else None, _ptr(out), _ptr(lse),
                                      _stream(stream)))
     return out, lse
+
+
+def vsa_debug_set_wait_limit(ns: int) -> None:
+    """Bound of the attention kernels' mbarrier waits from now on, in ns
+    (0: the 2 s default).  A test hook for the kernels' abort path."""
+    _check(lib().vsa_debug_set_wait_limit(int(ns)))
 
 
 def vsa_sync_status(plan: Plan, stream=None):
