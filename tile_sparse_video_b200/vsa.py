@@ -32,7 +32,7 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_coun
            "vsa_keep_count_ref", "vsa_select_reference",
            "vsa_sparse_attn_ref", "vsa_backward_workspace_size", "vsa_combine_backward",
            "vsa_coarse_backward", "vsa_sparse_attn_backward", "vsa_check_bounded_wait",
-           "vsa_sync_status", "vsa_last_error")
+           "vsa_debug_set_wait_limit", "vsa_sync_status", "vsa_last_error")
 
 
 class VsaError(RuntimeError):
