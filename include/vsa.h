@@ -105,9 +105,12 @@ vsa_status vsa_keep_count(vsa_plan plan, double keep_ratio, int32_t keep_tiles, 
 
 vsa_status vsa_plan_destroy(vsa_plan plan);
 
-/* Bytes of device workspace vsa_coarse_topk needs for B, H, D, k (the pooled
- * means; vsa_sparse_attn needs none and accepts ws = NULL).  Layout (fp32):
- * qbar at offset 0, kbar at B*H*T*D*4, vbar at 2*B*H*T*D*4, each [B,H,T,D]. */
+/* Bytes of device workspace vsa_coarse_topk needs for B, H, D, k
+ * (vsa_sparse_attn needs none and accepts ws = NULL).  Layout (fp32): the
+ * pooled means, qbar at offset 0, kbar at B*H*T*D*4, vbar at 2*B*H*T*D*4, each
+ * [B,H,T,D]; then, at 3*B*H*T*D*4, the coarse kernel's score rows (32 rows of
+ * ceil4(T) floats for each of its 2 x (SM count) persistent CTAs), which hold
+ * nothing on return. */
 vsa_status vsa_workspace_size(vsa_plan plan, int B, int H, int D, int k, size_t* bytes);
 
 /* Step 1 (device).  x_t[b,h,untile[n],:] = x[b,h,n,:]; pad rows are written 0.

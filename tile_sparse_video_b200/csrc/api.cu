@@ -178,7 +178,9 @@ vsa_status vsa_workspace_size(vsa_plan p, int B, int H, int D, int k, size_t* by
   if (B < 0 || H < 0) return fail(VSA_ERR_INVALID_ARG, "B and H must be >= 0");
   if (D != 64 && D != 128) return fail(VSA_ERR_UNSUPPORTED, "head dim D must be 64 or 128");
   (void)k;
-  *bytes = size_t(3) * size_t(B) * size_t(H) * size_t(p->n_tiles) * size_t(D) * sizeof(float);
+  // the pooled means, then the coarse kernel's score rows
+  *bytes = size_t(3) * size_t(B) * size_t(H) * size_t(p->n_tiles) * size_t(D) * sizeof(float) +
+           coarse_scratch_bytes(p->n_tiles, p->num_sms);
   return VSA_OK;
 }
 
@@ -238,8 +240,9 @@ vsa_status vsa_coarse_topk(vsa_plan p, const void* q_t, const void* k_t, const v
                               static_cast<const uint16_t*>(v_t), p->d_block_len, qbar, kbar, vbar,
                               bh, p->n_tiles, p->R, D, p->num_sms, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+  float* scratch = qbar + size_t(3) * bh * p->n_tiles * D;
   e = launch_coarse_topk(qbar, kbar, vbar, bh, p->n_tiles, p->n_prefix_tiles, D, scale, k,
-                         o_coarse, topk_idx, topk_score, s);
+                         o_coarse, topk_idx, topk_score, scratch, p->num_sms, s);
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "coarse_topk launch");
 }
 
@@ -282,8 +285,9 @@ vsa_status vsa_coarse_topk_pooled(vsa_plan p, int B, int H, int D, float scale, 
   const float* qbar = static_cast<const float*>(ws);
   const float* kbar = qbar + bh * p->n_tiles * D;
   const float* vbar = kbar + bh * p->n_tiles * D;
+  float* scratch = const_cast<float*>(qbar) + size_t(3) * bh * p->n_tiles * D;
   cudaError_t e = launch_coarse_topk(qbar, kbar, vbar, bh, p->n_tiles, p->n_prefix_tiles, D, scale,
-                                     k, o_coarse, topk_idx, topk_score,
+                                     k, o_coarse, topk_idx, topk_score, scratch, p->num_sms,
                                      static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "coarse_topk launch");
 }

@@ -17,6 +17,8 @@
 //   3. softmax and o_coarse = sum_j p[r][j] vbar_j: the scores become
 //      probabilities in place, value tiles are staged 64 at a time, lane l
 //      accumulates columns l, l+32, ... for the warp's RW rows.
+#include <algorithm>
+
 #include "vsa_internal.h"
 
 namespace vsa {
@@ -114,284 +116,304 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Persistent CTAs (two per SM); an item is (b*h, block of QB = NW*RW query
+// tiles).  The QB score rows of an item live in this CTA's slot of a global
+// scratch area (QB x Tpad fp32, read back from L2), so that QB no longer
+// depends on T: every warp keeps RW = 4 query rows in registers against the
+// keys it streams from shared memory.
 template <int D, int NW, int RW>
-__global__ void __launch_bounds__(NW * 32) coarse_topk_kernel(
+__global__ void __launch_bounds__(NW * 32, 2) coarse_topk_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ vbar,
-    int T, int n_p, float scale, int k, float* __restrict__ o_coarse, int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_score) {
+    int64_t n_bh, int T, int n_p, float scale, int k, float* __restrict__ o_coarse,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_score, float* __restrict__ scratch) {
   constexpr int kWarps = NW;
   constexpr int QB = kWarps * RW;
   constexpr int kStride = D + 4;
   extern __shared__ float4 smem4[];
   float* smem = reinterpret_cast<float*>(smem4);
-  float* qT = smem;                                   // [D][QB]
+  float* qT = smem;                                   // [D][QB]; phase 3: P chunk [QB][kKC]
   float* stage0 = qT + D * QB;                        // [2][kKC][kStride]
   uint32_t* hist = reinterpret_cast<uint32_t*>(stage0 + 2 * kKC * kStride);  // [kWarps][256]
-  float* sc = reinterpret_cast<float*>(hist + kWarps * 256);            // [QB][Tpad]
   const int Tpad = (T + 3) & ~3;
+  float* sc = scratch + int64_t(blockIdx.x) * QB * Tpad;   // this CTA's score rows [QB][Tpad]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t bh = blockIdx.y;
-  const int i0 = blockIdx.x * QB;
-  const float* kb = kbar + bh * int64_t(T) * D;
-  const float* vb = vbar + bh * int64_t(T) * D;
-
-  {
-    // transposed query block: qT[d][r]; batched loads as in stage_rows
-    constexpr int kNVec = QB * D / 4;
-    constexpr int kVec = (kNVec + kWarps * 32 - 1) / (kWarps * 32);
-    const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * T + i0) * D);
-    float4 v[kVec];
-#pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-      const int idx = threadIdx.x + u * kWarps * 32;
-      v[u] = (idx < kNVec && i0 + idx / (D / 4) < T) ? __ldg(q4 + idx)
-                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-      const int idx = threadIdx.x + u * kWarps * 32;
-      if (idx >= kNVec) continue;
-      const int r = idx / (D / 4), d = (idx % (D / 4)) * 4;
-      qT[(d + 0) * QB + r] = v[u].x;
-      qT[(d + 1) * QB + r] = v[u].y;
-      qT[(d + 2) * QB + r] = v[u].z;
-      qT[(d + 3) * QB + r] = v[u].w;
-    }
-  }
-
-  // ---- 1. scores (double-buffered key stages)
+  const int n_blk = (T + QB - 1) / QB;
   const int n_chunks = (T + kKC - 1) / kKC;
-  stage_rows_async<D, NW>(stage0, kb, min(kKC, T));
-  for (int c = 0; c < n_chunks; ++c) {
-    const int j0 = c * kKC;
-    const int nj = min(kKC, T - j0);
-    float* stage = stage0 + (c & 1) * kKC * kStride;
-    if (c + 1 < n_chunks) {
-      stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, kb + int64_t(j0 + kKC) * D,
-                          min(kKC, T - j0 - kKC));
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  const int n_v = T - n_p;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  for (int64_t item = blockIdx.x; item < n_bh * n_blk; item += gridDim.x) {
+    const int64_t bh = item / n_blk;
+    const int i0 = int(item % n_blk) * QB;
+    const float* kb = kbar + bh * int64_t(T) * D;
+    const float* vb = vbar + bh * int64_t(T) * D;
+    __syncthreads();     // the previous item is done with qT and the stages
+
+    {
+      // transposed query block: qT[d][r] (rows past T are zero)
+      constexpr int kNVec = QB * D / 4;
+      constexpr int kVec = (kNVec + kWarps * 32 - 1) / (kWarps * 32);
+      const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * T + i0) * D);
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int idx = threadIdx.x + u * kWarps * 32;
+        if (idx >= kNVec) continue;
+        const float4 v = i0 + idx / (D / 4) < T ? __ldg(q4 + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int r = idx / (D / 4), d = (idx % (D / 4)) * 4;
+        qT[(d + 0) * QB + r] = v.x;
+        qT[(d + 1) * QB + r] = v.y;
+        qT[(d + 2) * QB + r] = v.z;
+        qT[(d + 3) * QB + r] = v.w;
+      }
     }
-    __syncthreads();
-    constexpr int KPL = kKC / 32;                  // keys per lane: lane, lane + 32, ...
-    float acc[RW][KPL];
+
+    // ---- 1. scores (double-buffered key stages), written to the scratch rows
+    stage_rows_async<D, NW>(stage0, kb, min(kKC, T));
+    for (int c = 0; c < n_chunks; ++c) {
+      const int j0 = c * kKC;
+      const int nj = min(kKC, T - j0);
+      float* stage = stage0 + (c & 1) * kKC * kStride;
+      if (c + 1 < n_chunks) {
+        stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, kb + int64_t(j0 + kKC) * D,
+                                min(kKC, T - j0 - kKC));
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      constexpr int KPL = kKC / 32;                  // keys per lane: lane, lane + 32, ...
+      float acc[RW][KPL];
+#pragma unroll
+      for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int u = 0; u < KPL; ++u) acc[r][u] = 0.f;
+      const float* qw = qT + warp * RW;
+#pragma unroll 4
+      for (int d4 = 0; d4 < D / 4; ++d4) {
+        float av[KPL][4];
+#pragma unroll
+        for (int u = 0; u < KPL; ++u) {
+          const float4 a = reinterpret_cast<const float4*>(stage + (lane + 32 * u) * kStride)[d4];
+          av[u][0] = a.x;
+          av[u][1] = a.y;
+          av[u][2] = a.z;
+          av[u][3] = a.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float q[RW];
+          QVec<RW>::load(qw + (4 * d4 + e) * QB, q);
+#pragma unroll
+          for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int u = 0; u < KPL; ++u) acc[r][u] = fmaf(q[r], av[u][e], acc[r][u]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        float* row = sc + (warp * RW + r) * Tpad + j0;
+#pragma unroll
+        for (int u = 0; u < KPL; ++u)
+          if (lane + 32 * u < nj) row[lane + 32 * u] = scale * acc[r][u];
+      }
+      __syncthreads();     // stage (c & 1) is refilled two chunks later
+    }
+
+    // ---- 2. per row of this warp: the scores copied from the scratch row
+    // into a shared-memory row buffer of the warp (in the key stages, free
+    // now) when they fit, then the top-k over the video key tiles (video
+    // query tiles only) and the softmax, whose P goes back to the scratch row
+    uint32_t* h = hist + warp * 256;
+    const bool row_in_smem = size_t(kWarps) * Tpad <= size_t(2) * kKC * kStride;
+    float inv_l[RW];
+    for (int r = 0; r < RW; ++r) {
+      const int i = i0 + warp * RW + r;
+      float* srow = sc + (warp * RW + r) * Tpad;                 // global
+      float* s = row_in_smem ? stage0 + warp * Tpad : srow;     // where the passes read
+      if (row_in_smem) {
+        for (int j4 = lane; j4 < Tpad / 4; j4 += 32)
+          reinterpret_cast<float4*>(s)[j4] = reinterpret_cast<const float4*>(srow)[j4];
+        __syncwarp();
+      }
+      if (i < T && i >= n_p && k > 0) {
+        uint32_t prefix = 0u, mask = 0u;
+        int remaining = k;
+        for (int pass = 0; pass < 4; ++pass) {
+          const int shift = 24 - 8 * pass;
+#pragma unroll
+          for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
+          __syncwarp();
+          for (int jb = n_p; jb < T; jb += 32) {
+            const int j = jb + lane;
+            const uint32_t key = j < T ? order_key(s[j]) : 0u;
+            const bool in = j < T && (key & mask) == prefix;
+            // lanes with the same digit add once (scores cluster in few bins)
+            const uint32_t bin = in ? ((key >> shift) & 255u) : 256u;
+            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+            if (in && (__ffs(peers) - 1) == lane) atomicAdd(h + bin, uint32_t(__popc(peers)));
+          }
+          __syncwarp();
+          // lane L holds bins 255-8L .. 248-8L (lane 0 = highest digits)
+          uint32_t cnt = 0;
+#pragma unroll
+          for (int b = 0; b < 8; ++b) cnt += h[255 - 8 * lane - b];
+          uint32_t incl = cnt;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += o;
+          }
+          const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, incl >= uint32_t(remaining));
+          const int L = __ffs(ballot) - 1;
+          uint32_t digit = 0;
+          int rem_new = 0;
+          if (lane == L) {
+            uint32_t run = incl - cnt;                      // keys with a higher digit
+            for (int b = 0; b < 8; ++b) {
+              const uint32_t bin = 255 - 8 * L - b;
+              if (run + h[bin] >= uint32_t(remaining)) {
+                digit = bin;
+                rem_new = remaining - int(run);
+                break;
+              }
+              run += h[bin];
+            }
+          }
+          digit = __shfl_sync(0xFFFFFFFFu, digit, L);
+          remaining = __shfl_sync(0xFFFFFFFFu, rem_new, L);
+          prefix |= digit << shift;
+          mask |= 255u << shift;
+          __syncwarp();
+        }
+        // prefix = K*, remaining = number of keys equal to K* to keep (lowest j first)
+        int32_t* out_idx = topk_idx + ((bh * n_v) + (i - n_p)) * int64_t(k);
+        float* out_s = topk_score ? topk_score + ((bh * n_v) + (i - n_p)) * int64_t(k) : nullptr;
+        int pos = 0, eq_seen = 0;
+        for (int base = n_p; base < T; base += 32) {
+          const int j = base + lane;
+          const bool valid = j < T;
+          const float sv = valid ? s[j] : 0.f;
+          const uint32_t key = valid ? order_key(sv) : 0u;
+          const bool gt = valid && key > prefix;
+          const bool eq = valid && key == prefix;
+          const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
+          const int eq_rank = eq_seen + __popc(eqb & lt_mask);
+          const bool sel = gt || (eq && eq_rank < remaining);
+          const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
+          if (sel) {
+            const int o = pos + __popc(selb & lt_mask);
+            out_idx[o] = j;
+            if (out_s) out_s[o] = sv;
+          }
+          pos += __popc(selb);
+          eq_seen += __popc(eqb);
+        }
+      }
+      // ---- 3a. softmax of the row; P to the scratch row
+      float m = -INFINITY;
+      for (int j = lane; j < T; j += 32) m = fmaxf(m, s[j]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+      float l = 0.f;
+      for (int j = lane; j < T; j += 32) {
+        const float p = __expf(s[j] - m);
+        srow[j] = p;
+        l += p;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
+      inv_l[r] = 1.0f / l;
+      __syncwarp();        // the row buffer is refilled for the next row
+    }
+
+    // ---- 3b. o_coarse = P V / l: P chunks staged into shared memory next to
+    // the value chunks
+    float acc[RW][D / 32];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
-      for (int u = 0; u < KPL; ++u) acc[r][u] = 0.f;
-    const float* qw = qT + warp * RW;
-#pragma unroll 4
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      float av[KPL][4];
-#pragma unroll
-      for (int u = 0; u < KPL; ++u) {
-        const float4 a = reinterpret_cast<const float4*>(stage + (lane + 32 * u) * kStride)[d4];
-        av[u][0] = a.x;
-        av[u][1] = a.y;
-        av[u][2] = a.z;
-        av[u][3] = a.w;
+      for (int c = 0; c < D / 32; ++c) acc[r][c] = 0.f;
+    __syncthreads();     // every P row written; qT no longer needed (P stage)
+    float* pst = qT;     // [2][QB][kKC]
+    auto stage_p = [&](int buf, int j0, int nj) {
+      // P[r][j0 .. j0 + nj) of all QB rows; 16-byte pieces (j0 and Tpad are
+      // multiples of 4; a ragged tail piece reads past nj into the row's
+      // padding, never past the scratch slot)
+      constexpr int kPieces = QB * (kKC / 4);
+      for (int idx = threadIdx.x; idx < kPieces; idx += kWarps * 32) {
+        const int r = idx / (kKC / 4), q4 = (idx % (kKC / 4)) * 4;
+        if (q4 >= nj) continue;
+        const uint32_t dst = static_cast<uint32_t>(
+            __cvta_generic_to_shared(pst + buf * QB * kKC + r * kKC + q4));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                     "l"(sc + r * Tpad + j0 + q4)
+                     : "memory");
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float q[RW];
-        QVec<RW>::load(qw + (4 * d4 + e) * QB, q);
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-          for (int u = 0; u < KPL; ++u) acc[r][u] = fmaf(q[r], av[u][e], acc[r][u]);
+    };
+    stage_p(0, 0, min(kKC, T));
+    stage_rows_async<D, NW>(stage0, vb, min(kKC, T));
+    for (int c = 0; c < n_chunks; ++c) {
+      const int j0 = c * kKC;
+      const int nj = min(kKC, T - j0);
+      const float* stage = stage0 + (c & 1) * kKC * kStride;
+      const float* pc = pst + (c & 1) * QB * kKC;
+      if (c + 1 < n_chunks) {
+        stage_p((c + 1) & 1, j0 + kKC, min(kKC, T - j0 - kKC));
+        stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, vb + int64_t(j0 + kKC) * D,
+                                min(kKC, T - j0 - kKC));
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
       }
+      __syncthreads();
+      for (int jj = 0; jj < nj; ++jj) {
+        float v[D / 32];
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2) v[c2] = stage[jj * kStride + lane + 32 * c2];
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+          const float p = pc[(warp * RW + r) * kKC + jj];
+#pragma unroll
+          for (int c2 = 0; c2 < D / 32; ++c2) acc[r][c2] = fmaf(p, v[c2], acc[r][c2]);
+        }
+      }
+      __syncthreads();
     }
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
-      float* row = sc + (warp * RW + r) * Tpad + j0;
+      const int i = i0 + warp * RW + r;
+      if (i >= T) continue;
+      float* oc = o_coarse + (bh * T + i) * D;
 #pragma unroll
-      for (int u = 0; u < KPL; ++u)
-        if (lane + 32 * u < nj) row[lane + 32 * u] = scale * acc[r][u];
+      for (int c = 0; c < D / 32; ++c) oc[lane + 32 * c] = acc[r][c] * inv_l[r];
     }
-    __syncthreads();     // stage (c & 1) is refilled two chunks later
-  }
-
-  // ---- 2. top-k over video key tiles (video query tiles only), raw scores
-  const int n_v = T - n_p;
-  uint32_t* h = hist + warp * 256;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int r = 0; r < RW; ++r) {
-    const int i = i0 + warp * RW + r;
-    if (i >= T || i < n_p || k <= 0) continue;
-    const float* s = sc + (warp * RW + r) * Tpad;
-    uint32_t prefix = 0u, mask = 0u;
-    int remaining = k;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
-      __syncwarp();
-      for (int jb = n_p; jb < T; jb += 32) {
-        const int j = jb + lane;
-        const uint32_t key = j < T ? order_key(s[j]) : 0u;
-        const bool in = j < T && (key & mask) == prefix;
-        // lanes with the same digit add once (scores cluster in few bins)
-        const uint32_t bin = in ? ((key >> shift) & 255u) : 256u;
-        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-        if (in && (__ffs(peers) - 1) == lane) atomicAdd(h + bin, uint32_t(__popc(peers)));
-      }
-      __syncwarp();
-      // lane L holds bins 255-8L .. 248-8L (lane 0 = highest digits)
-      uint32_t cnt = 0;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) cnt += h[255 - 8 * lane - b];
-      uint32_t incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, incl >= uint32_t(remaining));
-      const int L = __ffs(ballot) - 1;
-      uint32_t digit = 0;
-      int rem_new = 0;
-      if (lane == L) {
-        uint32_t run = incl - cnt;                      // keys with a higher digit
-        for (int b = 0; b < 8; ++b) {
-          const uint32_t bin = 255 - 8 * L - b;
-          if (run + h[bin] >= uint32_t(remaining)) {
-            digit = bin;
-            rem_new = remaining - int(run);
-            break;
-          }
-          run += h[bin];
-        }
-      }
-      digit = __shfl_sync(0xFFFFFFFFu, digit, L);
-      remaining = __shfl_sync(0xFFFFFFFFu, rem_new, L);
-      prefix |= digit << shift;
-      mask |= 255u << shift;
-      __syncwarp();
-    }
-    // prefix = K*, remaining = number of keys equal to K* to keep (lowest j first)
-    int32_t* out_idx = topk_idx + ((bh * n_v) + (i - n_p)) * int64_t(k);
-    float* out_s = topk_score ? topk_score + ((bh * n_v) + (i - n_p)) * int64_t(k) : nullptr;
-    int pos = 0, eq_seen = 0;
-    for (int base = n_p; base < T; base += 32) {
-      const int j = base + lane;
-      const bool valid = j < T;
-      const float sv = valid ? s[j] : 0.f;
-      const uint32_t key = valid ? order_key(sv) : 0u;
-      const bool gt = valid && key > prefix;
-      const bool eq = valid && key == prefix;
-      const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
-      const int eq_rank = eq_seen + __popc(eqb & lt_mask);
-      const bool sel = gt || (eq && eq_rank < remaining);
-      const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
-      if (sel) {
-        const int o = pos + __popc(selb & lt_mask);
-        out_idx[o] = j;
-        if (out_s) out_s[o] = sv;
-      }
-      pos += __popc(selb);
-      eq_seen += __popc(eqb);
-    }
-  }
-
-  // ---- 3. softmax in place, then o_coarse
-  float inv_l[RW];
-#pragma unroll
-  for (int r = 0; r < RW; ++r) {
-    float* s = sc + (warp * RW + r) * Tpad;
-    float m = -INFINITY;
-    for (int j = lane; j < T; j += 32) m = fmaxf(m, s[j]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-    float l = 0.f;
-    for (int j = lane; j < T; j += 32) {
-      const float p = __expf(s[j] - m);
-      s[j] = p;
-      l += p;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-    inv_l[r] = 1.0f / l;
-  }
-  float acc[RW][D / 32];
-#pragma unroll
-  for (int r = 0; r < RW; ++r)
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) acc[r][c] = 0.f;
-  __syncthreads();
-  stage_rows_async<D, NW>(stage0, vb, min(kKC, T));
-  for (int c = 0; c < n_chunks; ++c) {
-    const int j0 = c * kKC;
-    const int nj = min(kKC, T - j0);
-    const float* stage = stage0 + (c & 1) * kKC * kStride;
-    if (c + 1 < n_chunks) {
-      stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, vb + int64_t(j0 + kKC) * D,
-                          min(kKC, T - j0 - kKC));
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    for (int jj = 0; jj < nj; ++jj) {
-      float v[D / 32];
-#pragma unroll
-      for (int c2 = 0; c2 < D / 32; ++c2) v[c2] = stage[jj * kStride + lane + 32 * c2];
-#pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        const float p = sc[(warp * RW + r) * Tpad + j0 + jj];
-#pragma unroll
-        for (int c2 = 0; c2 < D / 32; ++c2) acc[r][c2] = fmaf(p, v[c2], acc[r][c2]);
-      }
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int r = 0; r < RW; ++r) {
-    const int i = i0 + warp * RW + r;
-    if (i >= T) continue;
-    float* oc = o_coarse + (bh * T + i) * D;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) oc[lane + 32 * c] = acc[r][c] * inv_l[r];
   }
 }
 
-template <int D, int NW, int RW>
-size_t coarse_smem_bytes(int T) {
-  const int Tpad = (T + 3) & ~3;
-  return sizeof(float) * (size_t(D) * NW * RW + size_t(2) * kKC * (D + 4) + size_t(NW) * 256 +
-                          size_t(NW) * RW * Tpad);
-}
+constexpr int kCoarseWarps = 8, kCoarseRows = 4;          // QB = 32 query tiles per item
+constexpr int kCoarseQB = kCoarseWarps * kCoarseRows;
 
-template <int D, int NW, int RW>
-cudaError_t launch_coarse_cfg(const float* qbar, const float* kbar, const float* vbar, int64_t bh,
-                              int T, int n_p, float scale, int k, float* o_coarse,
-                              int32_t* topk_idx, float* topk_score, cudaStream_t stream) {
-  const size_t smem = coarse_smem_bytes<D, NW, RW>(T);
-  cudaError_t e = cudaFuncSetAttribute(coarse_topk_kernel<D, NW, RW>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  constexpr int QB = NW * RW;
-  const dim3 grid(unsigned((T + QB - 1) / QB), unsigned(bh), 1);
-  coarse_topk_kernel<D, NW, RW><<<grid, NW * 32, smem, stream>>>(
-      qbar, kbar, vbar, T, n_p, scale, k, o_coarse, topk_idx, topk_score);
-  return cudaGetLastError();
+template <int D>
+size_t coarse_smem_bytes() {
+  // qT [D][QB] (reused as two P stages [QB][kKC]), two key / value stages,
+  // the per-warp histograms
+  const size_t q = size_t(D) * kCoarseQB;
+  const size_t p = size_t(2) * kCoarseQB * kKC;
+  return sizeof(float) * ((q > p ? q : p) + size_t(2) * kKC * (D + 4) + size_t(kCoarseWarps) * 256);
 }
 
 template <int D>
 cudaError_t launch_coarse_d(const float* qbar, const float* kbar, const float* vbar, int64_t bh,
                             int T, int n_p, float scale, int k, float* o_coarse, int32_t* topk_idx,
-                            float* topk_score, cudaStream_t stream) {
-  // 16 warps per CTA (one CTA fills an SM's shared memory), and as many query
-  // tiles per CTA as the score rows leave room for
-  if (T <= 960)
-    return launch_coarse_cfg<D, VSA_COARSE_NW, VSA_COARSE_RW>(
-        qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx, topk_score, stream);
-  if (T <= 1920)
-    return launch_coarse_cfg<D, 16, 1>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
-                                       topk_score, stream);
-  return launch_coarse_cfg<D, 8, 1>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
-                                    topk_score, stream);
+                            float* topk_score, float* scratch, int grid, cudaStream_t stream) {
+  const size_t smem = coarse_smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(coarse_topk_kernel<D, kCoarseWarps, kCoarseRows>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  coarse_topk_kernel<D, kCoarseWarps, kCoarseRows><<<grid, kCoarseWarps * 32, smem, stream>>>(
+      qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx, topk_score, scratch);
+  return cudaGetLastError();
 }
 
 // Reference-tile selection (the Veda node's reference_sparsity): for every
@@ -476,15 +498,25 @@ cudaError_t launch_select_ref(const float* qbar, const float* kbar, int64_t bh, 
   return cudaGetLastError();
 }
 
+int coarse_grid(int num_sms) { return 2 * (num_sms > 0 ? num_sms : 148); }
+
+size_t coarse_scratch_bytes(int T, int num_sms) {
+  return sizeof(float) * size_t(coarse_grid(num_sms)) * kCoarseQB * size_t((T + 3) & ~3);
+}
+
 cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float* vbar, int64_t bh,
                                int T, int n_p, int D, float scale, int k, float* o_coarse,
-                               int32_t* topk_idx, float* topk_score, cudaStream_t stream) {
-  if (T > kMaxTiles || bh > 65535) return cudaErrorInvalidValue;
+                               int32_t* topk_idx, float* topk_score, float* scratch, int num_sms,
+                               cudaStream_t stream) {
+  if (T > kMaxTiles) return cudaErrorInvalidValue;
+  const int64_t items = bh * ((T + kCoarseQB - 1) / kCoarseQB);
+  if (items == 0) return cudaSuccess;
+  const int grid = int(std::min<int64_t>(items, coarse_grid(num_sms)));
   if (D == 128)
     return launch_coarse_d<128>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
-                                topk_score, stream);
+                                topk_score, scratch, grid, stream);
   return launch_coarse_d<64>(qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx,
-                             topk_score, stream);
+                             topk_score, scratch, grid, stream);
 }
 
 }  // namespace vsa

@@ -621,6 +621,12 @@ __device__ __noinline__ void mask_partial_tiles(uint32_t taddr, int bla, int blb
     for (int col = blb; col < 64; ++col) tmem_st1(taddr + 64 + col, ninf);
   tmem_wait_st();
 }
+// The same for one 128-row key tile: columns [bl, 128) of the S row.
+__device__ __noinline__ void mask_tile_tail(uint32_t taddr, int bl) {
+  const uint32_t ninf = __float_as_uint(-INFINITY);
+  for (int col = bl; col < 128; ++col) tmem_st1(taddr + col, ninf);
+  tmem_wait_st();
+}
 
 template <int R, int D, bool kRef>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
@@ -1145,6 +1151,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           if (!ok) break;
           if (threadIdx.x % 128 == 0) VSA_TL(1 + wg, 's', Gn);
           tc_fence_after();
+          // key rows past block_len (a partial key tile, rare): -inf in TMEM
+          if (rows_active && int(s_blen[n]) + 1 < BN) mask_tile_tail(t_lane + col_s, int(s_blen[n]) + 1);
           uint32_t r[BN / 32][32];
           if (rows_active) {
   #pragma unroll
@@ -1158,14 +1166,6 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           // row max over raw scores (scale > 0 commutes with max), four chains
           float mx = -INFINITY;
           if (rows_active) {
-            const int bl = int(s_blen[n]) + 1;
-            if (bl < BN) {
-  #pragma unroll
-              for (int c = 0; c < BN / 32; ++c)
-  #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  if (32 * c + e >= bl) r[c][e] = __float_as_uint(-INFINITY);
-            }
             float mx4[4];
   #pragma unroll
             for (int q = 0; q < 4; ++q) mx4[q] = -INFINITY;

@@ -56,10 +56,12 @@ cudaError_t launch_permute_pool(const uint16_t* src, uint16_t* dst, const int32_
                                 const int32_t* block_len, float* pooled, int64_t bh, int T, int R,
                                 int64_t src_rows, int64_t dst_rows, int D, int num_sms,
                                 cudaStream_t stream);
+// Score rows of the coarse kernel's persistent CTAs (global scratch, bytes).
+size_t coarse_scratch_bytes(int T, int num_sms);
 cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float* vbar,
                                int64_t bh, int T, int n_p, int D, float scale, int k,
                                float* o_coarse, int32_t* topk_idx, float* topk_score,
-                               cudaStream_t stream);
+                               float* scratch, int num_sms, cudaStream_t stream);
 // Top k_ref reference tiles per video query tile (n_p <= 256), ascending.
 cudaError_t launch_select_ref(const float* qbar, const float* kbar, int64_t bh, int T, int n_p, int D,
                               float scale, int k_ref, int32_t* topk_ref, int num_sms,
