@@ -91,7 +91,10 @@ def test_host_only_plan_refuses_launches(libvsa):
     assert b"host-only" in libvsa.vsa_last_error()
     n = ctypes.c_size_t()
     assert libvsa.vsa_workspace_size(p.handle, 1, 2, 64, 2, ctypes.byref(n)) == 0
-    assert n.value == 3 * 1 * 2 * p.n_tiles * 64 * 4
+    # the pooled means, then the coarse kernel's score rows: 32 rows of
+    # ceil4(T) floats for each of its 2 x 148 CTAs (a host-only plan assumes
+    # 148 SMs)
+    assert n.value == 3 * 1 * 2 * p.n_tiles * 64 * 4 + 2 * 148 * 32 * ((p.n_tiles + 3) // 4 * 4) * 4
     assert libvsa.vsa_workspace_size(p.handle, 1, 2, 96, 2, ctypes.byref(n)) == 2
     # the calls added for training and tile-before-projecting refuse a host-only plan too
     vp = ctypes.cast(buf, ctypes.c_void_p)
