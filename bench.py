@@ -49,7 +49,7 @@ UNIT = "ms/layer"
 # one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) at the
 # benchmark size, valid only for the kernel source it was taken on (checked
 # by hash below).
-ATTN_TRAFFIC = {"source_sha256_16": "0af39b16e1e9c15c", "bytes": 20.28e9}
+ATTN_TRAFFIC = {"source_sha256_16": "1ed1b44da672f7d9", "bytes": 9.42e9}
 
 
 # ----------------------------------------------------------------- accounting
@@ -58,6 +58,12 @@ ATTN_TRAFFIC = {"source_sha256_16": "0af39b16e1e9c15c", "bytes": 20.28e9}
 # doubled figure assumes 2:4 sparsity).  The roofline fractions use the
 # measured peak; this one is reported beside them.
 NOMINAL_DENSE_BF16_TFLOPS = 2250.0
+
+
+def fp32_core_peak_tflops(sm_count: int = 148, sm_mhz: float = 1965.0) -> float:
+    """fp32 CUDA-core peak from the unit counts: 128 fp32 FMA lanes per SM per
+    clock (4 sub-partitions x 32), 2 FLOP per FMA, at the maximum SM clock."""
+    return sm_count * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 def geometry_counts(w: Workload, n_p: int, T: int, k: int) -> dict:
@@ -78,6 +84,10 @@ def geometry_counts(w: Workload, n_p: int, T: int, k: int) -> dict:
         # is read in natural order by the fused attention + combine); the tile
         # means are taken in the same pass
         permute_bytes=3.0 * BH * (N + N_pad) * D * 2,
+        # coarse attention on the pooled tiles: scores and the weighted sum of
+        # the value means, 2*T*T*D FLOP each per head (exponentials and the
+        # top-k's comparisons not counted)
+        coarse_flop=4.0 * T * T * D * BH,
         # attention + combine: Q, K, V read once, the gate read and the output
         # written once (natural order)
         attn_bytes=3.0 * BH * N_pad * D * 2 + 2.0 * BH * N * D * 2,
@@ -591,6 +601,13 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "kernels_hbm_gbs": {"permute_pool_q_k_v": round(acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9, 1)},
         "kernels_hbm_frac": {"permute_pool_q_k_v": round(
             acct["permute_bytes"] / (part_ms[0] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "coarse_topk_roofline": {
+            "bound": "alu", "unit": "TFLOP/s",
+            "achieved": round(acct["coarse_flop"] / (part_ms[1] * 1e-3) / 1e12, 2),
+            "peak": round(fp32_core_peak_tflops(), 1),
+            "frac": round(acct["coarse_flop"] / (part_ms[1] * 1e-3) / 1e12 / fp32_core_peak_tflops(), 4),
+            "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 FLOP x 1965 MHz",
+            "work": "4*T*T*D FLOP per head (scores + weighted sum of the value means)"},
         "roofline": {"kernel": "sparse_attn_combine", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
                      "frac_of_sustained": round(achieved / peaks["bf16_sustained"], 4),

@@ -97,7 +97,7 @@ vsa_status vsa_plan_create(const vsa_geometry* geom, int device, vsa_plan* out) 
     if (e == cudaSuccess) e = cudaMalloc(&p->d_untile, nb_u);
     if (e == cudaSuccess) e = cudaMalloc(&p->d_row_src, nb_r);
     if (e == cudaSuccess) e = cudaMalloc(&p->d_block_len, nb_b);
-    if (e == cudaSuccess) e = cudaMalloc(&p->d_status, 16);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_status, 32);
     if (e == cudaSuccess && !p->untile.empty())
       e = cudaMemcpy(p->d_untile, p->untile.data(), p->untile.size() * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !p->row_src.empty())
@@ -105,7 +105,7 @@ vsa_status vsa_plan_create(const vsa_geometry* geom, int device, vsa_plan* out) 
     if (e == cudaSuccess && !p->block_len.empty())
       e = cudaMemcpy(p->d_block_len, p->block_len.data(), p->block_len.size() * 4,
                      cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, 16);
+    if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, 32);
     if (prev >= 0) cudaSetDevice(prev);
     if (e != cudaSuccess) {
       p->device = device;

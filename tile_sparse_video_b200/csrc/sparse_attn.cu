@@ -227,6 +227,7 @@ struct AttnArgs {
   float* lse;                 // [BH, N_pad] or null
   unsigned int* status;       // device status word
   unsigned long long wait_ns; // bound of every mbarrier wait (kWaitLimitNs unless shortened)
+  unsigned int* work;         // paired tiles: [next item, CTAs done], zero at launch
   // fused gated combine (step 5) in the epilogue: out[row_src[r]] =
   // o_fine[r] + sigmoid(gate[row_src[r]]) * o_coarse[tile(r)]
   const uint16_t* gate;       // bf16 [BH, N, D] natural order, or null (unfused)
@@ -268,8 +269,10 @@ struct Cfg {
   // barriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV],
   //           s_full[2], s_empty[2], p_full[2], pv_done[2], dec[4], o_full, o_empty,
   //           drain, drain2, list_full[2], list_empty[2] (paired tiles)
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 4 + (kPair ? 4 : 0);
-  static constexpr int TAIL = NBAR * 8 + 16;              // barriers + tmem slot + abort flag
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + 4 + 4 + 4;
+  // barriers, then the tmem slot, the abort flag and (128-row tiles) the
+  // item of each of the two list slots
+  static constexpr int TAIL = NBAR * 8 + 16;
   // TMEM columns: O [0, D), S_w [D + w*BN, D + (w+1)*BN), P_w (bf16 pairs)
   // [D + 2*BN + w*BN/2, D + 2*BN + (w+1)*BN/2)
   static constexpr uint32_t COL_O = 0;
@@ -399,6 +402,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
                                          const CUtensorMap* tm_t, const CUtensorMap* tm_other,
                                          uint32_t sQ, uint32_t sT, uint32_t full, uint32_t empty,
                                          uint32_t q_full, uint32_t q_empty, int32_t* s_list,
+                                         uint32_t list_full, uint32_t list_empty, int* items,
                                          volatile int* abort_flag, int lane, int BH, int n_v) {
   using C = Cfg<R, D>;
   constexpr int kPrefetch = VSA_PREFETCH;
@@ -406,7 +410,31 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
   uint32_t g = 0, q_issued = 0;
   int t = 0;
   bool ok = true;
-  for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+  for (; ok; ++t) {
+    // the item: the K warp takes the next one of the grid (head-major order)
+    // from the work counter and publishes it in slot t & 1 (-1: none left)
+    const int slot = t & 1;
+    int item = 0;
+    if (kIsK) {
+      if (t >= 2)
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(list_empty + 8 * slot, ((t >> 1) - 1) & 1, abort_flag,
+                                              a.status, 27, a.wait_ns));
+      if (!ok) break;
+      if (lane == 0) item = int(atomicAdd(a.work, 1u));
+      item = __shfl_sync(0xFFFFFFFFu, item, 0);
+      if (lane == 0) {
+        items[slot] = item < a.n_items ? item : -1;
+        mbar_arrive(list_full + 8 * slot);
+      }
+      __syncwarp();
+      if (item >= a.n_items) break;
+    } else {
+      ok = __all_sync(0xFFFFFFFFu,
+                      wait_bar(list_full + 8 * slot, (t >> 1) & 1, abort_flag, a.status, 28, a.wait_ns));
+      if (!ok) break;
+      item = items[slot];
+      if (item < 0) break;
+    }
     int64_t bh;
     int i;
     decode_item(item, BH, a.n_p, n_v, bh, i);
@@ -464,6 +492,7 @@ __device__ __forceinline__ void producer(const AttnArgs& a, const CUtensorMap* t
     }
     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     __syncwarp();
+    if (lane == 0) mbar_arrive(list_empty + 8 * slot);
   }
   if (lane == 0 && !ok) {
     // Abort: make sure none of our TMA writes is still in flight.
@@ -539,10 +568,9 @@ __device__ __forceinline__ void producer_pair(const AttnArgs& a, const CUtensorM
   uint32_t g = 0, q_issued = 0;
   int t = 0;
   bool ok = true;
-  for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+  for (; ok; ++t) {
     int64_t bh;
     int m;
-    decode_pair(item, a.BH, n_pp, n_pairs, bh, m);
     const int slot = t & 1;
     uint32_t* list = lists + slot * cap;
     int count;
@@ -551,9 +579,23 @@ __device__ __forceinline__ void producer_pair(const AttnArgs& a, const CUtensorM
         ok = __all_sync(0xFFFFFFFFu, wait_bar(list_empty + 8 * slot, ((t >> 1) - 1) & 1, abort_flag,
                                               a.status, 22, a.wait_ns));
       if (!ok) break;
+      // the next item of the whole grid, in the head-major item order
+      int item = 0;
+      if (lane == 0) item = int(atomicAdd(a.work, 1u));
+      item = __shfl_sync(0xFFFFFFFFu, item, 0);
+      if (item >= a.n_items) {          // none left: publish the end
+        if (lane == 0) {
+          counts[slot] = -1;
+          mbar_arrive(list_full + 8 * slot);
+        }
+        __syncwarp();
+        break;
+      }
+      decode_pair(item, a.BH, n_pp, n_pairs, bh, m);
       count = build_pair_list<kRef>(a, bh, m, bm, list, lane);
       if (lane == 0) {
         counts[slot] = count;
+        counts[2 + slot] = item;
         mbar_arrive(list_full + 8 * slot);
       }
       __syncwarp();
@@ -562,6 +604,8 @@ __device__ __forceinline__ void producer_pair(const AttnArgs& a, const CUtensorM
                       wait_bar(list_full + 8 * slot, (t >> 1) & 1, abort_flag, a.status, 23, a.wait_ns));
       if (!ok) break;
       count = counts[slot];
+      if (count < 0) break;              // no item left
+      decode_pair(counts[2 + slot], a.BH, n_pp, n_pairs, bh, m);
     }
     const int nk = (count + 1) >> 1;
     if (lane == 0) {
@@ -665,6 +709,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* s_blen = smem + C::OFF_BAR + C::TAIL;                  // [T]
   int32_t* s_klist = reinterpret_cast<int32_t*>(s_blen + ((a.T + 15) & ~15));
   int32_t* s_vlist = s_klist + ((a.k + 3) & ~3);
+  // 128-row tiles: the item of each list slot (-1: none left)
+  int* r_items = reinterpret_cast<int*>(smem + C::OFF_BAR + C::NBAR * 8 + 8);
   // paired tiles: list lengths [2], bitmaps [2][W], list slots [2][cap]
   int* p_counts = reinterpret_cast<int*>(smem + C::OFF_BAR + C::TAIL);
   uint32_t* p_bm = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::TAIL + 16);
@@ -698,11 +744,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
     mbar_init(drain2, 1);
-    if constexpr (C::kPair) {
-      for (int sl = 0; sl < 2; ++sl) {
-        mbar_init(list_full + 8 * sl, 1);
-        mbar_init(list_empty + 8 * sl, 12);
-      }
+    for (int sl = 0; sl < 2; ++sl) {
+      mbar_init(list_full + 8 * sl, 1);
+      mbar_init(list_empty + 8 * sl, 12);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -732,7 +776,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                         abort_flag, lane);
     else
       producer<R, D, NSK, true, kRef>(a, &tm_q, &tm_k, &tm_v, sQ, sK, k_full, k_empty, q_full,
-                                      q_empty, s_klist, abort_flag, lane, BH, n_v);
+                                      q_empty, s_klist, list_full, list_empty, r_items, abort_flag,
+                                      lane, BH, n_v);
   } else if (warp == kWarpTmaV) {
     if constexpr (C::kPair)
       producer_pair<D, NSV, false, kRef>(a, &tm_q, &tm_v, sQ, sV, v_full, v_empty, q_full, q_empty,
@@ -740,7 +785,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                          abort_flag, lane);
     else
       producer<R, D, NSV, false, kRef>(a, &tm_q, &tm_v, &tm_k, sQ, sV, v_full, v_empty, q_full,
-                                       q_empty, s_vlist, abort_flag, lane, BH, n_v);
+                                       q_empty, s_vlist, list_full, list_empty, r_items, abort_flag,
+                                       lane, BH, n_v);
   } else if (warp == kWarpMmaS) {
     // ------------------------------------------------------------ S issuer
     // S_n = Q K_n^T into S_w (w = n & 1) as soon as K_n is in and warpgroup w
@@ -752,19 +798,27 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       uint32_t g = 0;                    // tiles of earlier items (trace only)
       int t = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+      for (; ok; ++t) {
         int nk;
         if constexpr (C::kPair) {
           if (!wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag, a.status, 24, a.wait_ns)) {
             ok = false;
             break;
           }
+          if (p_counts[t & 1] < 0) break;          // no item left
           nk = (p_counts[t & 1] + 1) >> 1;
           mbar_arrive(list_empty + 8 * (t & 1));
         } else {
+          if (!wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag, a.status, 29, a.wait_ns)) {
+            ok = false;
+            break;
+          }
+          const int it = r_items[t & 1];
+          if (it < 0) break;                      // no item left
+          mbar_arrive(list_empty + 8 * (t & 1));
           int64_t bh;
           int i;
-          decode_item(item, BH, a.n_p, n_v, bh, i);
+          decode_item(it, BH, a.n_p, n_v, bh, i);
           nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
         }
         if (!wait_bar(q_full, t & 1, abort_flag, a.status, 5, a.wait_ns)) { ok = false; break; }
@@ -812,19 +866,27 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       uint32_t g = 0;                    // tiles of earlier items (trace only)
       int t = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+      for (; ok; ++t) {
         int nk;
         if constexpr (C::kPair) {
           if (!wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag, a.status, 25, a.wait_ns)) {
             ok = false;
             break;
           }
+          if (p_counts[t & 1] < 0) break;          // no item left
           nk = (p_counts[t & 1] + 1) >> 1;
           mbar_arrive(list_empty + 8 * (t & 1));
         } else {
+          if (!wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag, a.status, 30, a.wait_ns)) {
+            ok = false;
+            break;
+          }
+          const int it = r_items[t & 1];
+          if (it < 0) break;                      // no item left
+          mbar_arrive(list_empty + 8 * (t & 1));
           int64_t bh;
           int i;
-          decode_item(item, BH, a.n_p, n_v, bh, i);
+          decode_item(it, BH, a.n_p, n_v, bh, i);
           nk = (i < a.n_p) ? a.T : n_sink<kRef>(a) + a.k;
         }
         for (int n = 0; n < nk; ++n) {
@@ -887,17 +949,21 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       uint32_t cw = 0;             // steps processed by this warpgroup
       int t = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
-        int64_t bh;
-        int m;
-        decode_pair(item, BH, n_pp, n_pairs, bh, m);
+      for (; ok; ++t) {
         ok = __all_sync(0xFFFFFFFFu, wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag,
                                               a.status, 26, a.wait_ns));
         if (!ok) break;
-        int count;
+        int count, item;
         asm volatile("ld.shared.u32 %0, [%1];"
                      : "=r"(count)
                      : "r"(s_base + C::OFF_BAR + C::TAIL + 4 * (t & 1)));
+        if (count < 0) break;                              // no item left
+        asm volatile("ld.shared.u32 %0, [%1];"
+                     : "=r"(item)
+                     : "r"(s_base + C::OFF_BAR + C::TAIL + 8 + 4 * (t & 1)));
+        int64_t bh;
+        int m;
+        decode_pair(item, BH, n_pp, n_pairs, bh, m);
         const int nk = (count + 1) >> 1;
         const uint32_t plist = s_lists + 4 * (t & 1) * C::list_cap(a.T);
         const int i = 2 * m + half;                         // this warp's query tile
@@ -1122,7 +1188,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       uint32_t cw = 0;             // tiles processed by this warpgroup
       int t = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x, ++t) {
+      for (; ok; ++t) {
+        ok = __all_sync(0xFFFFFFFFu, wait_bar(list_full + 8 * (t & 1), (t >> 1) & 1, abort_flag,
+                                              a.status, 31, a.wait_ns));
+        if (!ok) break;
+        const int item = r_items[t & 1];
+        if (item < 0) break;                               // no item left
         int64_t bh;
         int i;
         decode_item(item, BH, a.n_p, n_v, bh, i);
@@ -1353,6 +1424,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         tc_fence_before();
         mbar_arrive(o_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(list_empty + 8 * (t & 1));   // this warp is done with the item
         if (lane == 0) VSA_TR(quad + 4 * wg, 18, g_last);
         G += nk;
       }
@@ -1363,6 +1436,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   if (lane == 0) VSA_TR(warp, 19, 0);
   tc_fence_before();
   __syncthreads();
+  // the last CTA to finish resets the work counter for the next launch (no
+  // CTA takes an item once it has counted itself done)
+  if (threadIdx.x == 0 && atomicAdd(a.work + 1, 1u) == gridDim.x - 1) {
+    atomicExch(a.work, 0u);
+    atomicExch(a.work + 1, 0u);
+  }
   if (warp == kWarpMmaS) {
     __syncwarp();
     tc_fence_after();
@@ -1414,6 +1493,7 @@ vsa_status launch_rd(const vsa_plan_s* p, const void* q_t, const void* k_t, cons
   a.lse = lse_t;
   a.status = p->d_status;
   a.wait_ns = wait_limit_ns();
+  a.work = p->d_status + 4;
   a.T = p->n_tiles;
   a.n_p = p->n_prefix_tiles;
   a.k = k;

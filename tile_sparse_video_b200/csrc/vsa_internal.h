@@ -25,7 +25,9 @@ struct vsa_plan_s {
   int32_t* d_untile = nullptr;
   int32_t* d_row_src = nullptr;
   int32_t* d_block_len = nullptr;
-  unsigned int* d_status = nullptr;   // device status word (0 = ok)
+  // device status word (0 = ok) in [0, 4); [4, 6): the attention kernel's
+  // work counter (next item, CTAs done), zero between launches
+  unsigned int* d_status = nullptr;
 };
 
 namespace vsa {
