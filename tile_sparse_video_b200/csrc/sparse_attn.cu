@@ -944,6 +944,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       const uint32_t dbar = dec + 8 * quad;
       const uint32_t s_lists =
           s_base + C::OFF_BAR + C::TAIL + 16 + 8 * ((C::bitmap_words(a.T) + 3) & ~3);
+      const uint32_t s_mbox = s_base + C::OFF_X;             // reference-max mailbox [2][128]
       uint32_t G = 0;              // global index of the item's first step
       uint32_t cnt[2] = {0, 0};    // steps of each warpgroup in earlier items
       uint32_t cw = 0;             // steps processed by this warpgroup
@@ -961,14 +962,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         asm volatile("ld.shared.u32 %0, [%1];"
                      : "=r"(item)
                      : "r"(s_base + C::OFF_BAR + C::TAIL + 8 + 4 * (t & 1)));
-        int64_t bh;
-        int m;
-        decode_pair(item, BH, n_pp, n_pairs, bh, m);
+        (void)item;                                        // decoded again at the epilogue
         const int nk = (count + 1) >> 1;
         const uint32_t plist = s_lists + 4 * (t & 1) * C::list_cap(a.T);
-        const int i = 2 * m + half;                         // this warp's query tile
-        const bool rows_active = i < a.T;                   // warp-uniform
-        const int q_live = rows_active ? __ldg(a.block_len + i) : 0;
 
         float m_mine = -INFINITY, l = 0.f;   // l: this warpgroup's row sum, relative to m_mine
         for (int n = wg; n < nk; n += 2, ++cw) {
@@ -1015,7 +1011,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           if (Gn > 0) {
             ok = __all_sync(0xFFFFFFFFu, wait_bar(dbar, (Gn - 1) & 1, abort_flag, a.status, 14, a.wait_ns));
             if (!ok) break;
-            if (n > 0) m_prev = mbox[((Gn - 1) & 1) * 128 + row];
+            if (n > 0) asm volatile("ld.shared.f32 %0, [%1];" : "=f"(m_prev) : "r"(s_mbox + 4 * (((Gn - 1) & 1) * 128 + row)));
           }
           const float m_cand = fmaxf(m_prev, mx * a.scale_log2);
           const bool rescale = __any_sync(0xFFFFFFFFu, m_cand > m_prev + 8.0f);
@@ -1041,17 +1037,18 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #pragma unroll
             for (int c2 = 0; c2 < 2; ++c2) {
               if (c2 == 1 && kPubChunk > 0 && kPubChunk < 4) {
-                mbox[(Gn & 1) * 128 + row] = m_new;
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(s_mbox + 4 * ((Gn & 1) * 128 + row)), "f"(m_new) : "memory");
                 mbar_arrive(dbar);
                 published = true;
               }
-              uint32_t pw[32];
-              if (bl2[c2] == 0) {
+              // P in 16-column stores, so that only 16 packed words are live
 #pragma unroll
-                for (int e = 0; e < 32; ++e) pw[e] = 0u;
-              } else {
+              for (int h = 0; h < 2; ++h) {
+                uint32_t pw[16];
+                if (bl2[c2] == 0) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                  for (int e = 0; e < 16; ++e) pw[e] = 0u;
+                } else {
 #pragma unroll
                   for (int e = 0; e < 32; e += 2) {
                     float x0, x1;
@@ -1061,17 +1058,18 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                              x0, x1);
                     const float p0 = ex2(x0), p1 = ex2(x1);
                     acc2[(e >> 1) & 1] = fadd2(acc2[(e >> 1) & 1], f2pack(p0, p1));
-                    pw[16 * h + (e >> 1)] = pack_bf16(p0, p1);
+                    pw[e >> 1] = pack_bf16(p0, p1);
                   }
+                }
+                tmem_st16(t_lane + col_p + 32 * c2 + 16 * h, pw);
               }
-              tmem_st32(t_lane + col_p + 32 * c2, pw);
             }
             float s0, s1;
             f2unpack(fadd2(acc2[0], acc2[1]), s0, s1);
             l += s0 + s1;
           }
           if (!published) {
-            mbox[(Gn & 1) * 128 + row] = m_new;
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(s_mbox + 4 * ((Gn & 1) * 128 + row)), "f"(m_new) : "memory");
             mbar_arrive(dbar);
           }
           // O rescale when the reference max moved: O holds PV_0..PV_{n-1}
@@ -1109,6 +1107,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         x_l[wg * 128 + row] = l;
         if (*abort_flag) { ok = false; break; }
         asm volatile("bar.sync 1, 256;" ::: "memory");
+        // the item (re-read from its slot: not kept in registers through the steps)
+        asm volatile("ld.shared.u32 %0, [%1];"
+                     : "=r"(item)
+                     : "r"(s_base + C::OFF_BAR + C::TAIL + 8 + 4 * (t & 1)));
+        int64_t bh;
+        int m;
+        decode_pair(item, BH, n_pp, n_pairs, bh, m);
+        const int i = 2 * m + half;                         // this warp's query tile
+        const bool rows_active = i < a.T;                   // warp-uniform
+        const int q_live = rows_active ? __ldg(a.block_len + i) : 0;
         if (rows_active) {
           const float m0 = x_m[row], m1 = x_m[128 + row];
           const float l0 = x_l[row], l1 = x_l[128 + row];
