@@ -1234,9 +1234,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           if (rows_active && int(s_blen[n]) + 1 < BN) mask_tile_tail(t_lane + col_s, int(s_blen[n]) + 1);
           uint32_t r[BN / 32][32];
           if (rows_active) {
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + col_s + 32 * c, r[c]);
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < BN / 32; ++c) tmem_wait_ld(r[c]);
           }
           tc_fence_before();
@@ -1246,11 +1246,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           float mx = -INFINITY;
           if (rows_active) {
             float mx4[4];
-  #pragma unroll
+#pragma unroll
             for (int q = 0; q < 4; ++q) mx4[q] = -INFINITY;
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < BN / 32; ++c)
-  #pragma unroll
+#pragma unroll
               for (int e = 0; e < 32; e += 2)
                 mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(r[c][e]),
                                           __uint_as_float(r[c][e + 1]));
@@ -1288,10 +1288,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             // exponential in kExp2FmaShare runs on the FMA pipe.
             const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(-m_new, -m_new);
             uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-  #pragma unroll
+#pragma unroll
             for (int c2 = 0; c2 < BN / 64; ++c2) {
               uint32_t pw[32];
-  #pragma unroll
+#pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const int c = 2 * c2 + h;
                 if (kPubChunk > 0 && kPubChunk < BN / 32 && c == kPubChunk) {
@@ -1299,7 +1299,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                   mbar_arrive(dbar);
                   published = true;
                 }
-  #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                   float x0, x1;
                   f2unpack(ffma2(f2pack(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), sc2,
@@ -1341,12 +1341,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             tc_fence_after();
             if (rows_active) {
               const float alpha = ex2(m_prev - m_new);
-  #pragma unroll
+#pragma unroll
               for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tmem_ld32(t_lane + C::COL_O + 32 * c, o);
                 tmem_wait_ld(o);
-  #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                 tmem_st32(t_lane + C::COL_O + 32 * c, o);
               }
@@ -1388,16 +1388,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                  : a.out + (bh * a.n_pad + int64_t(i) * R + row) * D + wg * (D / 2);
           const uint16_t* grow = fused ? a.gate + (bh * a.n_tok + tok) * D + wg * (D / 2) : nullptr;
           const float* ocrow = fused ? a.o_coarse + (bh * a.T + i) * D + wg * (D / 2) : nullptr;
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < D / 64; ++c) {
             uint32_t o[32];
             tmem_ld32(t_lane + C::COL_O + wg * (D / 2) + 32 * c, o);
             tmem_wait_ld(o);
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-  #pragma unroll
+#pragma unroll
             for (int q = 0; q < 4; ++q) {
               float v[8];
-  #pragma unroll
+#pragma unroll
               for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[8 * q + e]) * inv;
               if (fused) {
                 if (!live) continue;                  // pad rows have no natural token
@@ -1408,7 +1408,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                 const float4 c1v = __ldg(reinterpret_cast<const float4*>(ocrow + 32 * c + 8 * q + 4));
                 const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
                 const float cv[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
-  #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   v[2 * e] = fmaf(sigmoid_fast(__uint_as_float(gw[e] << 16)), cv[2 * e], v[2 * e]);
                   v[2 * e + 1] =
