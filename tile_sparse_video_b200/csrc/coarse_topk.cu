@@ -28,17 +28,16 @@ namespace {
 #define VSA_COARSE_KC 64
 #endif
 constexpr int kKC = VSA_COARSE_KC;     // key / value tiles per staged chunk
-// Warps per CTA for T <= 960 (32 query tiles per CTA, 32 / NW per warp).
 static_assert(kKC % 32 == 0, "staged chunk: a multiple of 32 tiles");
-// Fewer warps with more rows each reuse more registers but hide less
-// latency: at the 104k-token Veda layer 16 warps take 1.39 ms, 8 warps
-// 1.69 ms, 4 warps 2.93 ms on B200.  Two CTAs per SM (32-tile chunks, 8
-// warps x 2 rows) measured 1.32 ms, within the run-to-run spread of the layer.
-#ifndef VSA_COARSE_NW
-#define VSA_COARSE_NW 16
+// Warps per CTA, query rows per warp and CTAs per SM (tuning knobs).
+#ifndef VSA_COARSE_WARPS
+#define VSA_COARSE_WARPS 8
 #endif
-#ifndef VSA_COARSE_RW
-#define VSA_COARSE_RW (32 / VSA_COARSE_NW)
+#ifndef VSA_COARSE_ROWS
+#define VSA_COARSE_ROWS 4
+#endif
+#ifndef VSA_COARSE_CTAS
+#define VSA_COARSE_CTAS 2
 #endif
 constexpr int kMaxTiles = 4096;        // bound on T (shared-memory budget)
 
@@ -122,7 +121,7 @@ __device__ __forceinline__ void cp_async_wait() {
 // depends on T: every warp keeps RW = 4 query rows in registers against the
 // keys it streams from shared memory.
 template <int D, int NW, int RW>
-__global__ void __launch_bounds__(NW * 32, 2) coarse_topk_kernel(
+__global__ void __launch_bounds__(NW * 32, VSA_COARSE_CTAS) coarse_topk_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ vbar,
     int64_t n_bh, int T, int n_p, float scale, int k, float* __restrict__ o_coarse,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_score, float* __restrict__ scratch) {
@@ -391,7 +390,7 @@ __global__ void __launch_bounds__(NW * 32, 2) coarse_topk_kernel(
   }
 }
 
-constexpr int kCoarseWarps = 8, kCoarseRows = 4;          // QB = 32 query tiles per item
+constexpr int kCoarseWarps = VSA_COARSE_WARPS, kCoarseRows = VSA_COARSE_ROWS;   // QB = 32 query tiles per item
 constexpr int kCoarseQB = kCoarseWarps * kCoarseRows;
 
 template <int D>
@@ -498,7 +497,7 @@ cudaError_t launch_select_ref(const float* qbar, const float* kbar, int64_t bh, 
   return cudaGetLastError();
 }
 
-int coarse_grid(int num_sms) { return 2 * (num_sms > 0 ? num_sms : 148); }
+int coarse_grid(int num_sms) { return VSA_COARSE_CTAS * (num_sms > 0 ? num_sms : 148); }
 
 size_t coarse_scratch_bytes(int T, int num_sms) {
   return sizeof(float) * size_t(coarse_grid(num_sms)) * kCoarseQB * size_t((T + 3) & ~3);
