@@ -288,6 +288,48 @@ vsa_status vsa_gate_combine(vsa_plan plan, const void* o_fine_t, const void* gat
                             const float* o_coarse, void* out, int out_natural,
                             int B, int H, int D, void* stream);
 
+/* ---------------------------------------------------------------- runner
+ * The whole layer over inputs in HOST memory, layer after layer, with the
+ * transfers overlapped with the computation (an engineering addition: the
+ * pages describe the layer, not how its inputs reach the GPU).  The runner
+ * owns two sets of device buffers (natural and tiled Q/K/V, the gate, the
+ * workspace, o_coarse, the selection, the output) and three CUDA streams:
+ * while layer i computes, the inputs of layer i+1 are copied in and the
+ * output of layer i-1 is copied out.  Each layer is steps 1 to 5 as
+ * vsa_permute_pool (x3), vsa_coarse_topk_pooled and vsa_sparse_attn_combine
+ * compute them, so a layer's output is bit-identical to that chain's. */
+typedef struct vsa_runner_s* vsa_runner;
+
+/* Allocates the runner's device buffers (on the plan's device, which must be
+ * current) for B, H, D, k and scale as the layer calls take them.  The plan
+ * must outlive the runner.  Errors: VSA_ERR_INVALID_ARG / VSA_ERR_UNSUPPORTED
+ * for arguments the layer calls would reject, VSA_ERR_CUDA when an allocation
+ * fails (nothing is kept; *out = NULL). */
+vsa_status vsa_runner_create(vsa_plan plan, int B, int H, int D, int k, float scale,
+                             vsa_runner* out);
+
+/* Runs n_layers layers: layer i reads q[i], k[i], v[i], g[i] (host bf16
+ * [B,H,N,D], natural token order; g the gate projection split into heads) and
+ * writes out[i] (host bf16 [B,H,N,D]).  Host buffers should be page-locked
+ * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous; they
+ * must stay valid and untouched until the run has finished.  The run starts
+ * after the work already queued on `stream` and `stream` waits for its last
+ * copy-out; the call itself returns once everything is queued.  Kernel faults
+ * are recorded in the plan's status word (vsa_sync_status).  Runs of one
+ * runner must not overlap in time with each other, and nothing else may use
+ * the plan's attention kernels concurrently. */
+vsa_status vsa_runner_run(vsa_runner runner, int n_layers, const void* const* q,
+                          const void* const* k, const void* const* v, const void* const* g,
+                          void* const* out, void* stream);
+
+/* Device time of the last vsa_runner_run, in ms, from before its first
+ * copy-in to after its last copy-out (waits for the run to finish). */
+vsa_status vsa_runner_elapsed(vsa_runner runner, float* ms);
+
+/* Waits for the runner's streams, then frees its buffers, streams and events.
+ * NULL is a no-op. */
+vsa_status vsa_runner_destroy(vsa_runner runner);
+
 /* ---------------------------------------------------------------- backward
  * Gradients of a loss through steps 5 .. 1, for training (SnackOnAI, "The
  * Architecture, Unpacked": the coarse stage and the gate are learned; the VSA

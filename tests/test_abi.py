@@ -23,7 +23,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(libvsa):
     decl = declared_symbols()
-    assert len(decl) == 29
+    assert len(decl) == 33
     assert sorted(vsa.EXPORTS) == decl
     for name in decl:
         assert hasattr(libvsa, name), name
@@ -112,4 +112,20 @@ def test_host_only_plan_refuses_launches(libvsa):
     assert n.value == max(2 * 2 * T * T * 4, bitmap)
     assert libvsa.vsa_backward_workspace_size(p.handle, 1, 2, 96, ctypes.byref(n)) == 2
     assert libvsa.vsa_plan_destroy(None) == 0
+    p.close()
+
+
+def test_runner_argument_checks(libvsa):
+    """The host-buffer runner refuses what it cannot run before touching a
+    device: NULL handles and host-only plans."""
+    p = vsa.Plan((40, 70), (4, 8, 8), (4, 4, 4), device=-1)
+    r = ctypes.c_void_p(1234)
+    assert libvsa.vsa_runner_create(p.handle, 1, 2, 64, 2, 0.125, ctypes.byref(r)) == 1
+    assert b"host-only" in libvsa.vsa_last_error()
+    assert r.value is None                                       # *out cleared on failure
+    assert libvsa.vsa_runner_create(None, 1, 2, 64, 2, 0.125, ctypes.byref(r)) == 1
+    assert libvsa.vsa_runner_run(None, 1, None, None, None, None, None, None) == 1
+    ms = ctypes.c_float()
+    assert libvsa.vsa_runner_elapsed(None, ctypes.byref(ms)) == 1
+    assert libvsa.vsa_runner_destroy(None) == 0
     p.close()

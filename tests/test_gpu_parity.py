@@ -350,24 +350,45 @@ def test_empty_batch_is_a_no_op():
 
 
 def test_layer_pipeline_matches_layer():
-    """vsa.LayerPipeline (copy-in, compute and copy-out of consecutive layers
-    overlapped on three streams, two buffer sets) gives bit-identical outputs
-    to calling the Layer once per input set, for more layers than buffers."""
+    """The library's runner behind vsa.LayerPipeline (copy-in, compute and
+    copy-out of consecutive layers overlapped on three streams, two buffer
+    sets) gives bit-identical outputs to calling the Layer once per input set,
+    for more layers than buffer sets, and again on a second run of the same
+    runner."""
     from dataclasses import replace
     w = SMALL
     plan = vsa.Plan(w.prefix, w.grid, w.tile)
     k = _keep(plan, w)
     sets = [make_inputs(replace(w, seed_base=w.seed_base + 31 * i)) for i in range(5)]
     host = [{n: s[n].pin_memory() for n in "qkvg"} for s in sets]
-    outs = [torch.empty(w.B, w.H, plan.n_tokens, w.D, dtype=torch.bfloat16).pin_memory() for _ in sets]
     pipe = vsa.LayerPipeline(plan, w.B, w.H, w.D, k)
-    pipe.run(host, outs)
-    torch.cuda.synchronize()
     layer = vsa.Layer(plan, w.B, w.H, w.D, k)
-    for s, got in zip(sets, outs):
-        want = layer(*(s[n].cuda() for n in "qkvg")).cpu()
-        assert torch.equal(got, want)
+    wants = [layer(*(s[n].cuda() for n in "qkvg")).cpu() for s in sets]
+    for order in (range(5), (4, 2, 0)):
+        outs = [torch.empty(w.B, w.H, plan.n_tokens, w.D, dtype=torch.bfloat16).pin_memory()
+                for _ in order]
+        pipe.run([host[i] for i in order], outs)
+        torch.cuda.synchronize()
+        assert pipe.elapsed_ms() > 0
+        for i, got in zip(order, outs):
+            assert torch.equal(got, wants[i])
+    pipe.close()
     vsa.vsa_sync_status(plan)
+
+
+def test_runner_rejects_bad_host_tensors():
+    w = TINY
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    k = _keep(plan, w)
+    pipe = vsa.LayerPipeline(plan, w.B, w.H, w.D, k)
+    good = torch.zeros(w.B, w.H, plan.n_tokens, w.D, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        pipe.run([{n: good for n in "qkvg"}], [good.float()])
+    with pytest.raises(ValueError):
+        pipe.run([{n: good for n in "qkvg"}], [])
+    with pytest.raises(vsa.VsaError):
+        vsa.LayerPipeline(plan, w.B, w.H, 96, k)
+    pipe.close()
 
 
 REF_CASES = [

@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libvsa.so")
 SOURCES = ["api.cu", "memops.cu", "coarse_topk.cu", "sparse_attn.cu", "project.cu", "backward.cu",
-           "selftest.cu", "noalloc.cu", "plan.cpp"]
+           "selftest.cu", "noalloc.cu", "runner.cu", "plan.cpp"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3", "--expt-relaxed-constexpr",

@@ -32,6 +32,7 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_info", "vsa_plan_tables", "vsa_keep_coun
            "vsa_keep_count_ref", "vsa_select_reference",
            "vsa_sparse_attn_ref", "vsa_backward_workspace_size", "vsa_combine_backward",
            "vsa_coarse_backward", "vsa_sparse_attn_backward", "vsa_check_bounded_wait",
+           "vsa_runner_create", "vsa_runner_run", "vsa_runner_elapsed", "vsa_runner_destroy",
            "vsa_debug_set_wait_limit", "vsa_sync_status", "vsa_last_error")
 
 
@@ -86,6 +87,10 @@ def lib():
             "vsa_sparse_attn_backward": [P, V, V, V, V, V, I, V, I, V, V, V, V, V, I, I, I, F,
                                          V, V, V, V, Z, V],
             "vsa_check_bounded_wait": [P, V, V],
+            "vsa_runner_create": [P, I, I, I, I, F, ctypes.POINTER(P)],
+            "vsa_runner_run": [P, I, V, V, V, V, V, V],
+            "vsa_runner_elapsed": [P, ctypes.POINTER(F)],
+            "vsa_runner_destroy": [P],
             "vsa_debug_set_wait_limit": [ctypes.c_uint64],
             "vsa_sync_status": [P, V],
         }
@@ -626,67 +631,59 @@ class Layer:
 
 
 class LayerPipeline:
-    """Layers over host-resident inputs with the transfers overlapped: while
-    layer i computes, the inputs of layer i+1 are copied in and the output of
-    layer i-1 is copied out (three CUDA streams, ``depth`` sets of device
-    buffers, one Layer per set).  Host tensors must be pinned for the copies
-    to run asynchronously.  Each layer is the fused Layer above; results are
-    the same as calling it once per input set."""
+    """Layers over host-resident inputs through the library's runner
+    (vsa_runner_*): while layer i computes, the inputs of layer i+1 are copied
+    in and the output of layer i-1 is copied out (three CUDA streams and two
+    buffer sets, all inside the library).  Host tensors must be pinned for
+    the copies to run asynchronously.  Each layer's output is bit-identical to
+    the fused Layer's."""
 
     def __init__(self, plan: Plan, B: int, H: int, D: int, k: int, scale: Optional[float] = None,
-                 device=None, depth: int = 2):
-        if depth < 1:
-            raise ValueError("depth must be >= 1")
+                 device=None):
         dev = torch.device("cuda", plan.device) if device is None else torch.device(device)
-        self.plan, self.depth, self.dev = plan, depth, dev
-        self.layers = [Layer(plan, B, H, D, k, scale, dev) for _ in range(depth)]
-        shape = (B, H, plan.n_tokens, D)
-        self.inputs = [{n: torch.empty(shape, dtype=torch.bfloat16, device=dev) for n in "qkvg"}
-                       for _ in range(depth)]
-        self.s_in = torch.cuda.Stream(dev)
-        self.s_comp = torch.cuda.Stream(dev)
-        self.s_out = torch.cuda.Stream(dev)
+        self.plan, self.dev, self.B, self.H, self.D = plan, dev, B, H, D
+        self.scale = D ** -0.5 if scale is None else float(scale)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _check(lib().vsa_runner_create(plan.handle, B, H, D, k, self.scale, ctypes.byref(h)))
+        self._h = h
 
-    def run(self, host_inputs: Sequence[dict], host_outputs: Sequence[torch.Tensor],
-            start_event=None, end_event=None):
+    def run(self, host_inputs: Sequence[dict], host_outputs: Sequence[torch.Tensor]) -> None:
         """Layer i reads host_inputs[i] (dict of pinned "q", "k", "v", "g"
         [B,H,N,D] bf16) and writes host_outputs[i] (pinned [B,H,N,D] bf16).
-        Asynchronous: returns the event recorded after the last copy-out.
-        ``start_event`` / ``end_event`` (CUDA timing events) are recorded
-        before the first copy-in and after the last copy-out."""
+        Asynchronous: the current stream waits for the last copy-out."""
         n = len(host_inputs)
         if len(host_outputs) != n:
             raise ValueError("one output per input set")
-        mk = lambda: torch.cuda.Event()
-        ev_in, ev_comp, ev_out = [mk() for _ in range(n)], [mk() for _ in range(n)], [mk() for _ in range(n)]
-        # the new streams start after everything already queued on the current one
-        here = torch.cuda.current_stream(self.dev)
-        for st in (self.s_in, self.s_comp, self.s_out):
-            st.wait_stream(here)
-        if start_event is not None:
-            start_event.record(self.s_in)
-        for i in range(n):
-            b = i % self.depth
-            buf, layer = self.inputs[b], self.layers[b]
-            if i >= self.depth:
-                self.s_in.wait_event(ev_comp[i - self.depth])      # buffer set b read by layer i-depth
-            with torch.cuda.stream(self.s_in):
-                for name in "qkvg":
-                    buf[name].copy_(host_inputs[i][name], non_blocking=True)
-            ev_in[i].record(self.s_in)
-            self.s_comp.wait_event(ev_in[i])
-            if i >= self.depth:
-                self.s_comp.wait_event(ev_out[i - self.depth])     # layer b's output copied out
-            layer(buf["q"], buf["k"], buf["v"], buf["g"], stream=self.s_comp)
-            ev_comp[i].record(self.s_comp)
-            self.s_out.wait_event(ev_comp[i])
-            with torch.cuda.stream(self.s_out):
-                host_outputs[i].copy_(layer.out, non_blocking=True)
-            ev_out[i].record(self.s_out)
-        if end_event is not None:
-            end_event.record(self.s_out)
-        here.wait_event(ev_out[n - 1])
-        return ev_out[n - 1]
+        shape = (self.B, self.H, self.plan.n_tokens, self.D)
+        for t in [*(d[x] for d in host_inputs for x in "qkvg"), *host_outputs]:
+            if t.device.type != "cpu" or t.dtype != torch.bfloat16 or tuple(t.shape) != shape \
+                    or not t.is_contiguous():
+                raise ValueError(f"host tensors must be contiguous CPU bf16 {shape}")
+        arr = lambda ts: (ctypes.c_void_p * max(n, 1))(*(t.data_ptr() for t in ts))
+        q, k, v, g = (arr([d[x] for d in host_inputs]) for x in "qkvg")
+        out = arr(host_outputs)
+        with torch.cuda.device(self.dev):
+            _check(lib().vsa_runner_run(self._h, n, q, k, v, g, out,
+                                        _stream(torch.cuda.current_stream(self.dev))))
+
+    def elapsed_ms(self) -> float:
+        """Device time of the last run (first copy-in to last copy-out), in ms."""
+        ms = ctypes.c_float()
+        _check(lib().vsa_runner_elapsed(self._h, ctypes.byref(ms)))
+        return float(ms.value)
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            with torch.cuda.device(self.dev):
+                lib().vsa_runner_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class TrainingLayer:
