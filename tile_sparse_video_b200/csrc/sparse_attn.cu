@@ -8,13 +8,16 @@
 // plus its kept video tiles otherwise; key rows at or past block_len[j] are
 // masked; o = softmax(scale * q k^T) v per live query row.
 //
-// Design (one persistent CTA per SM, static round-robin over work items):
+// Design (one persistent CTA per SM; work items handed out in order from a
+// per-plan global counter):
 //   work item = (b*h, query tile i); the video items come first, head by
-//   head, so the CTAs share one or two heads' K/V in L2 at any time, and the
-//   prefix items (n_p per head, each T key tiles long, streaming a whole
-//   head's K/V) come last.  Run first, the prefix items kept their CTAs about
-//   a millisecond behind the others for the rest of the launch, spreading the
-//   concurrent items over three heads whose K/V no longer fit in L2.
+//   head, and the prefix items (n_p per head, each T key tiles long,
+//   streaming a whole head's K/V) come last.  The TMA K warp takes the next
+//   item from the counter (atomicAdd) and publishes it to the other roles
+//   through one of two shared-memory slots.  Taken in order, the items in
+//   flight span one or two heads, whose K/V stay in L2; a static split let
+//   CTAs drift apart by several heads, and prefix items run first kept their
+//   CTAs a millisecond behind for the rest of the launch.
 //   warp 8  (TMA K)  loads Q once per item (evict-first: it is read once) and
 //                    K_j per kept tile into a K ring.
 //   warp 9  (TMA V)  loads V_j into its own ring (V is needed later than K).
