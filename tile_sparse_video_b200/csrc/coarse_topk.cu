@@ -1,22 +1,29 @@
 // Coarse attention over pooled tiles and the per-head top-k of video key tiles.
 //
-// One CTA handles QB = 8*RW query tiles of one (b, h); warp w owns the RW
-// query tiles i0 + w*RW ...  The work is three register-tiled fp32 passes:
-//   1. scores: s[r][j] = scale * <qbar_r, kbar_j> for all T key tiles.  Key
-//      tiles are staged 64 at a time in shared memory (padded rows, so the 32
-//      lanes read 32 banks); lane l computes keys l and l+32 for the warp's RW
-//      rows, reading the RW query values of one dimension as one broadcast
-//      vector load (q is stored transposed).  Scores stay in shared memory.
-//   2. top-k (video query tiles only): a radix select over the 32-bit
-//      order-preserving image of s[r][j], j in [n_p, T): four 8-bit digit
-//      passes with a per-warp 256-bin histogram find the k-th largest key K*;
-//      one ascending sweep over j keeps every key > K* and the lowest-index
-//      keys == K* until k are kept, which writes the result already sorted by
-//      tile index with ties broken towards the lower index.  Bit-exact for
-//      given fp32 scores.
-//   3. softmax and o_coarse = sum_j p[r][j] vbar_j: the scores become
-//      probabilities in place, value tiles are staged 64 at a time, lane l
-//      accumulates columns l, l+32, ... for the warp's RW rows.
+// Persistent CTAs (two per SM, eight warps); an item is (b*h, block of QB = 32
+// query tiles).  The QB score rows of an item live in this CTA's slot of a
+// global scratch area (QB x ceil4(T) fp32, which stays in L2), so the block
+// size does not depend on T.  Three passes per item:
+//   1. scores: s[r][j] = scale * <qbar_r, kbar_j> for all T key tiles, fp32
+//      FMAs in ascending d.  Key tiles are staged 64 at a time in shared
+//      memory; lane (rg, kg) of warp w computes rows rg + 8i (i < 4) against
+//      keys 8w + 2kg + {0, 1}, so that every shared-memory read of a warp is a
+//      broadcast of at most eight distinct 16-byte words (one wavefront).
+//   2. per row (a warp takes four): the row max, then the top-k over the
+//      video key tiles (video query tiles only).  A histogram over the row's
+//      value range (256 equal-width bins of (s - min) * 256 / (max - min), a
+//      monotone map of s) finds the bin that holds the k-th largest score; its
+//      scores (at most 32, else the exact radix select below runs instead) are
+//      ranked against each other, which gives the k-th largest score K* and how
+//      many scores equal to K* to keep.  One ascending sweep then keeps every
+//      score > K* and the lowest-index scores == K*, so the result is sorted by
+//      tile index with ties broken towards the lower index; bit-exact for given
+//      fp32 scores.  The fallback radix select runs four 8-bit digit passes
+//      over the 32-bit order-preserving image of s.
+//   3. o_coarse = softmax(s) vbar: the probabilities p = exp(s - max) are made
+//      while staging, 64 key tiles at a time, next to the value tiles; lane
+//      (rg, cg) accumulates rows rg + 8i against D/32 consecutive columns, and
+//      the row sums of p in the same loop.
 #include <algorithm>
 
 #include "vsa_internal.h"
@@ -28,17 +35,15 @@ namespace {
 #define VSA_COARSE_KC 64
 #endif
 constexpr int kKC = VSA_COARSE_KC;     // key / value tiles per staged chunk
-static_assert(kKC % 32 == 0, "staged chunk: a multiple of 32 tiles");
-// Warps per CTA, query rows per warp and CTAs per SM (tuning knobs).
-#ifndef VSA_COARSE_WARPS
-#define VSA_COARSE_WARPS 8
-#endif
-#ifndef VSA_COARSE_ROWS
-#define VSA_COARSE_ROWS 4
-#endif
+static_assert(kKC == 64, "the lane maps below cover 64 key tiles per chunk");
+// CTAs per SM (tuning knob).
 #ifndef VSA_COARSE_CTAS
 #define VSA_COARSE_CTAS 2
 #endif
+constexpr int kWarps = 8;
+constexpr int kQB = 32;                // query tiles per item: 8 row groups x 4
+constexpr int kRowsPerWarp = kQB / kWarps;
+constexpr int kPStride = kKC + 4;      // row stride of a staged probability chunk
 constexpr int kMaxTiles = 4096;        // bound on T (shared-memory budget)
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -47,52 +52,11 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int RW>
-struct QVec;
-template <>
-struct QVec<1> {
-  __device__ static void load(const float* p, float (&q)[1]) { q[0] = p[0]; }
-};
-template <>
-struct QVec<2> {
-  __device__ static void load(const float* p, float (&q)[2]) {
-    const float2 v = *reinterpret_cast<const float2*>(p);
-    q[0] = v.x;
-    q[1] = v.y;
-  }
-};
-template <>
-struct QVec<4> {
-  __device__ static void load(const float* p, float (&q)[4]) {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    q[0] = v.x;
-    q[1] = v.y;
-    q[2] = v.z;
-    q[3] = v.w;
-  }
-};
-
-template <>
-struct QVec<8> {
-  __device__ static void load(const float* p, float (&q)[8]) {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    const float4 w = *reinterpret_cast<const float4*>(p + 4);
-    q[0] = v.x;
-    q[1] = v.y;
-    q[2] = v.z;
-    q[3] = v.w;
-    q[4] = w.x;
-    q[5] = w.y;
-    q[6] = w.z;
-    q[7] = w.w;
-  }
-};
-
 // Asynchronous copy of nj rows of a [*, D] fp32 matrix into a shared-memory
 // stage with a padded row stride (D + 4 floats: rows stay 16-byte aligned and
 // 128-bit reads of 8 consecutive rows hit 8 distinct bank groups).  One
 // commit group per call; the caller waits with cp_async_wait<N>.
-template <int D, int kWarps>
+template <int D>
 __device__ __forceinline__ void stage_rows_async(float* stage, const float* src, int nj) {
   constexpr int kStride = D + 4;
   constexpr int kVecPerRow = D / 4;
@@ -115,145 +79,219 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Persistent CTAs (two per SM); an item is (b*h, block of QB = NW*RW query
-// tiles).  The QB score rows of an item live in this CTA's slot of a global
-// scratch area (QB x Tpad fp32, read back from L2), so that QB no longer
-// depends on T: every warp keeps RW = 4 query rows in registers against the
-// keys it streams from shared memory.
-template <int D, int NW, int RW>
-__global__ void __launch_bounds__(NW * 32, VSA_COARSE_CTAS) coarse_topk_kernel(
+// Exact radix select of the k-th largest order key over s[n_p, T) (one warp):
+// four 8-bit digit passes, each a histogram of the digit among the keys that
+// match the digits chosen so far.  Returns (K*, number of keys equal to K* to
+// keep).  Out of line: it runs only when the range histogram cannot isolate
+// the k-th score.
+__device__ __noinline__ uint2 radix_select(const float* s, int T, int n_p, int k, uint32_t* h,
+                                           int lane) {
+  uint32_t prefix = 0u, mask = 0u;
+  int remaining = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
+    __syncwarp();
+    for (int jb = n_p; jb < T; jb += 32) {
+      const int j = jb + lane;
+      const uint32_t key = j < T ? order_key(s[j]) : 0u;
+      const bool in = j < T && (key & mask) == prefix;
+      // lanes with the same digit add once (scores cluster in few bins)
+      const uint32_t bin = in ? ((key >> shift) & 255u) : 256u;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+      if (in && (__ffs(peers) - 1) == lane) atomicAdd(h + bin, uint32_t(__popc(peers)));
+    }
+    __syncwarp();
+    // lane L holds bins 255-8L .. 248-8L (lane 0 = highest digits)
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) cnt += h[255 - 8 * lane - b];
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, incl >= uint32_t(remaining));
+    const int L = __ffs(ballot) - 1;
+    uint32_t digit = 0;
+    int rem_new = 0;
+    if (lane == L) {
+      uint32_t run = incl - cnt;                      // keys with a higher digit
+      for (int b = 0; b < 8; ++b) {
+        const uint32_t bin = 255 - 8 * L - b;
+        if (run + h[bin] >= uint32_t(remaining)) {
+          digit = bin;
+          rem_new = remaining - int(run);
+          break;
+        }
+        run += h[bin];
+      }
+    }
+    digit = __shfl_sync(0xFFFFFFFFu, digit, L);
+    remaining = __shfl_sync(0xFFFFFFFFu, rem_new, L);
+    prefix |= digit << shift;
+    mask |= 255u << shift;
+    __syncwarp();
+  }
+  return make_uint2(prefix, uint32_t(remaining));
+}
+
+// Range-histogram bin of a score: floor((s - lo) * sc) clamped to [0, 255]
+// (monotone non-decreasing in s: a larger score never lands in a lower bin).
+__device__ __forceinline__ int range_bin(float s, float lo, float sc) {
+  return int(fminf(fmaxf((s - lo) * sc, 0.0f), 255.0f));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ vbar,
     int64_t n_bh, int T, int n_p, float scale, int k, float* __restrict__ o_coarse,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_score, float* __restrict__ scratch) {
-  constexpr int kWarps = NW;
-  constexpr int QB = kWarps * RW;
   constexpr int kStride = D + 4;
+  constexpr int CPL = D / 32;                 // output columns per lane in pass 3
+  constexpr int kQFloats = D * kQB, kPFloats = 2 * kQB * kPStride;
   extern __shared__ float4 smem4[];
   float* smem = reinterpret_cast<float*>(smem4);
-  float* qT = smem;                                   // [D][QB]; phase 3: P chunk [QB][kKC]
-  float* stage0 = qT + D * QB;                        // [2][kKC][kStride]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(stage0 + 2 * kKC * kStride);  // [kWarps][256]
+  // qT [D][QB] in pass 1, the two probability stages [2][QB][kPStride] in pass 3
+  float* qT = smem;
+  float* stage0 = qT + (kQFloats > kPFloats ? kQFloats : kPFloats);   // [2][kKC][kStride]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(stage0 + 2 * kKC * kStride);   // [kWarps][256]
+  uint32_t* cand = hist + kWarps * 256;                                       // [kWarps][32]
+  float* row_max = reinterpret_cast<float*>(cand + kWarps * 32);              // [QB]
   const int Tpad = (T + 3) & ~3;
-  float* sc = scratch + int64_t(blockIdx.x) * QB * Tpad;   // this CTA's score rows [QB][Tpad]
+  float* sc = scratch + int64_t(blockIdx.x) * kQB * Tpad;   // this CTA's score rows [QB][Tpad]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_blk = (T + QB - 1) / QB;
+  const int rg = lane >> 2, sub = lane & 3;   // row group (rows rg + 8i), key / column group
+  const int n_blk = (T + kQB - 1) / kQB;
   const int n_chunks = (T + kKC - 1) / kKC;
   const int n_v = T - n_p;
   const uint32_t lt_mask = (1u << lane) - 1u;
 
   for (int64_t item = blockIdx.x; item < n_bh * n_blk; item += gridDim.x) {
     const int64_t bh = item / n_blk;
-    const int i0 = int(item % n_blk) * QB;
+    const int i0 = int(item % n_blk) * kQB;
     const float* kb = kbar + bh * int64_t(T) * D;
     const float* vb = vbar + bh * int64_t(T) * D;
-    __syncthreads();     // the previous item is done with qT and the stages
+    __syncthreads();     // the previous item is done with every shared buffer
 
     {
-      // transposed query block: qT[d][r] (rows past T are zero)
-      constexpr int kNVec = QB * D / 4;
-      constexpr int kVec = (kNVec + kWarps * 32 - 1) / (kWarps * 32);
+      // transposed query block: qT[d][4 * (r % 8) + r / 8] (rows past T are zero),
+      // so that a lane's four rows rg + 8i are one 16-byte word per dimension
+      constexpr int kNVec = kQB * D / 4;
       const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * T + i0) * D);
-#pragma unroll
-      for (int u = 0; u < kVec; ++u) {
-        const int idx = threadIdx.x + u * kWarps * 32;
-        if (idx >= kNVec) continue;
-        const float4 v = i0 + idx / (D / 4) < T ? __ldg(q4 + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int idx = threadIdx.x; idx < kNVec; idx += kWarps * 32) {
         const int r = idx / (D / 4), d = (idx % (D / 4)) * 4;
-        qT[(d + 0) * QB + r] = v.x;
-        qT[(d + 1) * QB + r] = v.y;
-        qT[(d + 2) * QB + r] = v.z;
-        qT[(d + 3) * QB + r] = v.w;
+        const float4 v = i0 + r < T ? __ldg(q4 + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int pos = 4 * (r & 7) + (r >> 3);
+        qT[(d + 0) * kQB + pos] = v.x;
+        qT[(d + 1) * kQB + pos] = v.y;
+        qT[(d + 2) * kQB + pos] = v.z;
+        qT[(d + 3) * kQB + pos] = v.w;
       }
     }
 
     // ---- 1. scores (double-buffered key stages), written to the scratch rows
-    stage_rows_async<D, NW>(stage0, kb, min(kKC, T));
+    stage_rows_async<D>(stage0, kb, min(kKC, T));
     for (int c = 0; c < n_chunks; ++c) {
       const int j0 = c * kKC;
       const int nj = min(kKC, T - j0);
-      float* stage = stage0 + (c & 1) * kKC * kStride;
+      const float* stage = stage0 + (c & 1) * kKC * kStride;
       if (c + 1 < n_chunks) {
-        stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, kb + int64_t(j0 + kKC) * D,
-                                min(kKC, T - j0 - kKC));
+        stage_rows_async<D>(stage0 + ((c + 1) & 1) * kKC * kStride, kb + int64_t(j0 + kKC) * D,
+                            min(kKC, T - j0 - kKC));
         cp_async_wait<1>();
       } else {
         cp_async_wait<0>();
       }
       __syncthreads();
-      constexpr int KPL = kKC / 32;                  // keys per lane: lane, lane + 32, ...
-      float acc[RW][KPL];
+      const int jl = 8 * warp + 2 * sub;             // this lane's two keys: jl, jl + 1
+      float acc[4][2];
 #pragma unroll
-      for (int r = 0; r < RW; ++r)
-#pragma unroll
-        for (int u = 0; u < KPL; ++u) acc[r][u] = 0.f;
-      const float* qw = qT + warp * RW;
+      for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
+      const float* k0 = stage + jl * kStride;
+      const float* qg = qT + 4 * rg;
 #pragma unroll 4
       for (int d4 = 0; d4 < D / 4; ++d4) {
-        float av[KPL][4];
-#pragma unroll
-        for (int u = 0; u < KPL; ++u) {
-          const float4 a = reinterpret_cast<const float4*>(stage + (lane + 32 * u) * kStride)[d4];
-          av[u][0] = a.x;
-          av[u][1] = a.y;
-          av[u][2] = a.z;
-          av[u][3] = a.w;
-        }
+        const float4 a = reinterpret_cast<const float4*>(k0)[d4];
+        const float4 b = reinterpret_cast<const float4*>(k0 + kStride)[d4];
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          float q[RW];
-          QVec<RW>::load(qw + (4 * d4 + e) * QB, q);
+          const float4 q = *reinterpret_cast<const float4*>(qg + (4 * d4 + e) * kQB);
+          const float qv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-          for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int u = 0; u < KPL; ++u) acc[r][u] = fmaf(q[r], av[u][e], acc[r][u]);
+          for (int i = 0; i < 4; ++i) {
+            acc[i][0] = fmaf(qv[i], av[e], acc[i][0]);
+            acc[i][1] = fmaf(qv[i], bv[e], acc[i][1]);
+          }
         }
       }
+      if (jl < nj) {
 #pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        float* row = sc + (warp * RW + r) * Tpad + j0;
-#pragma unroll
-        for (int u = 0; u < KPL; ++u)
-          if (lane + 32 * u < nj) row[lane + 32 * u] = scale * acc[r][u];
+        for (int i = 0; i < 4; ++i) {
+          float* row = sc + (rg + 8 * i) * Tpad + j0 + jl;
+          if (jl + 1 < nj)
+            *reinterpret_cast<float2*>(row) = make_float2(scale * acc[i][0], scale * acc[i][1]);
+          else
+            row[0] = scale * acc[i][0];
+        }
       }
       __syncthreads();     // stage (c & 1) is refilled two chunks later
     }
 
-    // ---- 2. per row of this warp: the scores copied from the scratch row
-    // into a shared-memory row buffer of the warp (in the key stages, free
-    // now) when they fit, then the top-k over the video key tiles (video
-    // query tiles only) and the softmax, whose P goes back to the scratch row
+    // ---- 2. per row of this warp: the row max (for the softmax) and, for
+    // video query tiles, the top-k over the video key tiles.  The row is
+    // copied from the scratch into a shared-memory row buffer of the warp (in
+    // the key stages, free now) when it fits.
     uint32_t* h = hist + warp * 256;
+    uint32_t* cw = cand + warp * 32;
     const bool row_in_smem = size_t(kWarps) * Tpad <= size_t(2) * kKC * kStride;
-    float inv_l[RW];
-    for (int r = 0; r < RW; ++r) {
-      const int i = i0 + warp * RW + r;
-      float* srow = sc + (warp * RW + r) * Tpad;                 // global
-      float* s = row_in_smem ? stage0 + warp * Tpad : srow;     // where the passes read
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+      const int r = warp * kRowsPerWarp + rr;
+      const int i = i0 + r;
+      const float* srow = sc + r * Tpad;                         // global
+      const float* s = srow;
       if (row_in_smem) {
+        float* buf = stage0 + warp * Tpad;
         for (int j4 = lane; j4 < Tpad / 4; j4 += 32)
-          reinterpret_cast<float4*>(s)[j4] = reinterpret_cast<const float4*>(srow)[j4];
+          reinterpret_cast<float4*>(buf)[j4] = reinterpret_cast<const float4*>(srow)[j4];
         __syncwarp();
+        s = buf;
       }
+      // row max over all T tiles; min and max over the video tiles
+      float m = -INFINITY, vlo = INFINITY, vhi = -INFINITY;
+      for (int j = lane; j < T; j += 32) {
+        const float v = s[j];
+        m = fmaxf(m, v);
+        if (j >= n_p) {
+          vlo = fminf(vlo, v);
+          vhi = fmaxf(vhi, v);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+        vlo = fminf(vlo, __shfl_xor_sync(0xFFFFFFFFu, vlo, off));
+        vhi = fmaxf(vhi, __shfl_xor_sync(0xFFFFFFFFu, vhi, off));
+      }
+      if (lane == 0) row_max[r] = i < T ? m : 0.f;
       if (i < T && i >= n_p && k > 0) {
-        uint32_t prefix = 0u, mask = 0u;
-        int remaining = k;
-        for (int pass = 0; pass < 4; ++pass) {
-          const int shift = 24 - 8 * pass;
+        uint32_t kstar = 0u;
+        int remaining = 0;
+        bool found = false;
+        const float range = vhi - vlo;
+        const float bsc = 256.0f / range;
+        if (range > 0.0f && range < INFINITY && bsc < INFINITY) {
+          // one histogram over the value range
 #pragma unroll
           for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
           __syncwarp();
-          for (int jb = n_p; jb < T; jb += 32) {
-            const int j = jb + lane;
-            const uint32_t key = j < T ? order_key(s[j]) : 0u;
-            const bool in = j < T && (key & mask) == prefix;
-            // lanes with the same digit add once (scores cluster in few bins)
-            const uint32_t bin = in ? ((key >> shift) & 255u) : 256u;
-            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-            if (in && (__ffs(peers) - 1) == lane) atomicAdd(h + bin, uint32_t(__popc(peers)));
-          }
+          for (int j = n_p + lane; j < T; j += 32) atomicAdd(h + range_bin(s[j], vlo, bsc), 1u);
           __syncwarp();
-          // lane L holds bins 255-8L .. 248-8L (lane 0 = highest digits)
+          // lane L holds bins 255-8L .. 248-8L (lane 0 = highest scores)
           uint32_t cnt = 0;
 #pragma unroll
           for (int b = 0; b < 8; ++b) cnt += h[255 - 8 * lane - b];
@@ -263,29 +301,63 @@ __global__ void __launch_bounds__(NW * 32, VSA_COARSE_CTAS) coarse_topk_kernel(
             const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
             if (lane >= off) incl += o;
           }
-          const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, incl >= uint32_t(remaining));
-          const int L = __ffs(ballot) - 1;
-          uint32_t digit = 0;
-          int rem_new = 0;
+          const int L = __ffs(__ballot_sync(0xFFFFFFFFu, incl >= uint32_t(k))) - 1;
+          int bstar = 0, above = 0, in_bin = 0;
           if (lane == L) {
-            uint32_t run = incl - cnt;                      // keys with a higher digit
+            uint32_t run = incl - cnt;                  // scores in higher bins
             for (int b = 0; b < 8; ++b) {
-              const uint32_t bin = 255 - 8 * L - b;
-              if (run + h[bin] >= uint32_t(remaining)) {
-                digit = bin;
-                rem_new = remaining - int(run);
+              const int bin = 255 - 8 * L - b;
+              if (run + h[bin] >= uint32_t(k)) {
+                bstar = bin;
+                above = int(run);
+                in_bin = int(h[bin]);
                 break;
               }
               run += h[bin];
             }
           }
-          digit = __shfl_sync(0xFFFFFFFFu, digit, L);
-          remaining = __shfl_sync(0xFFFFFFFFu, rem_new, L);
-          prefix |= digit << shift;
-          mask |= 255u << shift;
-          __syncwarp();
+          bstar = __shfl_sync(0xFFFFFFFFu, bstar, L);
+          above = __shfl_sync(0xFFFFFFFFu, above, L);
+          in_bin = __shfl_sync(0xFFFFFFFFu, in_bin, L);
+          if (in_bin <= 32) {
+            // the scores of bin b*, compacted; the k-th largest is among them
+            int base = 0;
+            for (int jb = n_p; jb < T; jb += 32) {
+              const int j = jb + lane;
+              const float v = j < T ? s[j] : 0.f;
+              const bool in = j < T && range_bin(v, vlo, bsc) == bstar;
+              const uint32_t b = __ballot_sync(0xFFFFFFFFu, in);
+              if (in) cw[base + __popc(b & lt_mask)] = order_key(v);
+              base += __popc(b);
+            }
+            __syncwarp();
+            const int need = k - above;                 // 1 <= need <= in_bin
+            uint32_t key = 0u;
+            int gt = 0, eq = 0;
+            if (lane < in_bin) {
+              key = cw[lane];
+              for (int u = 0; u < in_bin; ++u) {
+                const uint32_t o = cw[u];
+                gt += o > key ? 1 : 0;
+                eq += o == key ? 1 : 0;
+              }
+            }
+            const uint32_t hit = __ballot_sync(0xFFFFFFFFu, lane < in_bin && gt < need && need <= gt + eq);
+            if (hit != 0u) {
+              const int L2 = __ffs(hit) - 1;
+              kstar = __shfl_sync(0xFFFFFFFFu, key, L2);
+              remaining = need - __shfl_sync(0xFFFFFFFFu, gt, L2);
+              found = true;
+            }
+            __syncwarp();
+          }
         }
-        // prefix = K*, remaining = number of keys equal to K* to keep (lowest j first)
+        if (!found) {
+          const uint2 sel = radix_select(s, T, n_p, k, h, lane);
+          kstar = sel.x;
+          remaining = int(sel.y);
+        }
+        // keep every key > K* and the lowest-index `remaining` keys == K*
         int32_t* out_idx = topk_idx + ((bh * n_v) + (i - n_p)) * int64_t(k);
         float* out_s = topk_score ? topk_score + ((bh * n_v) + (i - n_p)) * int64_t(k) : nullptr;
         int pos = 0, eq_seen = 0;
@@ -294,8 +366,8 @@ __global__ void __launch_bounds__(NW * 32, VSA_COARSE_CTAS) coarse_topk_kernel(
           const bool valid = j < T;
           const float sv = valid ? s[j] : 0.f;
           const uint32_t key = valid ? order_key(sv) : 0u;
-          const bool gt = valid && key > prefix;
-          const bool eq = valid && key == prefix;
+          const bool gt = valid && key > kstar;
+          const bool eq = valid && key == kstar;
           const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
           const int eq_rank = eq_seen + __popc(eqb & lt_mask);
           const bool sel = gt || (eq && eq_rank < remaining);
@@ -309,97 +381,129 @@ __global__ void __launch_bounds__(NW * 32, VSA_COARSE_CTAS) coarse_topk_kernel(
           eq_seen += __popc(eqb);
         }
       }
-      // ---- 3a. softmax of the row; P to the scratch row
-      float m = -INFINITY;
-      for (int j = lane; j < T; j += 32) m = fmaxf(m, s[j]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-      float l = 0.f;
-      for (int j = lane; j < T; j += 32) {
-        const float p = __expf(s[j] - m);
-        srow[j] = p;
-        l += p;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-      inv_l[r] = 1.0f / l;
       __syncwarp();        // the row buffer is refilled for the next row
     }
 
-    // ---- 3b. o_coarse = P V / l: P chunks staged into shared memory next to
-    // the value chunks
-    float acc[RW][D / 32];
+    // ---- 3. o_coarse = sum_j p[r][j] vbar_j / sum_j p[r][j], p = exp(s - max):
+    // p made while staging (thread t: row t / 8, eight tiles from 8 (t % 8)),
+    // value chunks staged by cp.async beside them
+    __syncthreads();     // row maxima written; qT and the row buffers free
+    float* pst = qT;     // [2][QB][kPStride]
+    const int pr_row = threadIdx.x >> 3, pr_col = (threadIdx.x & 7) * 8;
+    float pv[8];
+    auto load_p = [&](int j0) {
 #pragma unroll
-    for (int r = 0; r < RW; ++r)
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) acc[r][c] = 0.f;
-    __syncthreads();     // every P row written; qT no longer needed (P stage)
-    float* pst = qT;     // [2][QB][kKC]
-    auto stage_p = [&](int buf, int j0, int nj) {
-      // P[r][j0 .. j0 + nj) of all QB rows; 16-byte pieces (j0 and Tpad are
-      // multiples of 4; a ragged tail piece reads past nj into the row's
-      // padding, never past the scratch slot)
-      constexpr int kPieces = QB * (kKC / 4);
-      for (int idx = threadIdx.x; idx < kPieces; idx += kWarps * 32) {
-        const int r = idx / (kKC / 4), q4 = (idx % (kKC / 4)) * 4;
-        if (q4 >= nj) continue;
-        const uint32_t dst = static_cast<uint32_t>(
-            __cvta_generic_to_shared(pst + buf * QB * kKC + r * kKC + q4));
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-                     "l"(sc + r * Tpad + j0 + q4)
-                     : "memory");
+      for (int hh = 0; hh < 2; ++hh) {
+        const int j = j0 + pr_col + 4 * hh;
+        const float4 v = j < Tpad ? *reinterpret_cast<const float4*>(sc + pr_row * Tpad + j)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        pv[4 * hh + 0] = v.x;
+        pv[4 * hh + 1] = v.y;
+        pv[4 * hh + 2] = v.z;
+        pv[4 * hh + 3] = v.w;
       }
     };
-    stage_p(0, 0, min(kKC, T));
-    stage_rows_async<D, NW>(stage0, vb, min(kKC, T));
+    auto store_p = [&](int buf, int j0) {
+      const float mr = row_max[pr_row];
+      float e[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) e[u] = j0 + pr_col + u < T ? __expf(pv[u] - mr) : 0.f;
+      float4* dst = reinterpret_cast<float4*>(pst + buf * kQB * kPStride + pr_row * kPStride + pr_col);
+      dst[0] = make_float4(e[0], e[1], e[2], e[3]);
+      dst[1] = make_float4(e[4], e[5], e[6], e[7]);
+    };
+    const int c0 = warp * 4 * CPL + sub * CPL;   // this lane's output columns
+    float acc[4][CPL], lsum[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lsum[i] = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[i][c] = 0.f;
+    }
+    load_p(0);
+    store_p(0, 0);
+    stage_rows_async<D>(stage0, vb, min(kKC, T));
     for (int c = 0; c < n_chunks; ++c) {
       const int j0 = c * kKC;
       const int nj = min(kKC, T - j0);
       const float* stage = stage0 + (c & 1) * kKC * kStride;
-      const float* pc = pst + (c & 1) * QB * kKC;
+      const float* pc = pst + (c & 1) * kQB * kPStride;
       if (c + 1 < n_chunks) {
-        stage_p((c + 1) & 1, j0 + kKC, min(kKC, T - j0 - kKC));
-        stage_rows_async<D, NW>(stage0 + ((c + 1) & 1) * kKC * kStride, vb + int64_t(j0 + kKC) * D,
-                                min(kKC, T - j0 - kKC));
+        stage_rows_async<D>(stage0 + ((c + 1) & 1) * kKC * kStride, vb + int64_t(j0 + kKC) * D,
+                            min(kKC, T - j0 - kKC));
+        load_p(j0 + kKC);
         cp_async_wait<1>();
       } else {
         cp_async_wait<0>();
       }
-      __syncthreads();
-      for (int jj = 0; jj < nj; ++jj) {
-        float v[D / 32];
+      __syncthreads();     // value chunk c landed, probability chunk c stored
+      const float* pr = pc + rg * kPStride;
+      const int nj4 = nj & ~3;
+      for (int jj = 0; jj < nj4; jj += 4) {
+        float p[4][4];
 #pragma unroll
-        for (int c2 = 0; c2 < D / 32; ++c2) v[c2] = stage[jj * kStride + lane + 32 * c2];
+        for (int i = 0; i < 4; ++i) {
+          const float4 t = *reinterpret_cast<const float4*>(pr + 8 * i * kPStride + jj);
+          p[i][0] = t.x;
+          p[i][1] = t.y;
+          p[i][2] = t.z;
+          p[i][3] = t.w;
+        }
 #pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          const float p = pc[(warp * RW + r) * kKC + jj];
+        for (int e = 0; e < 4; ++e) {
+          float v[CPL];
+          if constexpr (CPL == 4) {
+            const float4 t = *reinterpret_cast<const float4*>(stage + (jj + e) * kStride + c0);
+            v[0] = t.x;
+            v[1] = t.y;
+            v[2] = t.z;
+            v[3] = t.w;
+          } else {
+            const float2 t = *reinterpret_cast<const float2*>(stage + (jj + e) * kStride + c0);
+            v[0] = t.x;
+            v[1] = t.y;
+          }
 #pragma unroll
-          for (int c2 = 0; c2 < D / 32; ++c2) acc[r][c2] = fmaf(p, v[c2], acc[r][c2]);
+          for (int i = 0; i < 4; ++i) {
+            lsum[i] += p[i][e];
+#pragma unroll
+            for (int cc = 0; cc < CPL; ++cc) acc[i][cc] = fmaf(p[i][e], v[cc], acc[i][cc]);
+          }
         }
       }
-      __syncthreads();
+      for (int jj = nj4; jj < nj; ++jj) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float pp = pr[8 * i * kPStride + jj];
+          lsum[i] += pp;
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc)
+            acc[i][cc] = fmaf(pp, stage[jj * kStride + c0 + cc], acc[i][cc]);
+        }
+      }
+      if (c + 1 < n_chunks) store_p((c + 1) & 1, j0 + kKC);
+      __syncthreads();     // both stages of chunk c are refilled one chunk later
     }
 #pragma unroll
-    for (int r = 0; r < RW; ++r) {
-      const int i = i0 + warp * RW + r;
-      if (i >= T) continue;
-      float* oc = o_coarse + (bh * T + i) * D;
+    for (int i = 0; i < 4; ++i) {
+      const int r = rg + 8 * i;
+      if (i0 + r >= T) continue;
+      float* oc = o_coarse + (bh * T + i0 + r) * D + c0;
+      const float inv = 1.0f / lsum[i];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) oc[lane + 32 * c] = acc[r][c] * inv_l[r];
+      for (int cc = 0; cc < CPL; ++cc) oc[cc] = acc[i][cc] * inv;
     }
   }
 }
 
-constexpr int kCoarseWarps = VSA_COARSE_WARPS, kCoarseRows = VSA_COARSE_ROWS;   // QB = 32 query tiles per item
-constexpr int kCoarseQB = kCoarseWarps * kCoarseRows;
-
 template <int D>
 size_t coarse_smem_bytes() {
-  // qT [D][QB] (reused as two P stages [QB][kKC]), two key / value stages,
-  // the per-warp histograms
-  const size_t q = size_t(D) * kCoarseQB;
-  const size_t p = size_t(2) * kCoarseQB * kKC;
-  return sizeof(float) * ((q > p ? q : p) + size_t(2) * kKC * (D + 4) + size_t(kCoarseWarps) * 256);
+  // qT [D][QB] (reused as two probability stages [QB][kPStride]), two key /
+  // value stages, the per-warp histograms and candidate lists, the row maxima
+  const size_t q = size_t(D) * kQB;
+  const size_t p = size_t(2) * kQB * kPStride;
+  return sizeof(float) * ((q > p ? q : p) + size_t(2) * kKC * (D + 4) + size_t(kWarps) * (256 + 32) +
+                          kQB);
 }
 
 template <int D>
@@ -407,10 +511,10 @@ cudaError_t launch_coarse_d(const float* qbar, const float* kbar, const float* v
                             int T, int n_p, float scale, int k, float* o_coarse, int32_t* topk_idx,
                             float* topk_score, float* scratch, int grid, cudaStream_t stream) {
   const size_t smem = coarse_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(coarse_topk_kernel<D, kCoarseWarps, kCoarseRows>,
+  cudaError_t e = cudaFuncSetAttribute(coarse_topk_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  coarse_topk_kernel<D, kCoarseWarps, kCoarseRows><<<grid, kCoarseWarps * 32, smem, stream>>>(
+  coarse_topk_kernel<D><<<grid, kWarps * 32, smem, stream>>>(
       qbar, kbar, vbar, bh, T, n_p, scale, k, o_coarse, topk_idx, topk_score, scratch);
   return cudaGetLastError();
 }
@@ -500,7 +604,7 @@ cudaError_t launch_select_ref(const float* qbar, const float* kbar, int64_t bh, 
 int coarse_grid(int num_sms) { return VSA_COARSE_CTAS * (num_sms > 0 ? num_sms : 148); }
 
 size_t coarse_scratch_bytes(int T, int num_sms) {
-  return sizeof(float) * size_t(coarse_grid(num_sms)) * kCoarseQB * size_t((T + 3) & ~3);
+  return sizeof(float) * size_t(coarse_grid(num_sms)) * kQB * size_t((T + 3) & ~3);
 }
 
 cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float* vbar, int64_t bh,
@@ -508,7 +612,7 @@ cudaError_t launch_coarse_topk(const float* qbar, const float* kbar, const float
                                int32_t* topk_idx, float* topk_score, float* scratch, int num_sms,
                                cudaStream_t stream) {
   if (T > kMaxTiles) return cudaErrorInvalidValue;
-  const int64_t items = bh * ((T + kCoarseQB - 1) / kCoarseQB);
+  const int64_t items = bh * ((T + kQB - 1) / kQB);
   if (items == 0) return cudaSuccess;
   const int grid = int(std::min<int64_t>(items, coarse_grid(num_sms)));
   if (D == 128)
