@@ -8,17 +8,24 @@
 //   fp32 accumulation in TMEM, round to nearest even on the store.
 //
 // Design (one persistent CTA per SM, static round-robin over output tiles of
-// 128 rows (tokens) x 256 columns (H*D), M-major so that concurrent CTAs
+// 256 rows (tokens) x 256 columns (H*D), M-major so that concurrent CTAs
 // share the x rows and all of W in L2):
-//   warp 0  (TMA)       per 64-wide K block, the x box [128 x 64] and the W box
-//                       [256 x 64] (128-byte swizzle) into a 4-stage ring.
+//   warp 0  (TMA)       per 64-wide K block, the x box [256 x 64] and the W box
+//                       [256 x 64] (128-byte swizzle) into a 3-stage ring.
 //   warp 1  (MMA)       one lane issues tcgen05.mma kind::f16, M=128, N=256,
-//                       K=16 (four per K block) into one of two TMEM
-//                       accumulators (2 x 256 columns), so that the epilogue of a
-//                       tile overlaps the MMAs of the next.
-//   warps 2-5 (epilogue) thread = accumulator row = TMEM lane: 32-column
-//                       tcgen05.ld chunks, optional sigmoid, bf16 pack, 16-byte
-//                       stores into the row's per-head segments.
+//                       K=16, two per K step (rows 0-127 and 128-255 of the
+//                       tile against the same W box), into one TMEM
+//                       accumulator of 2 x 256 columns.  A 256 x 256 tile reads
+//                       a third fewer operand bytes per FLOP from L2 than
+//                       128 x 256 (which bound the earlier kernel), at the
+//                       price of a single accumulator.
+//   warps 2-9 (epilogue) thread = accumulator row = TMEM lane (warps 2-5 rows
+//                       0-127, warps 6-9 rows 128-255): the row's 256 columns
+//                       are read with tcgen05.ld in 32-column chunks, passed
+//                       through the optional sigmoid and packed to bf16 in
+//                       registers; the accumulator is handed back to the MMA
+//                       warp before the 16-byte stores into the row's per-head
+//                       segments, so the stores overlap the next tile's MMAs.
 // Every mbarrier wait is bounded (abort flag + status word, as in the
 // attention kernel); rows past B*N and columns past H*D are loaded as zeros by
 // TMA and never stored.
@@ -29,14 +36,15 @@ namespace vsa {
 namespace {
 using namespace sm100;
 
-constexpr int kPBM = 128, kPBN = 256, kPBK = 64, kPStages = 4;
-constexpr int kPThreads = 192;                  // TMA, MMA, 4 epilogue warps
-constexpr int kPABytes = kPBM * kPBK * 2;      // 16 KB
+constexpr int kPBM = 256, kPBN = 256, kPBK = 64, kPStages = 3;
+constexpr int kPThreads = 320;                  // TMA, MMA, 8 epilogue warps
+constexpr int kPABytes = kPBM * kPBK * 2;      // 32 KB
 constexpr int kPBBytes = kPBN * kPBK * 2;      // 32 KB
 constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr uint32_t kPIdesc = idesc_bf16(kPBM, kPBN, false, false);
-// barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
-constexpr int kPNBar = 2 * kPStages + 5;
+constexpr int kPHalfA = 128 * kPBK * 2;        // byte offset of rows 128-255 in the x box
+constexpr uint32_t kPIdesc = idesc_bf16(128, kPBN, false, false);
+// barriers: full[S], empty[S], acc_full, acc_empty, drain
+constexpr int kPNBar = 2 * kPStages + 3;
 constexpr size_t kPSmem = size_t(kPStages) * kPStageBytes + kPNBar * 8 + 16 + 1024;
 
 struct ProjArgs {
@@ -66,7 +74,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   // full/empty complete once per K block, acc_full/acc_empty once per use of
   // the accumulator; each waiter observes every phase in order
   const uint32_t full = bar0, empty = full + 8 * kPStages, acc_full = empty + 8 * kPStages,
-                 acc_empty = acc_full + 16, drain = acc_empty + 16;
+                 acc_empty = acc_full + 8, drain = acc_empty + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPStages * kPStageBytes + kPNBar * 8);
   volatile int* abort_flag =
       reinterpret_cast<volatile int*>(smem + kPStages * kPStageBytes + kPNBar * 8 + 4);
@@ -78,10 +86,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(full + 8 * s, 1);
       mbar_init(empty + 8 * s, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, 128);
-    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -136,9 +142,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       int lt = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
-        const int acc = lt & 1;
-        if (lt >= 2 &&
-            !wait_bar(acc_empty + 8 * acc, ((lt >> 1) - 1) & 1, abort_flag, a.status, 22)) {
+        // the accumulator of the previous tile has been read out
+        if (lt >= 1 && !wait_bar(acc_empty, (lt - 1) & 1, abort_flag, a.status, 22)) {
           ok = false;
           break;
         }
@@ -153,13 +158,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
           const uint32_t sa = s_base + s * kPStageBytes;
 #pragma unroll
           for (int ks = 0; ks < kPBK / 16; ++ks) {
-            const uint64_t ad = sdesc_sw128(sa + ks * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(sa + kPABytes + ks * 32, 16, 1024);
-            umma_bf16(tmem + acc * kPBN, ad, bd, kPIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            const uint32_t accum = (kb > 0 || ks > 0) ? 1u : 0u;
+            umma_bf16(tmem, sdesc_sw128(sa + ks * 32, 16, 1024), bd, kPIdesc, accum);
+            umma_bf16(tmem + kPBN, sdesc_sw128(sa + kPHalfA + ks * 32, 16, 1024), bd, kPIdesc,
+                      accum);
           }
           umma_commit(empty + 8 * s);
         }
-        if (ok) umma_commit(acc_full + 8 * acc);
+        if (ok) umma_commit(acc_full);
       }
       // drain: every MMA issued above complete before TMEM is freed
       umma_commit(drain);
@@ -169,46 +176,48 @@ __global__ void __launch_bounds__(kPThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quad = warp & 3;                       // TMEM lane quadrant of this warp
-    const int row = quad * 32 + lane;
-    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
+    const int half = (warp - 2) >> 2;                // rows 0-127 or 128-255 of the tile
+    const int row = half * 128 + quad * 32 + lane;
+    const uint32_t t_row = tmem + (uint32_t(quad * 32) << 16) + uint32_t(half * kPBN);
     int lt = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
-      const int acc = lt & 1;
       const int m = t / a.n_tiles, n = t % a.n_tiles;
-      if (!__all_sync(0xFFFFFFFFu,
-                      wait_bar(acc_full + 8 * acc, (lt >> 1) & 1, abort_flag, a.status, 24)))
-        break;
+      if (!__all_sync(0xFFFFFFFFu, wait_bar(acc_full, lt & 1, abort_flag, a.status, 24))) break;
       tc_fence_after();
-      const int64_t r = int64_t(m) * kPBM + row;     // global row = b * N + token
-      const bool live = r < a.M;
-      const int64_t b = live ? r / a.N : 0, tok = live ? r % a.N : 0;
-#pragma unroll 1
+      // the row's 256 columns, packed to bf16 pairs in registers
+      uint32_t pk[kPBN / 2];
+#pragma unroll
       for (int c = 0; c < kPBN / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(t_lane + acc * kPBN + 32 * c, v);
+        tmem_ld32(t_row + 32 * c, v);
         tmem_wait_ld(v);
-        const int col0 = n * kPBN + 32 * c;            // 32 columns within one head (D >= 64)
-        if (!live || col0 >= a.H * a.D) continue;
-        const int h = col0 / a.D, d0 = col0 % a.D;
-        uint4* dst = reinterpret_cast<uint4*>(a.y + ((b * a.H + h) * a.N + tok) * a.D + d0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            f[e] = __uint_as_float(v[8 * q + e]);
-            if (a.act == 1) f[e] = sigmoid_tanh(f[e]);
+        for (int e = 0; e < 16; ++e) {
+          float lo = __uint_as_float(v[2 * e]), hi = __uint_as_float(v[2 * e + 1]);
+          if (a.act == 1) {
+            lo = sigmoid_tanh(lo);
+            hi = sigmoid_tanh(hi);
           }
-          uint4 u;
-          u.x = pack_bf16(f[0], f[1]);
-          u.y = pack_bf16(f[2], f[3]);
-          u.z = pack_bf16(f[4], f[5]);
-          u.w = pack_bf16(f[6], f[7]);
-          dst[q] = u;
+          pk[16 * c + e] = pack_bf16(lo, hi);
         }
       }
       tc_fence_before();
-      mbar_arrive(acc_empty + 8 * acc);
+      mbar_arrive(acc_empty);                        // the MMAs of the next tile may start
+      const int64_t r = int64_t(m) * kPBM + row;     // global row = b * N + token
+      if (r < a.M) {
+        const int64_t b = r / a.N, tok = r % a.N;
+#pragma unroll
+        for (int c = 0; c < kPBN / 32; ++c) {
+          const int col0 = n * kPBN + 32 * c;          // 32 columns within one head (D >= 64)
+          if (col0 >= a.H * a.D) continue;
+          const int h = col0 / a.D, d0 = col0 % a.D;
+          uint4* dst = reinterpret_cast<uint4*>(a.y + ((b * a.H + h) * a.N + tok) * a.D + d0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pk[16 * c + 4 * q], pk[16 * c + 4 * q + 1], pk[16 * c + 4 * q + 2],
+                                pk[16 * c + 4 * q + 3]);
+        }
+      }
     }
   }
 
