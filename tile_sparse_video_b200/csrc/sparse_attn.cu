@@ -52,9 +52,12 @@
 // tiled layout, so one Q box loads both), and a step is a pair of key tiles
 // taken in ascending order from the union of the two query tiles' key sets.
 // Each entry of that list carries a mask of the query tiles whose set holds
-// it; the softmax warps of the other query tile treat its keys as masked, and
-// warps whose query tile holds neither key tile of a step write P = 0 without
-// exponentials.  A key tile both query tiles kept is loaded once for both.
+// it; the softmax warps of the other query tile set its scores to -inf in
+// registers, so that both query tiles run one branch-free path (row max,
+// exponentials, P) in which those keys count for nothing (measured on B200: 6 %
+// faster than skipping their exponentials on a separate path, whose code the
+// two halves of a pair then ran at once).  A key tile both query tiles kept is
+// loaded once for both.
 // The list is built per item by the K producer warp (two bitmaps over the T
 // tiles, then a ballot compaction) into one of two shared-memory slots that
 // the other roles read.
@@ -933,8 +936,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       // list (columns [0, 64) and [64, 128)); a key tile outside this half's
       // set counts as fully masked.  The protocol is the one of the 128-row
       // kernel below (one O, a reference max shared through the mailbox,
-      // lazy rescale).  Key tiles outside the set skip their exponentials and
-      // write P = 0.
+      // lazy rescale).  Key tiles outside the set enter as -inf scores (P = 0).
       VSA_TL_DECL;
       const int wg = warp >> 2;                            // 0 or 1
       const int quad = warp & 3;
@@ -994,12 +996,23 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           for (int c = 0; c < 4; ++c) tmem_wait_ld(r[c]);
           tc_fence_before();
           mbar_arrive(s_empty + 8 * wg);
-          // row max over raw scores (scale > 0 commutes with max), four chains;
-          // a key tile outside this half's set is left out
+          // a key tile outside this half's set: its scores become -inf in
+          // registers, so that the row max, the exponentials (exp2(-inf) = 0)
+          // and the row sums below run one branch-free code path for both
+          // query tiles of the pair
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            if (bl2[c2] == 0) {                              // warp-uniform
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[2 * c2 + h][e] = __float_as_uint(-INFINITY);
+            }
+          }
+          // row max over raw scores (scale > 0 commutes with max), four chains
           float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c2 = 0; c2 < 2; ++c2) {
-            if (bl2[c2] == 0) continue;                     // warp-uniform
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -1048,21 +1061,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 uint32_t pw[16];
-                if (bl2[c2] == 0) {
 #pragma unroll
-                  for (int e = 0; e < 16; ++e) pw[e] = 0u;
-                } else {
-#pragma unroll
-                  for (int e = 0; e < 32; e += 2) {
-                    float x0, x1;
-                    f2unpack(ffma2(f2pack(__uint_as_float(r[2 * c2 + h][e]),
-                                          __uint_as_float(r[2 * c2 + h][e + 1])),
-                                   sc2, nm2),
-                             x0, x1);
-                    const float p0 = ex2(x0), p1 = ex2(x1);
-                    acc2[(e >> 1) & 1] = fadd2(acc2[(e >> 1) & 1], f2pack(p0, p1));
-                    pw[e >> 1] = pack_bf16(p0, p1);
-                  }
+                for (int e = 0; e < 32; e += 2) {
+                  float x0, x1;
+                  f2unpack(ffma2(f2pack(__uint_as_float(r[2 * c2 + h][e]),
+                                        __uint_as_float(r[2 * c2 + h][e + 1])),
+                                 sc2, nm2),
+                           x0, x1);
+                  const float p0 = ex2(x0), p1 = ex2(x1);
+                  acc2[(e >> 1) & 1] = fadd2(acc2[(e >> 1) & 1], f2pack(p0, p1));
+                  pw[e >> 1] = pack_bf16(p0, p1);
                 }
                 tmem_st16(t_lane + col_p + 32 * c2 + 16 * h, pw);
               }
