@@ -163,6 +163,46 @@ def _check_layer(w: Workload, inp):
     assert torch.equal(vsa.vsa_unpermute(plan, out_t), out)
 
 
+@pytest.mark.parametrize("law", ["three_keys", "one_key", "quantised"])
+def test_topk_heavy_ties(law):
+    """Selections whose k-th score sits among many equal scores, against the
+    oracle's (score descending, index ascending) order, which is unique here,
+    so the kept tiles must match exactly.  three_keys: every pooled key is one
+    of three vectors (about 50 equal scores per value in a row of 153 key
+    tiles, more than the range histogram's 32-candidate bin, so the exact
+    radix select decides); one_key: every score of a row equal (a zero range);
+    quantised: one-hot pooled queries against keys on an 1/8 grid (8 distinct
+    scores per row, the candidate ranking inside one histogram bin decides
+    among equal scores).  Equal pooled keys give equal fp32 and fp64 scores,
+    and distinct grid values stay ordered, so rounding cannot move a tie."""
+    w = SMALL
+    B, H, D = 1, 2, w.D
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    T = p.n_tiles
+    k = plan.keep_count(keep_tiles=40)
+    g = torch.Generator().manual_seed(4242)
+    q = torch.randn(B, H, T, D, generator=g)
+    v = torch.randn(B, H, T, D, generator=g)
+    if law == "three_keys":
+        kk = torch.randn(3, D, generator=g)[torch.randint(0, 3, (B, H, T), generator=g)]
+    elif law == "one_key":
+        kk = torch.randn(D, generator=g).expand(B, H, T, D).contiguous()
+    else:
+        q = torch.zeros(B, H, T, D)
+        q[..., 0] = 1.0
+        kk = torch.randn(B, H, T, D, generator=g)
+        kk[..., 0] = torch.randint(0, 8, (B, H, T), generator=g).float() / 8
+    ws = torch.zeros(plan.workspace_size(B, H, D, k), dtype=torch.uint8, device="cuda")
+    for slot, x in zip(vsa.pooled_slots(plan, ws, B, H, D), (q, kk, v)):
+        slot.copy_(x.cuda())
+    oc, idx, _ = vsa.vsa_coarse_topk_pooled(plan, B, H, D, k, ws)
+    s, oc_ref = O.coarse_attention(q.double().numpy(), kk.double().numpy(), v.double().numpy(), D ** -0.5)
+    assert np.array_equal(idx.cpu().numpy().astype(np.int64), O.select_topk(s, p, k))
+    np.testing.assert_allclose(f64(oc), oc_ref, rtol=1e-4, atol=1e-5)
+    vsa.vsa_sync_status(plan)
+
+
 def test_keep_all_equals_dense_attention():
     """k = every video tile: the fine output is plain dense attention over all
     real tokens (torch's own routine, fp32 on the GPU)."""
