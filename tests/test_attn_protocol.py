@@ -20,11 +20,18 @@ random) and checks:
 * O is rescaled only while no PV product is in flight, read by the epilogue only
   after the item's last PV, and restarted (first PV of an item) only after the
   previous epilogue has read it;
+* the item of each step is handed out through two list slots: the K producer
+  takes it (from the grid's work counter) and publishes it in slot t % 2
+  (list_full), every other role reads it there, and the slot is rewritten only
+  after all twelve roles released the item it held two items earlier
+  (list_empty); a role must never read a stale or rewritten slot, and the end
+  marker (-1) stops every role;
 * the 256-thread group barriers match, and the run ends (no deadlock).
 
 Planted mistakes (P written without waiting for the warpgroup's previous PV, S
 issued without waiting for the warpgroup to have loaded its previous S, O
-rescaled without waiting for the partner's PV) must be caught.
+rescaled without waiting for the partner's PV, a list slot rewritten without
+waiting for its readers) must be caught.
 """
 import random
 
@@ -56,6 +63,9 @@ class Model:
             self.need[f"pv_done{w}"] = 1
         for q in range(4):
             self.need[f"dec{q}"] = 1
+        for sl in range(2):
+            self.need[f"list_full{sl}"] = 1
+            self.need[f"list_empty{sl}"] = 12   # K, V, S issuer, PV issuer, 8 softmax warps
         for b in self.need:
             self.done[b] = 0
             self.count[b] = 0
@@ -68,6 +78,8 @@ class Model:
         self.mbox_read = set()       # (quadrant, global tile) values consumed
         self.epi = {}                # item -> warps done with the epilogue
         self.item_first = []         # global index of each item's first tile
+        self.slot = [None, None]     # item published in each list slot (-1: none left)
+        self.released = {}           # item -> roles that released its list slot
         G = 0
         for nk in items:
             self.item_first.append(G)
@@ -83,10 +95,34 @@ class Model:
     def ready(self, b, k):
         return self.done[b] >= k + 1
 
+    # ---------------------------------------------------------------- list slots
+    def publish(self, t):
+        """K producer: item t (or the end marker) into slot t % 2."""
+        if t >= 2:
+            if "list_early" not in self.plant:
+                yield ("wait", f"list_empty{t & 1}", (t >> 1) - 1)
+            if len(self.released.get(t - 2, ())) < 12:
+                raise Violation(f"list slot {t & 1} rewritten with item {t} while item {t - 2} is still "
+                                f"being read ({12 - len(self.released.get(t - 2, ()))} roles)")
+        self.slot[t & 1] = t if t < len(self.items) else -1
+        self.arrive(f"list_full{t & 1}")
+
+    def read_slot(self, who, t):
+        """A reader: wait for slot t % 2 and check that it holds item t."""
+        yield ("wait", f"list_full{t & 1}", t >> 1)
+        want = t if t < len(self.items) else -1
+        if self.slot[t & 1] != want:
+            raise Violation(f"{who} read item {self.slot[t & 1]} from slot {t & 1}, expected {want}")
+
+    def release(self, who, t):
+        self.released.setdefault(t, set()).add(who)
+        self.arrive(f"list_empty{t & 1}")
+
     # ---------------------------------------------------------------- actors
     def k_producer(self):
         g = 0
         for t, nk in enumerate(self.items):
+            yield from self.publish(t)
             if t > 0:
                 yield ("wait", "q_empty", t - 1)
                 first = self.item_first[t - 1]
@@ -101,10 +137,15 @@ class Model:
                         raise Violation(f"K slot {s} refilled before the S product of tile {g - self.NSK} read it")
                 self.fifo["tk"].append(("k", s, g))
                 g += 1
+            self.release("kp", t)
+        yield from self.publish(len(self.items))
 
     def v_producer(self):
         g = 0
-        for nk in self.items:
+        for t, nk in enumerate(self.items + [None]):
+            yield from self.read_slot("vp", t)
+            if nk is None:
+                return
             for n in range(nk):
                 s = g % self.NSV
                 if g >= self.NSV:
@@ -113,12 +154,17 @@ class Model:
                         raise Violation(f"V slot {s} refilled before the PV product of tile {g - self.NSV} read it")
                 self.fifo["tv"].append(("v", s, g))
                 g += 1
+            self.release("vp", t)
 
     def s_issuer(self):
         gk = 0
         si = [0, 0]
         last_of_w = [None, None]
-        for t, nk in enumerate(self.items):
+        for t, nk in enumerate(self.items + [None]):
+            yield from self.read_slot("si", t)
+            if nk is None:
+                return
+            self.release("si", t)
             yield ("wait", "q_full", t)
             for n in range(nk):
                 w = n & 1
@@ -137,7 +183,11 @@ class Model:
     def pv_issuer(self):
         gv = 0
         pf = [0, 0]
-        for t, nk in enumerate(self.items):
+        for t, nk in enumerate(self.items + [None]):
+            yield from self.read_slot("pvi", t)
+            if nk is None:
+                return
+            self.release("pvi", t)
             for n in range(nk):
                 w = n & 1
                 if n == 0 and t > 0:
@@ -155,7 +205,10 @@ class Model:
     def softmax_warp(self, wg, q):
         cw = 0
         cnt = [0, 0]
-        for t, nk in enumerate(self.items):
+        for t, nk in enumerate(self.items + [None]):
+            yield from self.read_slot(f"sm{wg}{q}", t)
+            if nk is None:
+                return
             G = self.item_first[t]
             yield ("bar",)
             yield ("bar",)
@@ -204,6 +257,7 @@ class Model:
             yield ("bar",)
             self.epi.setdefault(t, set()).add((wg, q))
             self.arrive("o_empty")
+            self.release(f"sm{wg}{q}", t)
 
     def tile_wg(self, x):
         for t, first in enumerate(self.item_first):
@@ -300,7 +354,7 @@ def test_attention_protocol_holds_under_random_schedules(items, NSK, NSV):
         Model(items, NSK=NSK, NSV=NSV, seed=seed).run()
 
 
-@pytest.mark.parametrize("plant", ["p_early", "s_issue_early", "rescale_early"])
+@pytest.mark.parametrize("plant", ["p_early", "s_issue_early", "rescale_early", "list_early"])
 def test_planted_attention_mistakes_are_caught(plant):
     caught = 0
     for seed in range(150):
