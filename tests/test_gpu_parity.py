@@ -203,6 +203,50 @@ def test_topk_heavy_ties(law):
     vsa.vsa_sync_status(plan)
 
 
+def test_topk_non_finite_scores_stay_valid():
+    """Pooled means holding NaN and +-inf (whole key rows of NaN, keys with
+    infinite entries, a query row of NaN): the selection is still k distinct
+    video tile indices per row in ascending order, nothing is recorded in the
+    status word, and rows without a non-finite score match the oracle.  A NaN
+    score ranks by its order key (the exact radix select), so the keep pass
+    never selects more than k."""
+    w = SMALL
+    B, H, D = 1, 2, w.D
+    plan = vsa.Plan(w.prefix, w.grid, w.tile)
+    p = O.plan(w.prefix, w.grid, w.tile)
+    T, n_p = p.n_tiles, p.n_prefix_tiles
+    k = plan.keep_count(keep_tiles=40)
+    g = torch.Generator().manual_seed(515)
+    q = torch.randn(B, H, T, D, generator=g)
+    kk = torch.randn(B, H, T, D, generator=g)
+    v = torch.randn(B, H, T, D, generator=g)
+    # head 0: a NaN key row, keys with +-inf entries (+-inf or NaN scores);
+    # head 1: one NaN query row, every other row finite
+    kk[0, 0, n_p + 3] = float("nan")
+    kk[0, 0, n_p + 10, 5] = float("inf")
+    kk[0, 0, n_p + 7, 0] = float("-inf")
+    kk[0, 0, n_p + 9, 1] = float("inf")
+    kk[0, 0, n_p + 9, 2] = float("-inf")
+    q[0, 1, n_p + 20] = float("nan")
+    ws = torch.zeros(plan.workspace_size(B, H, D, k), dtype=torch.uint8, device="cuda")
+    for slot, x in zip(vsa.pooled_slots(plan, ws, B, H, D), (q, kk, v)):
+        slot.copy_(x.cuda())
+    _, idx, _ = vsa.vsa_coarse_topk_pooled(plan, B, H, D, k, ws)
+    vsa.vsa_sync_status(plan)
+    got = idx.cpu().numpy().astype(np.int64)
+    assert np.all(np.diff(got, axis=-1) > 0) and got.min() >= n_p and got.max() < T
+    with np.errstate(invalid="ignore", over="ignore"):
+        s, _ = O.coarse_attention(q.double().numpy(), kk.double().numpy(), v.double().numpy(), D ** -0.5)
+    checked = 0
+    for h in range(H):
+        for i in range(n_p, T):
+            row = s[0, h, i]
+            if np.all(np.isfinite(row[n_p:])):
+                check_topk_row(got[0, h, i - n_p], row, n_p, k)
+                checked += 1
+    assert checked == T - n_p - 1        # head 1 without its NaN query row
+
+
 def test_keep_all_equals_dense_attention():
     """k = every video tile: the fine output is plain dense attention over all
     real tokens (torch's own routine, fp32 on the GPU)."""

@@ -13,9 +13,9 @@
 //      video key tiles (video query tiles only).  A histogram over the row's
 //      value range (256 equal-width bins of (s - min) * 256 / (max - min), a
 //      monotone map of s) finds the bin that holds the k-th largest score; its
-//      scores (at most 32, else the exact radix select below runs instead) are
-//      ranked against each other, which gives the k-th largest score K* and how
-//      many scores equal to K* to keep.  One ascending sweep then keeps every
+//      scores (at most 32; else, and for a row holding a NaN score, the exact
+//      radix select below runs instead) are ranked against each other, which
+//      gives the k-th largest score K* and how many scores equal to K* to keep.  One ascending sweep then keeps every
 //      score > K* and the lowest-index scores == K*, so the result is sorted by
 //      tile index with ties broken towards the lower index; bit-exact for given
 //      fp32 scores.  The fallback radix select runs four 8-bit digit passes
@@ -261,16 +261,21 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
         __syncwarp();
         s = buf;
       }
-      // row max over all T tiles; min and max over the video tiles
+      // row max over all T tiles; min and max over the video tiles, and
+      // whether one of them is NaN (the range histogram would bin it apart
+      // from where its order key ranks it, so such rows take the radix select)
       float m = -INFINITY, vlo = INFINITY, vhi = -INFINITY;
+      bool nan_seen = false;
       for (int j = lane; j < T; j += 32) {
         const float v = s[j];
         m = fmaxf(m, v);
         if (j >= n_p) {
           vlo = fminf(vlo, v);
           vhi = fmaxf(vhi, v);
+          nan_seen |= v != v;
         }
       }
+      const bool row_nan = __any_sync(0xFFFFFFFFu, nan_seen);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
@@ -284,7 +289,7 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
         bool found = false;
         const float range = vhi - vlo;
         const float bsc = 256.0f / range;
-        if (range > 0.0f && range < INFINITY && bsc < INFINITY) {
+        if (!row_nan && range > 0.0f && range < INFINITY && bsc < INFINITY) {
           // one histogram over the value range
 #pragma unroll
           for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
@@ -374,8 +379,10 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
           const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
           if (sel) {
             const int o = pos + __popc(selb & lt_mask);
-            out_idx[o] = j;
-            if (out_s) out_s[o] = sv;
+            if (o < k) {             // exactly k are selected; the bound only guards the row
+              out_idx[o] = j;
+              if (out_s) out_s[o] = sv;
+            }
           }
           pos += __popc(selb);
           eq_seen += __popc(eqb);
