@@ -30,6 +30,8 @@
  *     an index out of range) are recorded in the plan's device status word and
  *     reported by vsa_sync_status().
  *   - Supported: D in {64, 128}; R = tile_t*tile_h*tile_w in {64, 128}.
+ *   - Every call that launches work opens an NVTX range named after itself
+ *     (a no-op unless a profiler is attached).
  */
 #ifndef VSA_H_
 #define VSA_H_

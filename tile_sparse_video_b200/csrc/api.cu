@@ -185,6 +185,7 @@ vsa_status vsa_workspace_size(vsa_plan p, int B, int H, int D, int k, size_t* by
 }
 
 vsa_status vsa_permute(vsa_plan p, const void* x, void* x_t, int B, int H, int D, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (empty) return VSA_OK;
@@ -197,6 +198,7 @@ vsa_status vsa_permute(vsa_plan p, const void* x, void* x_t, int B, int H, int D
 }
 
 vsa_status vsa_unpermute(vsa_plan p, const void* x_t, void* x, int B, int H, int D, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (empty) return VSA_OK;
@@ -211,6 +213,7 @@ vsa_status vsa_unpermute(vsa_plan p, const void* x_t, void* x, int B, int H, int
 vsa_status vsa_coarse_topk(vsa_plan p, const void* q_t, const void* k_t, const void* v_t, int B,
                            int H, int D, float scale, int k, float* o_coarse, int32_t* topk_idx,
                            float* topk_score, void* ws, size_t ws_bytes, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   VSA_TRY(check_k(p, k));
@@ -248,6 +251,7 @@ vsa_status vsa_coarse_topk(vsa_plan p, const void* q_t, const void* k_t, const v
 
 vsa_status vsa_permute_pool(vsa_plan p, const void* x, void* x_t, int B, int H, int D,
                             float* pooled, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (empty) return VSA_OK;
@@ -264,6 +268,7 @@ vsa_status vsa_permute_pool(vsa_plan p, const void* x, void* x_t, int B, int H, 
 vsa_status vsa_coarse_topk_pooled(vsa_plan p, int B, int H, int D, float scale, int k,
                                   float* o_coarse, int32_t* topk_idx, float* topk_score, void* ws,
                                   size_t ws_bytes, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   VSA_TRY(check_k(p, k));
@@ -294,6 +299,7 @@ vsa_status vsa_coarse_topk_pooled(vsa_plan p, int B, int H, int D, float scale, 
 
 vsa_status vsa_project(vsa_plan p, const void* x, const void* w, int B, int H, int D, int C,
                        int act, void* y, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (C <= 0 || C % 8 != 0) return fail(VSA_ERR_INVALID_ARG, "C must be a positive multiple of 8");
@@ -307,6 +313,7 @@ vsa_status vsa_project(vsa_plan p, const void* x, const void* w, int B, int H, i
 
 vsa_status vsa_project_tiled(vsa_plan p, const void* x_t, const void* w, int B, int H, int D, int C,
                              int act, void* y_t, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (C <= 0 || C % 8 != 0) return fail(VSA_ERR_INVALID_ARG, "C must be a positive multiple of 8");
@@ -319,6 +326,7 @@ vsa_status vsa_project_tiled(vsa_plan p, const void* x_t, const void* w, int B, 
 }
 
 vsa_status vsa_permute_rows(vsa_plan p, const void* x, void* x_t, int B, int C, void* stream) {
+  VSA_NVTX_RANGE();
   if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
   if (p->device < 0) return fail(VSA_ERR_INVALID_ARG, "host-only plan (device = -1) cannot launch");
   if (B < 0) return fail(VSA_ERR_INVALID_ARG, "B must be >= 0");
@@ -340,6 +348,7 @@ vsa_status vsa_sparse_attn(vsa_plan p, const void* q_t, const void* k_t, const v
                            const int32_t* topk_idx, int B, int H, int D, int k, float scale,
                            void* o_fine_t, float* lse_t, void* ws, size_t ws_bytes,
                            void* stream) {
+  VSA_NVTX_RANGE();
   (void)ws;
   (void)ws_bytes;
   bool empty = false;
@@ -364,6 +373,7 @@ vsa_status vsa_sparse_attn_combine(vsa_plan p, const void* q_t, const void* k_t,
                                    const int32_t* topk_idx, int B, int H, int D, int k, float scale,
                                    const void* gate, const float* o_coarse, void* out,
                                    float* lse_t, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   VSA_TRY(check_k(p, k));
@@ -402,6 +412,7 @@ vsa_status vsa_keep_count_ref(vsa_plan p, double keep_ratio, int32_t keep_tiles,
 vsa_status vsa_select_reference(vsa_plan p, int B, int H, int D, float scale, int k_ref,
                                 int32_t* topk_ref_idx, const void* ws, size_t ws_bytes,
                                 void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (k_ref < 0 || k_ref > p->n_prefix_tiles)
@@ -428,6 +439,7 @@ vsa_status vsa_sparse_attn_ref(vsa_plan p, const void* q_t, const void* k_t, con
                                const int32_t* topk_idx, int k, const int32_t* topk_ref_idx,
                                int k_ref, int B, int H, int D, float scale, const void* gate,
                                const float* o_coarse, void* out, float* lse_t, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   const int n_p = p->n_prefix_tiles, n_v = p->n_tiles - p->n_prefix_tiles;
@@ -462,6 +474,7 @@ vsa_status vsa_sparse_attn_ref(vsa_plan p, const void* q_t, const void* k_t, con
 vsa_status vsa_gate_combine(vsa_plan p, const void* o_fine_t, const void* gate_t,
                             const float* o_coarse, void* out, int out_natural, int B, int H,
                             int D, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (empty) return VSA_OK;
@@ -490,6 +503,7 @@ vsa_status vsa_backward_workspace_size(vsa_plan p, int B, int H, int D, size_t* 
 vsa_status vsa_combine_backward(vsa_plan p, const void* d_out_t, const void* o_fine_t,
                                 const void* gate_t, const float* o_coarse, int B, int H, int D,
                                 float* delta, void* d_gate_t, float* d_o_coarse, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (empty) return VSA_OK;
@@ -510,6 +524,7 @@ vsa_status vsa_coarse_backward(vsa_plan p, const float* qbar, const float* kbar,
                                const float* d_o_coarse, int B, int H, int D, float scale,
                                float* d_qbar, float* d_kbar, float* d_vbar, void* ws,
                                size_t ws_bytes, void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   if (empty) return VSA_OK;
@@ -537,6 +552,7 @@ vsa_status vsa_sparse_attn_backward(vsa_plan p, const void* q_t, const void* k_t
                                     const float* d_vbar, int B, int H, int D, float scale,
                                     void* dq_t, void* dk_t, void* dv_t, void* ws, size_t ws_bytes,
                                     void* stream) {
+  VSA_NVTX_RANGE();
   bool empty = false;
   VSA_TRY(check_launch(p, B, H, D, &empty));
   const int n_p = p->n_prefix_tiles, n_v = p->n_tiles - p->n_prefix_tiles;
@@ -577,6 +593,7 @@ vsa_status vsa_sparse_attn_backward(vsa_plan p, const void* q_t, const void* k_t
 }
 
 vsa_status vsa_check_bounded_wait(vsa_plan p, int32_t* result, void* stream) {
+  VSA_NVTX_RANGE();
   if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
   if (p->device < 0) return fail(VSA_ERR_INVALID_ARG, "host-only plan (device = -1) cannot launch");
   VSA_TRY(check_ptr(result, "result"));
@@ -599,6 +616,7 @@ vsa_status vsa_debug_set_wait_limit(uint64_t ns) {
 }
 
 vsa_status vsa_sync_status(vsa_plan p, void* stream) {
+  VSA_NVTX_RANGE();
   if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
   if (p->device < 0) return VSA_OK;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

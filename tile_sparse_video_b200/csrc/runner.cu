@@ -127,6 +127,7 @@ vsa_status vsa_runner_create(vsa_plan p, int B, int H, int D, int k, float scale
 vsa_status vsa_runner_run(vsa_runner r, int n_layers, const void* const* q, const void* const* k_in,
                           const void* const* v, const void* const* g, void* const* out,
                           void* stream) {
+  VSA_NVTX_RANGE();
   if (r == nullptr) return vsa::fail(VSA_ERR_INVALID_ARG, "runner is NULL");
   if (n_layers < 0) return vsa::fail(VSA_ERR_INVALID_ARG, "n_layers < 0");
   if (n_layers == 0) return VSA_OK;

@@ -7,6 +7,7 @@
 #include <vector>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/vsa.h"
 
@@ -31,6 +32,18 @@ struct vsa_plan_s {
 };
 
 namespace vsa {
+
+// An NVTX range named after the entry point around each call that launches
+// work, so that a profiler's timeline (and ncu's --nvtx filters) show the
+// library's calls.  NVTX is header-only and does nothing unless a tool is
+// attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define VSA_NVTX_RANGE() ::vsa::NvtxRange vsa_nvtx_range_(__func__)
 
 // Bound of the attention kernels' mbarrier waits, in ns (2 s unless a test
 // shortened it through vsa_debug_set_wait_limit).
