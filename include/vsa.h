@@ -319,7 +319,9 @@ vsa_status vsa_runner_create(vsa_plan plan, int B, int H, int D, int k, float sc
  * copy-out; the call itself returns once everything is queued.  Kernel faults
  * are recorded in the plan's status word (vsa_sync_status).  Runs of one
  * runner must not overlap in time with each other, and nothing else may use
- * the plan's attention kernels concurrently. */
+ * the plan's attention kernels concurrently.  On an error return the layers
+ * queued before the failing call may still run; `stream` then does not wait
+ * for them, vsa_runner_destroy does. */
 vsa_status vsa_runner_run(vsa_runner runner, int n_layers, const void* const* q,
                           const void* const* k, const void* const* v, const void* const* g,
                           void* const* out, void* stream);
