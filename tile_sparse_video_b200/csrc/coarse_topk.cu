@@ -266,6 +266,7 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
       // from where its order key ranks it, so such rows take the radix select)
       float m = -INFINITY, vlo = INFINITY, vhi = -INFINITY;
       bool nan_seen = false;
+#pragma unroll 2
       for (int j = lane; j < T; j += 32) {
         const float v = s[j];
         m = fmaxf(m, v);
@@ -294,6 +295,7 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
 #pragma unroll
           for (int b = 0; b < 8; ++b) h[lane * 8 + b] = 0u;
           __syncwarp();
+#pragma unroll 2
           for (int j = n_p + lane; j < T; j += 32) atomicAdd(h + range_bin(s[j], vlo, bsc), 1u);
           __syncwarp();
           // lane L holds bins 255-8L .. 248-8L (lane 0 = highest scores)
@@ -327,6 +329,7 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
           if (in_bin <= 32) {
             // the scores of bin b*, compacted; the k-th largest is among them
             int base = 0;
+#pragma unroll 2
             for (int jb = n_p; jb < T; jb += 32) {
               const int j = jb + lane;
               const float v = j < T ? s[j] : 0.f;
@@ -366,6 +369,7 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
         int32_t* out_idx = topk_idx + ((bh * n_v) + (i - n_p)) * int64_t(k);
         float* out_s = topk_score ? topk_score + ((bh * n_v) + (i - n_p)) * int64_t(k) : nullptr;
         int pos = 0, eq_seen = 0;
+#pragma unroll 2
         for (int base = n_p; base < T; base += 32) {
           const int j = base + lane;
           const bool valid = j < T;
@@ -446,6 +450,7 @@ __global__ void __launch_bounds__(kWarps * 32, VSA_COARSE_CTAS) coarse_topk_kern
       __syncthreads();     // value chunk c landed, probability chunk c stored
       const float* pr = pc + rg * kPStride;
       const int nj4 = nj & ~3;
+#pragma unroll 4
       for (int jj = 0; jj < nj4; jj += 4) {
         float p[4][4];
 #pragma unroll
