@@ -175,8 +175,9 @@ __device__ __forceinline__ float ex2(float x) {
 #define VSA_EXP2_FMA_SHARE 0
 #endif
 // One exponential in kExp2FmaShare runs on the FMA pipe (0: all on MUFU).  On
-// B200 every share measured slower (the softmax is issue-bound, not MUFU-bound:
-// 27.6 ms with none, 28.6 / 30.7 / 31.6 ms with 1 in 8 / 4 / 2), so it is off.
+// B200 every share measured slower (27.6 ms with none, 28.6 / 30.7 / 31.6 ms
+// with 1 in 8 / 4 / 2 on an earlier kernel; 24.0 ms with none, 25.6 / 35.4 ms
+// with 1 in 16 / 8 on the current one), so it is off.
 constexpr int kExp2FmaShare = VSA_EXP2_FMA_SHARE;
 // The reference-max decision of a tile is published after this many of the
 // tile's 32-score exponential chunks (R/32 or more: after all of them), so
