@@ -105,6 +105,9 @@ vsa_status vsa_plan_tables(vsa_plan plan, int32_t* untile, int32_t* row_src,
  * rejected (VSA_ERR_INVALID_ARG): a query tile would have no key. */
 vsa_status vsa_keep_count(vsa_plan plan, double keep_ratio, int32_t keep_tiles, int32_t* k);
 
+/* Frees the plan's host and device tables and its status block (after a
+ * device synchronisation when the plan has a device).  The caller must not
+ * use the plan, nor any runner built on it, afterwards.  NULL is a no-op. */
 vsa_status vsa_plan_destroy(vsa_plan plan);
 
 /* Bytes of device workspace vsa_coarse_topk needs for B, H, D, k
